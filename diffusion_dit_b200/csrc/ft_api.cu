@@ -1,0 +1,433 @@
+// C ABI of the W4A4G4 triple-branch linear (declared in include/fourtune.h).
+// Host side only: argument checks, workspace carving, TMA descriptors, launch order.
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "fourtune.h"
+#include "ft_internal.h"
+
+namespace {
+
+using ft::GemmFp4Args;
+
+constexpr size_t kAlign = 256;
+
+size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+struct DeviceInfo {
+    int device = -1;
+    int num_sms = 0;
+    int cc_major = 0;
+};
+
+ft_status device_info(DeviceInfo* out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return FT_ERR_CUDA;
+    static std::mutex mu;
+    static DeviceInfo cache[64];
+    std::lock_guard<std::mutex> lock(mu);
+    if (dev < 0 || dev >= 64) return FT_ERR_CUDA;
+    if (cache[dev].device != dev) {
+        DeviceInfo d;
+        d.device = dev;
+        if (cudaDeviceGetAttribute(&d.num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            return FT_ERR_CUDA;
+        if (cudaDeviceGetAttribute(&d.cc_major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess)
+            return FT_ERR_CUDA;
+        cache[dev] = d;
+    }
+    *out = cache[dev];
+    if (out->cc_major != 10) return FT_ERR_UNSUPPORTED;
+    return FT_OK;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+// 2-D row-major tensor map with a 128-byte swizzle.
+ft_status make_tmap(CUtensorMap* map, const void* base, CUtensorMapDataType dt, uint64_t inner_elems,
+                    uint64_t rows, uint64_t row_bytes, uint32_t box_inner, uint32_t box_rows) {
+    auto fn = encode_fn();
+    if (!fn) return FT_ERR_CUDA;
+    cuuint64_t dims[2] = {inner_elems, rows};
+    cuuint64_t strides[1] = {row_bytes};
+    cuuint32_t box[2] = {box_inner, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(map, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? FT_OK : FT_ERR_CUDA;
+}
+
+ft_status cuda_status(cudaError_t e) { return e == cudaSuccess ? FT_OK : FT_ERR_CUDA; }
+
+#define FT_TRY(expr)                          \
+    do {                                      \
+        ft_status _s = (expr);                \
+        if (_s != FT_OK) return _s;           \
+    } while (0)
+#define FT_CUDA(expr) FT_TRY(cuda_status(expr))
+
+int low_rank_width(int R) { return R == 0 ? 0 : static_cast<int>(align_up(2 * static_cast<size_t>(R), 64)); }
+
+// Workspace of the layer calls.  Regions are 256-byte aligned.
+struct LinearWs {
+    size_t status, scal, qx_codes, qx_scales, qx_sf, dn, upcat, tcat;
+    size_t qg_codes, qg_scales, qg_sf, upt, dntcat, u, ucat, total;
+};
+
+LinearWs linear_ws(int64_t M, int64_t N, int64_t K, int R) {
+    const int KL = low_rank_width(R);
+    LinearWs w{};
+    size_t o = 0;
+    auto take = [&](size_t bytes) {
+        size_t at = o;
+        o = align_up(o + bytes, kAlign);
+        return at;
+    };
+    w.status = take(16);
+    w.scal = take(16 * sizeof(float));
+    w.qx_codes = take(static_cast<size_t>(M) * K / 2);
+    w.qx_scales = take(static_cast<size_t>(M) * K / 256);
+    w.qx_sf = take(static_cast<size_t>(M) * K / 16);
+    w.dn = take(static_cast<size_t>(R) * K * 2);
+    w.upcat = take(static_cast<size_t>(N) * KL * 2);
+    w.tcat = take(static_cast<size_t>(M) * KL * 2);
+    w.qg_codes = take(static_cast<size_t>(M) * N / 2);
+    w.qg_scales = take(static_cast<size_t>(M) * N / 256);
+    w.qg_sf = take(static_cast<size_t>(M) * N / 16);
+    w.upt = take(static_cast<size_t>(R) * N * 2);
+    w.dntcat = take(static_cast<size_t>(K) * KL * 2);
+    w.u = take(static_cast<size_t>(M) * R * 4);
+    w.ucat = take(static_cast<size_t>(M) * KL * 2);
+    w.total = o;
+    return w;
+}
+
+// scal[] slots
+enum { SC_AMAX_X = 0, SC_G_X = 1, SC_AMAX_G = 2, SC_G_G = 3 };
+
+ft_status check_fp4(const ft_fp4& q, int64_t rows, int64_t cols, bool need_sf) {
+    if (!q.codes || !q.scales || !q.g) return FT_ERR_INVALID_ARG;
+    if (need_sf && !q.sf_mma) return FT_ERR_INVALID_ARG;
+    if (q.rows != rows || q.cols != cols) return FT_ERR_SHAPE;
+    if (!aligned16(q.codes) || !aligned16(q.scales) || (q.sf_mma && !aligned16(q.sf_mma)) ||
+        (reinterpret_cast<uintptr_t>(q.g) & 3u))
+        return FT_ERR_ALIGN;
+    return FT_OK;
+}
+
+ft_status check_layer(const ft_linear* L) {
+    if (!L) return FT_ERR_INVALID_ARG;
+    if (L->N <= 0 || L->K <= 0 || L->r_s < 0 || L->r < 0) return FT_ERR_INVALID_ARG;
+    if (L->r_s + L->r > 256 || L->r > 64) return FT_ERR_SHAPE;
+    if (L->N % 256 || L->K % 256) return FT_ERR_SHAPE;
+    FT_TRY(check_fp4(L->qr, L->N, L->K, true));
+    FT_TRY(check_fp4(L->qr_t, L->K, L->N, true));
+    if (L->r_s > 0 && (!L->ls_down || !L->ls_up)) return FT_ERR_INVALID_ARG;
+    if (L->r > 0 && (!L->lora_a || !L->lora_b)) return FT_ERR_INVALID_ARG;
+    if ((L->ls_down && !aligned16(L->ls_down)) || (L->ls_up && !aligned16(L->ls_up)) ||
+        (L->lora_a && !aligned16(L->lora_a)) || (L->lora_b && !aligned16(L->lora_b)))
+        return FT_ERR_ALIGN;
+    return FT_OK;
+}
+
+const __nv_bfloat16* bf(const void* p) { return static_cast<const __nv_bfloat16*>(p); }
+__nv_bfloat16* bfm(void* p) { return static_cast<__nv_bfloat16*>(p); }
+
+// Quantize a bf16 [rows, cols] operand into (codes, scales, g, sf_mma) held in the workspace.
+ft_status quantize_operand(const void* x, int64_t rows, int64_t cols, const float* amax_or_null,
+                           float* amax_slot, uint8_t* codes, uint8_t* scales, uint8_t* sf, float* g,
+                           const DeviceInfo& dev, cudaStream_t st) {
+    const float* amax = amax_or_null;
+    if (!amax) {
+        FT_CUDA(ft::launch_amax(x, false, rows, cols, cols, amax_slot, dev.num_sms, st));
+        amax = amax_slot;
+    }
+    FT_CUDA(ft::launch_quant_block16(x, false, rows, cols, cols, amax, codes, scales, g, dev.num_sms, st));
+    FT_CUDA(ft::launch_expand_scales(scales, rows, cols, sf, st));
+    return FT_OK;
+}
+
+// One 4-bit GEMM with its low-rank tail: out[M, N] from A (M x K) and B (N x K).
+ft_status run_gemm(const uint8_t* a_codes, const uint8_t* a_sf, const float* ga, const ft_fp4& b,
+                   const __nv_bfloat16* la, const __nv_bfloat16* lb, int KL, int64_t M, int64_t N,
+                   int64_t K, void* out, int* status, const DeviceInfo& dev, cudaStream_t st) {
+    CUtensorMap tA, tB, tLA, tLB;
+    FT_TRY(make_tmap(&tA, a_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, K / 2, M, K / 2, 128, 128));
+    FT_TRY(make_tmap(&tB, b.codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, K / 2, N, K / 2, 128, 256));
+    if (KL > 0) {
+        FT_TRY(make_tmap(&tLA, la, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, KL, M, KL * 2, 64, 128));
+        FT_TRY(make_tmap(&tLB, lb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, KL, N, KL * 2, 64, 256));
+    } else {
+        tLA = tA;
+        tLB = tB;
+    }
+    GemmFp4Args g{};
+    g.sfa = a_sf;
+    g.sfb = b.sf_mma;
+    g.ga = ga;
+    g.gb = b.g;
+    g.out = bfm(out);
+    g.ldo = N;
+    g.M = static_cast<int>(M);
+    g.N = static_cast<int>(N);
+    g.K = static_cast<int>(K);
+    g.KL = KL;
+    g.status = status;
+    FT_CUDA(ft::launch_gemm_fp4_lowrank(tA, tB, tLA, tLB, g, dev.num_sms, st));
+    return FT_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* fourtune_status_string(int s) {
+    switch (s) {
+        case FT_OK: return "ok";
+        case FT_ERR_INVALID_ARG: return "invalid argument";
+        case FT_ERR_SHAPE: return "unsupported shape";
+        case FT_ERR_ALIGN: return "misaligned pointer";
+        case FT_ERR_WORKSPACE: return "workspace too small";
+        case FT_ERR_CUDA: return "CUDA error";
+        case FT_ERR_UNSUPPORTED: return "device is not sm_100";
+        case FT_ERR_TIMEOUT: return "device wait timed out";
+        default: return "unknown status";
+    }
+}
+
+size_t fourtune_quantize_workspace_bytes(int64_t rows, int64_t cols, int32_t r_down) {
+    (void)rows;
+    (void)cols;
+    (void)r_down;
+    return 2 * kAlign;  // status word + amax slot
+}
+
+ft_status fourtune_quantize_block16(const void* x_dev, int32_t x_dtype, int64_t rows, int64_t cols,
+                                    int64_t ld, const float* amax_or_null, const void* down_dev,
+                                    int32_t r_down, float* down_out_dev, const ft_fp4* out,
+                                    const ft_fp4* out_t, void* ws, size_t ws_bytes, void* stream) {
+    if (!x_dev || !out || (x_dtype != FT_DTYPE_BF16 && x_dtype != FT_DTYPE_F32)) return FT_ERR_INVALID_ARG;
+    if (rows <= 0 || cols <= 0 || ld < cols || r_down < 0 || r_down > 256) return FT_ERR_INVALID_ARG;
+    if (rows % 16 || cols % 16 || ld % 8) return FT_ERR_SHAPE;
+    if (r_down > 0 && (!down_dev || !down_out_dev || x_dtype != FT_DTYPE_BF16)) return FT_ERR_INVALID_ARG;
+    if (r_down > 0 && rows % 32) return FT_ERR_SHAPE;
+    FT_TRY(check_fp4(*out, rows, cols, false));
+    const bool want_sf = out->sf_mma != nullptr;
+    if ((want_sf || out_t) && (rows % 128 || cols % 128)) return FT_ERR_SHAPE;
+    if (out_t) FT_TRY(check_fp4(*out_t, cols, rows, true));
+    if (!aligned16(x_dev) || (down_dev && !aligned16(down_dev)) || (down_out_dev && !aligned16(down_out_dev)))
+        return FT_ERR_ALIGN;
+    if (!ws || ws_bytes < fourtune_quantize_workspace_bytes(rows, cols, r_down)) return FT_ERR_WORKSPACE;
+    if (reinterpret_cast<uintptr_t>(ws) % kAlign) return FT_ERR_ALIGN;
+    DeviceInfo dev;
+    FT_TRY(device_info(&dev));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    float* amax_slot = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + kAlign);
+    const bool f32 = x_dtype == FT_DTYPE_F32;
+    const float* amax = amax_or_null;
+    if (!amax) {
+        FT_CUDA(ft::launch_amax(x_dev, f32, rows, cols, ld, amax_slot, dev.num_sms, st));
+        amax = amax_slot;
+    }
+    FT_CUDA(ft::launch_quant_block16(x_dev, f32, rows, cols, ld, amax, out->codes, out->scales, out->g,
+                                     dev.num_sms, st));
+    if (want_sf) FT_CUDA(ft::launch_expand_scales(out->scales, rows, cols, out->sf_mma, st));
+    if (out_t) {
+        FT_CUDA(ft::launch_transpose_q(out->codes, out->scales, rows, cols, out_t->codes, out_t->scales, st));
+        FT_CUDA(ft::launch_copy_scalar(out->g, out_t->g, st));
+        FT_CUDA(ft::launch_expand_scales(out_t->scales, cols, rows, out_t->sf_mma, st));
+    }
+    if (r_down > 0) {
+        // the down-projection alone: out = x down^T (fp32); its bf16 split is not needed
+        ft::LowRankDownArgs a{};
+        a.x = bf(x_dev);
+        a.ldx = ld;
+        a.M = rows;
+        a.K = cols;
+        a.w = bf(down_dev);
+        a.R = r_down;
+        a.r_s = r_down;
+        a.s = 1.0f;
+        a.ga = nullptr;
+        a.gb = nullptr;
+        a.out = down_out_dev;
+        a.cat = nullptr;
+        a.KL = 0;
+        FT_CUDA(ft::launch_lowrank_down(a, st));
+    }
+    return FT_OK;
+}
+
+size_t fourtune_linear_workspace_bytes(const ft_linear* L, int64_t M) {
+    if (!L || M <= 0) return 0;
+    return linear_ws(M, L->N, L->K, L->r_s + L->r).total;
+}
+
+ft_status fourtune_linear_fwd(const ft_linear* L, const void* x_dev, int64_t M, const float* amax_or_null,
+                              void* y_dev, float* t_saved_dev, void* ws, size_t ws_bytes, void* stream) {
+    FT_TRY(check_layer(L));
+    const int R = L->r_s + L->r;
+    if (!x_dev || !y_dev || (R > 0 && !t_saved_dev) || M <= 0) return FT_ERR_INVALID_ARG;
+    if (M % 128) return FT_ERR_SHAPE;
+    if (!aligned16(x_dev) || !aligned16(y_dev) || (t_saved_dev && !aligned16(t_saved_dev))) return FT_ERR_ALIGN;
+    const LinearWs w = linear_ws(M, L->N, L->K, R);
+    if (!ws || ws_bytes < w.total) return FT_ERR_WORKSPACE;
+    if (reinterpret_cast<uintptr_t>(ws) % kAlign) return FT_ERR_ALIGN;
+    DeviceInfo dev;
+    FT_TRY(device_info(&dev));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    uint8_t* W = static_cast<uint8_t*>(ws);
+    float* scal = reinterpret_cast<float*>(W + w.scal);
+    int* status = reinterpret_cast<int*>(W + w.status);
+    const int64_t N = L->N, K = L->K;
+    const int KL = low_rank_width(R);
+
+    FT_TRY(quantize_operand(x_dev, M, K, amax_or_null, scal + SC_AMAX_X, W + w.qx_codes, W + w.qx_scales,
+                            W + w.qx_sf, scal + SC_G_X, dev, st));
+    if (R > 0) {
+        FT_CUDA(ft::launch_build_factors(bf(L->ls_down), bf(L->lora_a), bf(L->ls_up), bf(L->lora_b), N, K,
+                                         L->r_s, L->r, KL, bfm(W + w.dn), bfm(W + w.upcat), nullptr, nullptr,
+                                         st));
+        ft::LowRankDownArgs a{};
+        a.x = bf(x_dev);
+        a.ldx = K;
+        a.M = M;
+        a.K = K;
+        a.w = bf(W + w.dn);
+        a.R = R;
+        a.r_s = L->r_s;
+        a.s = L->lora_scale;
+        a.ga = scal + SC_G_X;
+        a.gb = L->qr.g;
+        a.out = t_saved_dev;
+        a.cat = bfm(W + w.tcat);
+        a.KL = KL;
+        FT_CUDA(ft::launch_lowrank_down(a, st));
+    }
+    return run_gemm(W + w.qx_codes, W + w.qx_sf, scal + SC_G_X, L->qr, bf(W + w.tcat), bf(W + w.upcat), KL, M,
+                    N, K, y_dev, status, dev, st);
+}
+
+ft_status fourtune_linear_bwd(const ft_linear* L, const void* x_dev, const float* t_saved_dev,
+                              const void* dy_dev, int64_t M, const float* amax_or_null, void* dx_dev,
+                              float* da_dev, float* db_dev, void* ws, size_t ws_bytes, void* stream) {
+    FT_TRY(check_layer(L));
+    const int R = L->r_s + L->r;
+    if (!x_dev || !dy_dev || !dx_dev || M <= 0) return FT_ERR_INVALID_ARG;
+    if (L->r > 0 && (!t_saved_dev || !da_dev || !db_dev)) return FT_ERR_INVALID_ARG;
+    if (M % 128) return FT_ERR_SHAPE;
+    if (!aligned16(x_dev) || !aligned16(dy_dev) || !aligned16(dx_dev) ||
+        (t_saved_dev && !aligned16(t_saved_dev)) || (da_dev && !aligned16(da_dev)) ||
+        (db_dev && !aligned16(db_dev)))
+        return FT_ERR_ALIGN;
+    const LinearWs w = linear_ws(M, L->N, L->K, R);
+    if (!ws || ws_bytes < w.total) return FT_ERR_WORKSPACE;
+    if (reinterpret_cast<uintptr_t>(ws) % kAlign) return FT_ERR_ALIGN;
+    DeviceInfo dev;
+    FT_TRY(device_info(&dev));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    uint8_t* W = static_cast<uint8_t*>(ws);
+    float* scal = reinterpret_cast<float*>(W + w.scal);
+    int* status = reinterpret_cast<int*>(W + w.status);
+    const int64_t N = L->N, K = L->K;
+    const int KL = low_rank_width(R);
+
+    FT_TRY(quantize_operand(dy_dev, M, N, amax_or_null, scal + SC_AMAX_G, W + w.qg_codes, W + w.qg_scales,
+                            W + w.qg_sf, scal + SC_G_G, dev, st));
+    float* U = reinterpret_cast<float*>(W + w.u);
+    if (R > 0) {
+        FT_CUDA(ft::launch_build_factors(bf(L->ls_down), bf(L->lora_a), bf(L->ls_up), bf(L->lora_b), N, K,
+                                         L->r_s, L->r, KL, nullptr, nullptr, bfm(W + w.upt),
+                                         bfm(W + w.dntcat), st));
+        ft::LowRankDownArgs a{};
+        a.x = bf(dy_dev);
+        a.ldx = N;
+        a.M = M;
+        a.K = N;
+        a.w = bf(W + w.upt);
+        a.R = R;
+        a.r_s = L->r_s;
+        a.s = L->lora_scale;
+        a.ga = scal + SC_G_G;
+        a.gb = L->qr_t.g;
+        a.out = U;
+        a.cat = bfm(W + w.ucat);
+        a.KL = KL;
+        FT_CUDA(ft::launch_lowrank_down(a, st));
+    }
+    FT_TRY(run_gemm(W + w.qg_codes, W + w.qg_sf, scal + SC_G_G, L->qr_t, bf(W + w.ucat), bf(W + w.dntcat), KL,
+                    M, K, N, dx_dev, status, dev, st));
+    if (L->r > 0) {
+        FT_CUDA(ft::launch_lora_db(bf(dy_dev), M, N, t_saved_dev, R, L->r_s, L->r, L->lora_scale, db_dev, st));
+        FT_CUDA(ft::launch_lora_da(U, R, L->r_s, L->r, bf(x_dev), M, K, L->lora_scale, da_dev, st));
+    }
+    return FT_OK;
+}
+
+ft_status fourtune_device_status(void* ws, int32_t* status_out, void* stream) {
+    if (!ws || !status_out) return FT_ERR_INVALID_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    int32_t v = 0;
+    FT_CUDA(cudaMemcpyAsync(&v, ws, sizeof(int32_t), cudaMemcpyDeviceToHost, st));
+    FT_CUDA(cudaStreamSynchronize(st));
+    FT_CUDA(cudaMemsetAsync(ws, 0, sizeof(int32_t), st));
+    *status_out = v;
+    return FT_OK;
+}
+
+ft_status fourtune_gelu_tanh_fwd(const void* p_dev, void* h_dev, int64_t n, void* stream) {
+    if (!p_dev || !h_dev || n < 0) return FT_ERR_INVALID_ARG;
+    if (n % 8) return FT_ERR_SHAPE;
+    if (!aligned16(p_dev) || !aligned16(h_dev)) return FT_ERR_ALIGN;
+    if (n == 0) return FT_OK;
+    DeviceInfo dev;
+    FT_TRY(device_info(&dev));
+    FT_CUDA(ft::launch_gelu_fwd(bf(p_dev), bfm(h_dev), n, static_cast<cudaStream_t>(stream)));
+    return FT_OK;
+}
+
+ft_status fourtune_gelu_tanh_bwd(const void* p_dev, const void* dh_dev, void* dp_dev, int64_t n, void* stream) {
+    if (!p_dev || !dh_dev || !dp_dev || n < 0) return FT_ERR_INVALID_ARG;
+    if (n % 8) return FT_ERR_SHAPE;
+    if (!aligned16(p_dev) || !aligned16(dh_dev) || !aligned16(dp_dev)) return FT_ERR_ALIGN;
+    if (n == 0) return FT_OK;
+    DeviceInfo dev;
+    FT_TRY(device_info(&dev));
+    FT_CUDA(ft::launch_gelu_bwd(bf(p_dev), bf(dh_dev), bfm(dp_dev), n, static_cast<cudaStream_t>(stream)));
+    return FT_OK;
+}
+
+ft_status fourtune_encode_e2m1(const float* v_dev, int64_t n, uint8_t* out_dev, void* stream) {
+    if (!v_dev || !out_dev || n < 0) return FT_ERR_INVALID_ARG;
+    if (n == 0) return FT_OK;
+    DeviceInfo dev;
+    FT_TRY(device_info(&dev));
+    FT_CUDA(ft::launch_encode_e2m1(v_dev, n, out_dev, static_cast<cudaStream_t>(stream)));
+    return FT_OK;
+}
+
+ft_status fourtune_encode_ue4m3(const float* v_dev, int64_t n, uint8_t* out_dev, void* stream) {
+    if (!v_dev || !out_dev || n < 0) return FT_ERR_INVALID_ARG;
+    if (n == 0) return FT_OK;
+    DeviceInfo dev;
+    FT_TRY(device_info(&dev));
+    FT_CUDA(ft::launch_encode_ue4m3(v_dev, n, out_dev, static_cast<cudaStream_t>(stream)));
+    return FT_OK;
+}
+
+}  // extern "C"

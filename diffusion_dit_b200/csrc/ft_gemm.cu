@@ -1,0 +1,276 @@
+// Block-scaled FP4 GEMM with the low-rank branches added in the same accumulator.
+//
+//   OUT[M, N] = bf16( ( sum_k a(m,k) sfa(m,k/16) * b(n,k) sfb(n,k/16)        (E2M1 x E2M1)
+//                      + sum_j LA(m, j) LB(n, j) ) * 1/(g_a g_b) )            (bf16 x bf16)
+//
+// FourTune (arXiv 2607.05711), Eq. (2) forward: a = Q(X), b = Q(R), and the low-rank
+// operands carry X [Ls_down; A]^T and [Ls_up, B] (section 3.3 "LoRA Fusion": the up-
+// projections are fused into the 4-bit GEMM).  Eq. (3) backward: a = Q(G), b = Q(R)^T,
+// low-rank operands G [Ls_up, B] and [Ls_down; A]^T.  The caller pre-multiplies the
+// low-rank A operand by g_a g_b and splits it into a bf16 high and low part (both
+// multiplied by the same B operand), so the branch keeps ~16 mantissa bits.
+//
+// B200 design: persistent CTAs (one per SM), 128x256 output tile per CTA, a 4-stage
+// shared-memory ring fed by TMA (128-byte swizzle), tcgen05.mma with the fp32
+// accumulator in tensor memory, scale factors copied smem -> TMEM with tcgen05.cp, and
+// an epilogue that drains TMEM into registers before storing so the next tile's MMAs
+// start while the stores are still in flight.
+//
+// Warp roles (192 threads): warp 0 = TMA producer, warp 1 = MMA issuer (and TMEM
+// owner), warps 2..5 = epilogue (warp w reads TMEM lanes 32 (w % 4) .. +31).
+#include "ft_internal.h"
+#include "ft_ptx.cuh"
+
+namespace ft {
+namespace gemm {
+
+constexpr int BM = 128;
+constexpr int BN = 256;
+constexpr int BK_BYTES = 128;            // one 128-byte swizzle row: 256 fp4 or 64 bf16
+constexpr int STAGES = 4;
+constexpr int A_BYTES = BM * BK_BYTES;   // 16 KB
+constexpr int B_BYTES = BN * BK_BYTES;   // 32 KB
+constexpr int SFA_BYTES = 4 * 512;       // 4 k-blocks of 64 x 128 rows
+constexpr int SFB_BYTES = 2 * 4 * 512;   // 2 row bands of 128
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;  // 55296
+constexpr int OFF_B = A_BYTES;
+constexpr int OFF_SFA = A_BYTES + B_BYTES;
+constexpr int OFF_SFB = OFF_SFA + SFA_BYTES;
+constexpr int BAR_BYTES = 256;
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + BAR_BYTES + 1024;  // + alignment slack
+constexpr int THREADS = 192;
+
+// Tensor memory columns: accumulator [0,256), scale slots per stage after it.
+constexpr uint32_t TMEM_COLS = 512;
+constexpr uint32_t COL_ACC = 0;
+constexpr uint32_t COL_SFA = 256;  // 4 stages x 16 columns
+constexpr uint32_t COL_SFB = 320;  // 4 stages x 32 columns
+
+static_assert(STAGE_BYTES % 1024 == 0, "stage must keep 1024-byte alignment");
+static_assert(SMEM_BYTES <= 232448, "exceeds 227 KB of dynamic shared memory");
+
+struct Smem {
+    uint8_t* base;    // 1024-aligned
+    uint32_t base_u32;
+    __device__ uint32_t stage(int s) const { return base_u32 + s * STAGE_BYTES; }
+    __device__ uint32_t bar(int i) const { return base_u32 + STAGES * STAGE_BYTES + 8 * i; }
+};
+// barrier indices
+__host__ __device__ constexpr int BAR_FULL(int s) { return s; }
+__host__ __device__ constexpr int BAR_EMPTY(int s) { return STAGES + s; }
+constexpr int BAR_TMEM_FULL = 2 * STAGES;
+constexpr int BAR_TMEM_EMPTY = 2 * STAGES + 1;
+constexpr int BAR_FINAL = 2 * STAGES + 2;
+constexpr int NUM_BARS = 2 * STAGES + 3;
+constexpr int OFF_TMEM_SLOT = 8 * 16;   // inside the barrier area
+constexpr int OFF_ABORT = 8 * 16 + 4;
+
+__global__ void __launch_bounds__(THREADS, 1)
+    gemm_fp4_lowrank_kernel(const __grid_constant__ CUtensorMap tmA,
+                            const __grid_constant__ CUtensorMap tmB,
+                            const __grid_constant__ CUtensorMap tmLA,
+                            const __grid_constant__ CUtensorMap tmLB, const GemmFp4Args p) {
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw_u32 = smem_u32(smem_raw);
+    const uint32_t pad = (1024 - (raw_u32 & 1023)) & 1023;
+    Smem sm{smem_raw + pad, raw_u32 + pad};
+    uint8_t* bar_area = sm.base + STAGES * STAGE_BYTES;
+    volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(bar_area + OFF_TMEM_SLOT);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(bar_area + OFF_ABORT);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int MB = p.M / BM;
+    const int NB = p.N / BN;
+    const int num_tiles = MB * NB;
+    const int KT = p.K / 256;      // fp4 stages
+    const int KLS = p.KL / 64;     // low-rank stages
+    const int k64 = p.K / 64;      // scale atoms per 128-row band
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < STAGES; ++i) {
+            mbar_init(sm.bar(BAR_FULL(i)), 1);
+            mbar_init(sm.bar(BAR_EMPTY(i)), 1);
+        }
+        mbar_init(sm.bar(BAR_TMEM_FULL), 1);
+        mbar_init(sm.bar(BAR_TMEM_EMPTY), 4);
+        mbar_init(sm.bar(BAR_FINAL), 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+        fence_proxy_async_smem();
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&tmA);
+        tma_prefetch_desc(&tmB);
+        if (KLS > 0) {
+            tma_prefetch_desc(&tmLA);
+            tma_prefetch_desc(&tmLB);
+        }
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_u32(const_cast<uint32_t*>(tmem_slot)), TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0) {
+            int it = 0;
+            for (int t = blockIdx.x; t < num_tiles && !*abort_flag; t += gridDim.x) {
+                const int mb = t % MB, nb = t / MB;
+                const int m0 = mb * BM, n0 = nb * BN;
+                for (int kt = 0; kt < KT; ++kt, ++it) {
+                    const int s = it % STAGES;
+                    const uint32_t ph = (it / STAGES) & 1;
+                    if (!mbar_wait(sm.bar(BAR_EMPTY(s)), ph ^ 1, abort_flag, p.status)) break;
+                    const uint32_t full = sm.bar(BAR_FULL(s));
+                    const uint32_t st = sm.stage(s);
+                    mbar_arrive_expect_tx(full, STAGE_BYTES);
+                    tma_load_2d(st, &tmA, full, kt * BK_BYTES, m0);
+                    tma_load_2d(st + OFF_B, &tmB, full, kt * BK_BYTES, n0);
+                    bulk_load(st + OFF_SFA, p.sfa + (static_cast<size_t>(mb) * k64 + kt * 4) * 512,
+                              SFA_BYTES, full);
+#pragma unroll
+                    for (int rb = 0; rb < 2; ++rb)
+                        bulk_load(st + OFF_SFB + rb * 2048,
+                                  p.sfb + (static_cast<size_t>(nb * 2 + rb) * k64 + kt * 4) * 512,
+                                  2048, full);
+                }
+                if (*abort_flag) break;
+                for (int kl = 0; kl < KLS; ++kl, ++it) {
+                    const int s = it % STAGES;
+                    const uint32_t ph = (it / STAGES) & 1;
+                    if (!mbar_wait(sm.bar(BAR_EMPTY(s)), ph ^ 1, abort_flag, p.status)) break;
+                    const uint32_t full = sm.bar(BAR_FULL(s));
+                    const uint32_t st = sm.stage(s);
+                    mbar_arrive_expect_tx(full, A_BYTES + B_BYTES);
+                    tma_load_2d(st, &tmLA, full, kl * 64, m0);
+                    tma_load_2d(st + OFF_B, &tmLB, full, kl * 64, n0);
+                }
+            }
+            // Drain: every copy this thread issued has landed before the CTA may exit.
+            // (Already true on the normal path; on an abort it bounds the wait.)
+            for (int j = it - 1; j >= 0 && j >= it - STAGES; --j) {
+                volatile int no_abort = 0;
+                mbar_wait(sm.bar(BAR_FULL(j % STAGES)), (j / STAGES) & 1, &no_abort, p.status);
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            const uint32_t idesc4 = idesc_fp4_block16(BM, BN);
+            const uint32_t idesc16 = idesc_bf16(BM, BN);
+            int it = 0, ti = 0;
+            for (int t = blockIdx.x; t < num_tiles && !*abort_flag; t += gridDim.x, ++ti) {
+                if (!mbar_wait(sm.bar(BAR_TMEM_EMPTY), (ti & 1) ^ 1, abort_flag, p.status)) break;
+                tc_fence_after();
+                const uint32_t acc = tmem + COL_ACC;
+                bool ok = true;
+                for (int kt = 0; kt < KT; ++kt, ++it) {
+                    const int s = it % STAGES;
+                    const uint32_t ph = (it / STAGES) & 1;
+                    if (!mbar_wait(sm.bar(BAR_FULL(s)), ph, abort_flag, p.status)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t st = sm.stage(s);
+                    const uint32_t sfa_t = tmem + COL_SFA + 16 * s;
+                    const uint32_t sfb_t = tmem + COL_SFB + 32 * s;
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        tmem_cp_32x128b_x4(sfa_t + 4 * i, sdesc_scale_32x16(st + OFF_SFA + 512 * i));
+#pragma unroll
+                        for (int rb = 0; rb < 2; ++rb)
+                            tmem_cp_32x128b_x4(sfb_t + 8 * i + 4 * rb,
+                                               sdesc_scale_32x16(st + OFF_SFB + rb * 2048 + 512 * i));
+                    }
+                    const uint64_t ad = sdesc_kmajor_sw128(st);
+                    const uint64_t bd = sdesc_kmajor_sw128(st + OFF_B);
+#pragma unroll
+                    for (int i = 0; i < 4; ++i)
+                        mma_fp4_block16(acc, ad + 2 * i, bd + 2 * i, idesc4, sfa_t + 4 * i,
+                                        sfb_t + 8 * i, (kt | i) != 0);
+                    tc_commit(sm.bar(BAR_EMPTY(s)));
+                }
+                if (!ok) break;
+                for (int kl = 0; kl < KLS; ++kl, ++it) {
+                    const int s = it % STAGES;
+                    const uint32_t ph = (it / STAGES) & 1;
+                    if (!mbar_wait(sm.bar(BAR_FULL(s)), ph, abort_flag, p.status)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t st = sm.stage(s);
+                    const uint64_t ad = sdesc_kmajor_sw128(st);
+                    const uint64_t bd = sdesc_kmajor_sw128(st + OFF_B);
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) mma_bf16(acc, ad + 2 * i, bd + 2 * i, idesc16, 1);
+                    tc_commit(sm.bar(BAR_EMPTY(s)));
+                }
+                if (!ok) break;
+                tc_commit(sm.bar(BAR_TMEM_FULL));
+            }
+            // Every MMA issued by this thread has retired before TMEM is released.
+            tc_commit(sm.bar(BAR_FINAL));
+            volatile int no_abort = 0;
+            mbar_wait(sm.bar(BAR_FINAL), 0, &no_abort, p.status);
+        }
+    } else {
+        // ------------------------------------------------------------ epilogue
+        const int q = warp & 3;  // TMEM lane quarter this warp may access
+        const float ga = *p.ga, gb = *p.gb;
+        const float c = 1.0f / (ga * gb);
+        int ti = 0;
+        for (int t = blockIdx.x; t < num_tiles && !*abort_flag; t += gridDim.x, ++ti) {
+            const int mb = t % MB, nb = t / MB;
+            if (!mbar_wait(sm.bar(BAR_TMEM_FULL), ti & 1, abort_flag, p.status)) break;
+            tc_fence_after();
+            uint32_t pk[BN / 2];
+            const uint32_t lane_addr = tmem + COL_ACC + (static_cast<uint32_t>(32 * q) << 16);
+#pragma unroll
+            for (int ch = 0; ch < BN / 32; ++ch) {
+                uint32_t v[32];
+                tmem_ld_32x32b_x32(lane_addr + ch * 32, v);
+                tmem_ld_wait();
+#pragma unroll
+                for (int j = 0; j < 16; ++j)
+                    pk[ch * 16 + j] = pack_bf16x2(__uint_as_float(v[2 * j]) * c,
+                                                  __uint_as_float(v[2 * j + 1]) * c);
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(sm.bar(BAR_TMEM_EMPTY));
+            const int row = mb * BM + 32 * q + lane;
+            uint4* dst = reinterpret_cast<uint4*>(p.out + static_cast<size_t>(row) * p.ldo + nb * BN);
+#pragma unroll
+            for (int j = 0; j < BN / 8; ++j)
+                dst[j] = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tmem, TMEM_COLS);
+}
+
+}  // namespace gemm
+
+cudaError_t launch_gemm_fp4_lowrank(const CUtensorMap& tmA, const CUtensorMap& tmB,
+                                    const CUtensorMap& tmLA, const CUtensorMap& tmLB,
+                                    const GemmFp4Args& args, int num_sms, cudaStream_t stream) {
+    using namespace gemm;
+    static bool attr_set = false;
+    if (!attr_set) {
+        cudaError_t e = cudaFuncSetAttribute(gemm_fp4_lowrank_kernel,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+        if (e != cudaSuccess) return e;
+        attr_set = true;
+    }
+    const int tiles = (args.M / BM) * (args.N / BN);
+    const int grid = tiles < num_sms ? tiles : num_sms;
+    gemm_fp4_lowrank_kernel<<<grid, THREADS, SMEM_BYTES, stream>>>(tmA, tmB, tmLA, tmLB, args);
+    return cudaGetLastError();
+}
+
+}  // namespace ft

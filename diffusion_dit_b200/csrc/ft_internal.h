@@ -1,0 +1,73 @@
+// Host-side declarations shared by the library's translation units (not public).
+#pragma once
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace ft {
+
+struct GemmFp4Args {
+    const uint8_t* sfa;     // tensor-core scale layout of A (rows M, cols K)
+    const uint8_t* sfb;     // tensor-core scale layout of B (rows N, cols K)
+    const float* ga;        // tensor factor of A
+    const float* gb;        // tensor factor of B
+    __nv_bfloat16* out;     // [M, ldo]
+    int64_t ldo;
+    int M, N, K;            // K: reduction length in elements (multiple of 256)
+    int KL;                 // low-rank reduction length in bf16 elements (multiple of 64), 0 = none
+    int* status;            // device status word
+};
+
+cudaError_t launch_gemm_fp4_lowrank(const CUtensorMap& tmA, const CUtensorMap& tmB,
+                                    const CUtensorMap& tmLA, const CUtensorMap& tmLB,
+                                    const GemmFp4Args& args, int num_sms, cudaStream_t stream);
+
+// quantizer and helpers (ft_quant.cu)
+cudaError_t launch_amax(const void* x, bool is_f32, int64_t rows, int64_t cols, int64_t ld,
+                        float* amax_out, int num_sms, cudaStream_t stream);
+cudaError_t launch_quant_block16(const void* x, bool is_f32, int64_t rows, int64_t cols, int64_t ld,
+                                 const float* amax, uint8_t* codes, uint8_t* scales, float* g_out,
+                                 int num_sms, cudaStream_t stream);
+cudaError_t launch_expand_scales(const uint8_t* scales, int64_t rows, int64_t cols, uint8_t* sf_mma,
+                                 cudaStream_t stream);
+cudaError_t launch_transpose_q(const uint8_t* codes, const uint8_t* scales, int64_t rows, int64_t cols,
+                               uint8_t* codes_t, uint8_t* scales_t, cudaStream_t stream);
+cudaError_t launch_copy_scalar(const float* src, float* dst, cudaStream_t stream);
+cudaError_t launch_encode_e2m1(const float* v, int64_t n, uint8_t* out, cudaStream_t stream);
+cudaError_t launch_encode_ue4m3(const float* v, int64_t n, uint8_t* out, cudaStream_t stream);
+cudaError_t launch_gelu_fwd(const __nv_bfloat16* p, __nv_bfloat16* h, int64_t n, cudaStream_t stream);
+cudaError_t launch_gelu_bwd(const __nv_bfloat16* p, const __nv_bfloat16* dh, __nv_bfloat16* dp,
+                            int64_t n, cudaStream_t stream);
+
+// low-rank branches (ft_lowrank.cu)
+struct LowRankDownArgs {
+    const __nv_bfloat16* x;  // [M, ldx], reduction over K columns
+    int64_t ldx;
+    int64_t M, K;
+    const __nv_bfloat16* w;  // [R, K] down factor (rows = output columns)
+    int R, r_s;              // columns >= r_s are scaled by `s` before the split
+    float s;
+    const float* ga;         // g of the quantized operand of the following GEMM
+    const float* gb;
+    float* out;              // fp32 [M, R] unscaled product (may be null)
+    __nv_bfloat16* cat;      // bf16 [M, KL]: hi(g v'), lo(g v'), zeros
+    int KL;
+};
+cudaError_t launch_lowrank_down(const LowRankDownArgs& a, cudaStream_t stream);
+
+// Build the concatenated low-rank factors used by the forward and backward GEMMs.
+cudaError_t launch_build_factors(const __nv_bfloat16* ls_down, const __nv_bfloat16* lora_a,
+                                 const __nv_bfloat16* ls_up, const __nv_bfloat16* lora_b, int64_t N,
+                                 int64_t K, int r_s, int r, int KL, __nv_bfloat16* dn,
+                                 __nv_bfloat16* upcat, __nv_bfloat16* upt, __nv_bfloat16* dntcat,
+                                 cudaStream_t stream);
+
+// adapter gradients (ft_lowrank.cu)
+cudaError_t launch_lora_db(const __nv_bfloat16* g, int64_t M, int64_t N, const float* t, int R,
+                           int r_s, int r, float s, float* db, cudaStream_t stream);
+cudaError_t launch_lora_da(const float* u, int R, int r_s, int r, const __nv_bfloat16* x, int64_t M,
+                           int64_t K, float s, float* da, cudaStream_t stream);
+
+}  // namespace ft

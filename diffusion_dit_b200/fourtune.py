@@ -1,0 +1,299 @@
+"""Python binding of the C ABI in include/fourtune.h (argument marshalling only).
+
+Every step of the layer runs in the CUDA library ``_lib/libfourtune.so``; this module
+allocates device tensors with PyTorch, passes raw pointers and the current stream,
+and raises on any non-OK status.  There is no fallback: if the library is missing or
+the device is not sm_100 the calls fail loudly.
+"""
+from __future__ import annotations
+
+import ctypes
+import dataclasses
+import os
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "_lib", "libfourtune.so")
+
+FT_DTYPE_BF16 = 0
+FT_DTYPE_F32 = 1
+
+STATUS = {0: "FT_OK", 1: "FT_ERR_INVALID_ARG", 2: "FT_ERR_SHAPE", 3: "FT_ERR_ALIGN",
+          4: "FT_ERR_WORKSPACE", 5: "FT_ERR_CUDA", 6: "FT_ERR_UNSUPPORTED", 7: "FT_ERR_TIMEOUT"}
+
+
+class FourTuneError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        super().__init__(f"{fn} failed: {STATUS.get(status, status)}")
+        self.status = status
+
+
+class FtFp4(ctypes.Structure):
+    _fields_ = [("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p), ("sf_mma", ctypes.c_void_p),
+                ("g", ctypes.c_void_p), ("rows", ctypes.c_int64), ("cols", ctypes.c_int64)]
+
+
+class FtLinear(ctypes.Structure):
+    _fields_ = [("N", ctypes.c_int64), ("K", ctypes.c_int64), ("r_s", ctypes.c_int32),
+                ("r", ctypes.c_int32), ("lora_scale", ctypes.c_float), ("qr", FtFp4),
+                ("qr_t", FtFp4), ("ls_down", ctypes.c_void_p), ("ls_up", ctypes.c_void_p),
+                ("lora_a", ctypes.c_void_p), ("lora_b", ctypes.c_void_p)]
+
+
+EXPORTS = {
+    # name: (argtypes, restype)
+    "fourtune_status_string": ([ctypes.c_int], ctypes.c_char_p),
+    "fourtune_quantize_workspace_bytes": ([ctypes.c_int64, ctypes.c_int64, ctypes.c_int32], ctypes.c_size_t),
+    "fourtune_quantize_block16": ([ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_int64,
+                                   ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int32,
+                                   ctypes.c_void_p, ctypes.POINTER(FtFp4), ctypes.POINTER(FtFp4),
+                                   ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p], ctypes.c_int),
+    "fourtune_linear_workspace_bytes": ([ctypes.POINTER(FtLinear), ctypes.c_int64], ctypes.c_size_t),
+    "fourtune_linear_fwd": ([ctypes.POINTER(FtLinear), ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p,
+                             ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t,
+                             ctypes.c_void_p], ctypes.c_int),
+    "fourtune_linear_bwd": ([ctypes.POINTER(FtLinear), ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                             ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                             ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p],
+                            ctypes.c_int),
+    "fourtune_device_status": ([ctypes.c_void_p, ctypes.POINTER(ctypes.c_int32), ctypes.c_void_p], ctypes.c_int),
+    "fourtune_gelu_tanh_fwd": ([ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p], ctypes.c_int),
+    "fourtune_gelu_tanh_bwd": ([ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64,
+                                ctypes.c_void_p], ctypes.c_int),
+    "fourtune_encode_e2m1": ([ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p], ctypes.c_int),
+    "fourtune_encode_ue4m3": ([ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p], ctypes.c_int),
+}
+
+_lib = None
+
+
+def lib():
+    """Load the CUDA library (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"CUDA library not built: {LIB_PATH} (run diffusion_dit_b200/build.py)")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (argt, rest) in EXPORTS.items():
+            fn = getattr(L, name)
+            fn.argtypes = argt
+            fn.restype = rest
+        _lib = L
+    return _lib
+
+
+def _check(name: str, status: int):
+    if status != 0:
+        raise FourTuneError(name, status)
+
+
+def _p(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream: Optional[torch.cuda.Stream] = None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _require_cuda(*ts):
+    for t in ts:
+        if t is not None and not t.is_cuda:
+            raise ValueError("all tensors must be CUDA tensors")
+
+
+# ---------------------------------------------------------------------------
+@dataclasses.dataclass
+class QuantizedMatrix:
+    """Device tensors of one 16x16-block quantized matrix (see ft_fp4)."""
+
+    codes: torch.Tensor            # uint8 [rows, cols/2]
+    scales: torch.Tensor           # uint8 [rows/16, cols/16]
+    sf_mma: Optional[torch.Tensor]  # uint8 [rows * cols / 16] or None
+    g: torch.Tensor                # float32 [1]
+    rows: int
+    cols: int
+
+    @staticmethod
+    def empty(rows: int, cols: int, device, with_sf: bool = True) -> "QuantizedMatrix":
+        return QuantizedMatrix(
+            codes=torch.empty(rows, cols // 2, dtype=torch.uint8, device=device),
+            scales=torch.empty(rows // 16, cols // 16, dtype=torch.uint8, device=device),
+            sf_mma=torch.empty(rows * cols // 16, dtype=torch.uint8, device=device) if with_sf else None,
+            g=torch.empty(1, dtype=torch.float32, device=device), rows=rows, cols=cols)
+
+    def c_struct(self) -> FtFp4:
+        return FtFp4(self.codes.data_ptr(), self.scales.data_ptr(),
+                     self.sf_mma.data_ptr() if self.sf_mma is not None else None,
+                     self.g.data_ptr(), self.rows, self.cols)
+
+
+def quantize_block16(x: torch.Tensor, amax: Optional[torch.Tensor] = None, with_sf: bool = False,
+                     transposed: bool = False, down: Optional[torch.Tensor] = None,
+                     stream=None):
+    """Q(x) in 16x16 blocks on the GPU.  Returns (q, q_t or None, down_out or None)."""
+    _require_cuda(x, amax, down)
+    if x.dim() != 2 or x.stride(1) != 1:
+        raise ValueError("x must be a row-major 2-D tensor")
+    rows, cols = x.shape
+    dt = {torch.bfloat16: FT_DTYPE_BF16, torch.float32: FT_DTYPE_F32}[x.dtype]
+    q = QuantizedMatrix.empty(rows, cols, x.device, with_sf=with_sf or transposed)
+    qt = QuantizedMatrix.empty(cols, rows, x.device, with_sf=True) if transposed else None
+    r_down = 0 if down is None else down.shape[0]
+    down_out = torch.empty(rows, r_down, dtype=torch.float32, device=x.device) if r_down else None
+    nws = lib().fourtune_quantize_workspace_bytes(rows, cols, r_down)
+    ws = torch.zeros(nws, dtype=torch.uint8, device=x.device)
+    qs = q.c_struct()
+    qts = qt.c_struct() if qt is not None else None
+    st = lib().fourtune_quantize_block16(_p(x), dt, rows, cols, x.stride(0), _p(amax), _p(down), r_down,
+                                         _p(down_out), ctypes.byref(qs),
+                                         ctypes.byref(qts) if qts is not None else None,
+                                         _p(ws), nws, _stream(stream))
+    _check("fourtune_quantize_block16", st)
+    return q, qt, down_out
+
+
+@dataclasses.dataclass
+class LinearWeights:
+    """Frozen backbone + adapter of one layer, on the device."""
+
+    qr: QuantizedMatrix
+    qr_t: QuantizedMatrix
+    ls_down: torch.Tensor   # bf16 [r_s, K]
+    ls_up: torch.Tensor     # bf16 [N, r_s]
+    lora_a: torch.Tensor    # bf16 [r, K]
+    lora_b: torch.Tensor    # bf16 [N, r]
+    lora_scale: float
+
+    @property
+    def N(self):
+        return self.qr.rows
+
+    @property
+    def K(self):
+        return self.qr.cols
+
+    @property
+    def r_s(self):
+        return self.ls_down.shape[0]
+
+    @property
+    def r(self):
+        return self.lora_a.shape[0]
+
+    def c_struct(self) -> FtLinear:
+        return FtLinear(self.N, self.K, self.r_s, self.r, self.lora_scale, self.qr.c_struct(),
+                        self.qr_t.c_struct(), self.ls_down.data_ptr() if self.r_s else None,
+                        self.ls_up.data_ptr() if self.r_s else None,
+                        self.lora_a.data_ptr() if self.r else None,
+                        self.lora_b.data_ptr() if self.r else None)
+
+
+def prepare_weights(residual: torch.Tensor, ls_up: torch.Tensor, ls_down: torch.Tensor,
+                    lora_a: torch.Tensor, lora_b: torch.Tensor, lora_scale: float) -> LinearWeights:
+    """Q(R) offline (section 3.1) with its transposed copy (section 3.2), on the GPU.
+    ``residual`` is the fp32 (or bf16) R [N, K] on the device."""
+    qr, qr_t, _ = quantize_block16(residual.contiguous(), with_sf=True, transposed=True)
+    return LinearWeights(qr, qr_t, ls_down.contiguous(), ls_up.contiguous(), lora_a.contiguous(),
+                         lora_b.contiguous(), float(lora_scale))
+
+
+class Workspace:
+    """Caller-owned scratch for the layer calls, sized by the library's query."""
+
+    def __init__(self, weights: LinearWeights, M: int, device):
+        s = weights.c_struct()
+        self.nbytes = int(lib().fourtune_linear_workspace_bytes(ctypes.byref(s), M))
+        self.buf = torch.zeros(self.nbytes, dtype=torch.uint8, device=device)
+        self.M = M
+
+    def device_status(self, stream=None) -> int:
+        v = ctypes.c_int32(0)
+        _check("fourtune_device_status",
+               lib().fourtune_device_status(_p(self.buf), ctypes.byref(v), _stream(stream)))
+        return int(v.value)
+
+
+def linear_fwd(w: LinearWeights, x: torch.Tensor, ws: Workspace, y: Optional[torch.Tensor] = None,
+               t_saved: Optional[torch.Tensor] = None, amax: Optional[torch.Tensor] = None, stream=None):
+    """Eq. (2).  Returns (Y bf16 [M, N], T fp32 [M, r_s + r])."""
+    _require_cuda(x)
+    M = x.shape[0]
+    if y is None:
+        y = torch.empty(M, w.N, dtype=torch.bfloat16, device=x.device)
+    R = w.r_s + w.r
+    if t_saved is None:
+        t_saved = torch.empty(M, max(R, 1), dtype=torch.float32, device=x.device)
+    s = w.c_struct()
+    st = lib().fourtune_linear_fwd(ctypes.byref(s), _p(x), M, _p(amax), _p(y), _p(t_saved), _p(ws.buf),
+                                   ws.nbytes, _stream(stream))
+    _check("fourtune_linear_fwd", st)
+    return y, t_saved
+
+
+def linear_bwd(w: LinearWeights, x: torch.Tensor, t_saved: torch.Tensor, dy: torch.Tensor, ws: Workspace,
+               dx: Optional[torch.Tensor] = None, da: Optional[torch.Tensor] = None,
+               db: Optional[torch.Tensor] = None, amax: Optional[torch.Tensor] = None, stream=None):
+    """Eq. (3) and the adapter gradients.  Returns (dX bf16 [M, K], dA fp32 [r, K], dB fp32 [N, r])."""
+    _require_cuda(x, t_saved, dy)
+    M = x.shape[0]
+    if dx is None:
+        dx = torch.empty(M, w.K, dtype=torch.bfloat16, device=x.device)
+    if da is None:
+        da = torch.empty(max(w.r, 1), w.K, dtype=torch.float32, device=x.device)
+    if db is None:
+        db = torch.empty(w.N, max(w.r, 1), dtype=torch.float32, device=x.device)
+    s = w.c_struct()
+    st = lib().fourtune_linear_bwd(ctypes.byref(s), _p(x), _p(t_saved), _p(dy), M, _p(amax), _p(dx), _p(da),
+                                   _p(db), _p(ws.buf), ws.nbytes, _stream(stream))
+    _check("fourtune_linear_bwd", st)
+    return dx, da, db
+
+
+def gelu_tanh_fwd(p: torch.Tensor, h: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    _require_cuda(p)
+    h = torch.empty_like(p) if h is None else h
+    _check("fourtune_gelu_tanh_fwd", lib().fourtune_gelu_tanh_fwd(_p(p), _p(h), p.numel(), _stream(stream)))
+    return h
+
+
+def gelu_tanh_bwd(p: torch.Tensor, dh: torch.Tensor, dp: Optional[torch.Tensor] = None, stream=None):
+    _require_cuda(p, dh)
+    dp = torch.empty_like(p) if dp is None else dp
+    _check("fourtune_gelu_tanh_bwd",
+           lib().fourtune_gelu_tanh_bwd(_p(p), _p(dh), _p(dp), p.numel(), _stream(stream)))
+    return dp
+
+
+def encode_e2m1(v: torch.Tensor, stream=None) -> torch.Tensor:
+    _require_cuda(v)
+    out = torch.empty(v.numel(), dtype=torch.uint8, device=v.device)
+    _check("fourtune_encode_e2m1", lib().fourtune_encode_e2m1(_p(v), v.numel(), _p(out), _stream(stream)))
+    return out
+
+
+def encode_ue4m3(v: torch.Tensor, stream=None) -> torch.Tensor:
+    _require_cuda(v)
+    out = torch.empty(v.numel(), dtype=torch.uint8, device=v.device)
+    _check("fourtune_encode_ue4m3", lib().fourtune_encode_ue4m3(_p(v), v.numel(), _p(out), _stream(stream)))
+    return out
+
+
+class FourTuneLinearFunction(torch.autograd.Function):
+    """autograd wrapper: forward Eq. (2), backward Eq. (3) + adapter gradients.
+    Gradients flow to X, lora_a and lora_b only (R and the stabilizer are frozen)."""
+
+    @staticmethod
+    def forward(ctx, x, lora_a, lora_b, weights: LinearWeights, ws: Workspace):
+        y, t = linear_fwd(weights, x, ws)
+        ctx.save_for_backward(x, t)
+        ctx.weights, ctx.ws = weights, ws
+        return y
+
+    @staticmethod
+    def backward(ctx, dy):
+        x, t = ctx.saved_tensors
+        dx, da, db = linear_bwd(ctx.weights, x, t, dy.contiguous(), ctx.ws)
+        return dx, da.to(torch.bfloat16), db.to(torch.bfloat16), None, None

@@ -1,0 +1,207 @@
+/*
+ * fourtune.h -- C ABI of the W4A4G4 triple-branch linear layer on NVIDIA B200 (sm_100a).
+ *
+ * The layer is the one of "FourTune: Towards Fully 4-Bit Efficient Post-Training for
+ * Diffusion Models" (arXiv 2607.05711), section 3.  Layout (PyTorch's): X [M, K] tokens
+ * by input features, W and its residual R [N, K], Y [M, N].  The paper writes
+ * Y = X W with W in R^{m x n}; the algebra is the same, transposed.
+ *
+ *   Eq. (1)  W ~= R + L_stab,  L_stab = Ls_up * Ls_down     (frozen, high precision)
+ *   Eq. (2)  Y  = GEMM4(Q(X), Q(R)) + X L_stab^T + s (X A^T) B^T
+ *   Eq. (3)  dX = GEMM4(Q(G), Q(R)^T) + G L_stab + s (G B) A
+ *   sec. 3.2 dB = s G^T (X A^T),  dA = s (G B)^T X           (only the adapter trains)
+ *
+ * with G = dL/dY, LoRA factors A [r, K] and B [N, r], s = alpha / r.
+ *
+ * Q(.) is the 16x16-block NVFP4 quantizer (sections 3.1-3.2, Table 5): E2M1 element
+ * codes, one UE4M3 scale per 16x16 block, one fp32 factor g per tensor:
+ *   g  = 2688 / max|x|                              (fp32; g = 1 and all-zero output
+ *                                                    when max|x| == 0 or g overflows)
+ *   sb = UE4M3_rn_sat( fl32(fl32(max_block|x| / 6) * g) )
+ *   code(x) = sign(x) | E2M1_rn_sat( fl32(x * fl32(g / val(sb))) )   (0 when sb == 0)
+ *   xhat = val(code) * val(sb) / g
+ * Q is applied offline to R and on the fly to X and G.  Q(R)^T is the same codes and
+ * scales transposed block by block; nothing is requantized (section 3.2).
+ *
+ * CONVENTIONS (all entry points)
+ *  - Every pointer argument named *_dev or held in an ft_* struct is DEVICE memory owned
+ *    by the caller and must be 16-byte aligned.  Host pointers appear only where noted.
+ *  - `stream` is a cudaStream_t (NULL = the legacy default stream).  Calls are
+ *    asynchronous: they enqueue kernels and return.  The returned status reports
+ *    argument validation and launch errors only.
+ *  - Errors detected on the device (a bounded wait that expired) are recorded in a
+ *    status word inside the workspace; read it with fourtune_device_status().
+ *  - Matrices are row-major and dense (row stride == number of columns) unless an
+ *    `ld` argument says otherwise.  bf16 is IEEE bfloat16 stored as 16-bit words.
+ *  - The library allocates no device memory and keeps no state between calls other
+ *    than a per-process cache of driver entry points.  All scratch comes from the
+ *    caller's workspace `ws` of `ws_bytes` bytes (256-byte aligned); query the size first.
+ *  - Kernels never trap.  Shapes are checked on the host before any launch.
+ */
+#ifndef FOURTUNE_H_
+#define FOURTUNE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    FT_OK = 0,
+    FT_ERR_INVALID_ARG = 1, /* null pointer, negative size, bad flag */
+    FT_ERR_SHAPE = 2,       /* a dimension is not a supported multiple (see each call) */
+    FT_ERR_ALIGN = 3,       /* a device pointer is not 16-byte aligned */
+    FT_ERR_WORKSPACE = 4,   /* workspace missing or smaller than the query returned */
+    FT_ERR_CUDA = 5,        /* a CUDA runtime or driver call failed */
+    FT_ERR_UNSUPPORTED = 6, /* the current device is not sm_100 */
+    FT_ERR_TIMEOUT = 7      /* (device status) a bounded wait inside a kernel expired */
+} ft_status;
+
+/* Human-readable name of a status code (static string). */
+const char* fourtune_status_string(int status);
+
+/*
+ * A 16x16-block quantized matrix [rows, cols] (section 3.1 NVFP4, 16x16 blocks).
+ *   codes  : uint8 [rows, cols/2]; element (i, 2j) in the low nibble of byte (i, j),
+ *            element (i, 2j+1) in the high nibble; nibble = sign<<3 | E2M1 magnitude.
+ *   scales : uint8 [rows/16, cols/16], UE4M3 scale of each 16x16 block (row-major).
+ *   sf_mma : the same scales expanded to one scale per (row, 16 columns) and laid out
+ *            for the tensor core's block-scaled MMA: 512-byte atoms, one per 128 rows
+ *            x 64 columns, atoms of a 128-row band stored consecutively along the
+ *            columns; inside an atom the scale of (row m, column block b) sits at byte
+ *            16*(m%32) + 4*((m%128)/32) + b%4.  Size rows*cols/16 bytes.  Needs
+ *            rows % 128 == 0 and cols % 64 == 0.  May be NULL on output (not written).
+ *   g      : float[1], the tensor factor g.
+ */
+typedef struct {
+    uint8_t* codes;
+    uint8_t* scales;
+    uint8_t* sf_mma;
+    float* g;
+    int64_t rows;
+    int64_t cols;
+} ft_fp4;
+
+/*
+ * One frozen-backbone linear layer with its adapter (Eq. 1-2).
+ *   qr      : Q(R), rows = N, cols = K, sf_mma required.
+ *   qr_t    : Q(R)^T, rows = K, cols = N, sf_mma required (written by
+ *             fourtune_quantize_block16 with an out_t argument).
+ *   ls_down : bf16 [r_s, K]   (L_stab = ls_up * ls_down)
+ *   ls_up   : bf16 [N, r_s]
+ *   lora_a  : bf16 [r, K]
+ *   lora_b  : bf16 [N, r]
+ *   lora_scale : s = alpha / r.
+ * r_s + r must be >= 1 and <= 240 (either may be 0).
+ */
+typedef struct {
+    int64_t N;
+    int64_t K;
+    int32_t r_s;
+    int32_t r;
+    float lora_scale;
+    ft_fp4 qr;
+    ft_fp4 qr_t;
+    const void* ls_down;
+    const void* ls_up;
+    const void* lora_a;
+    const void* lora_b;
+} ft_linear;
+
+/* Input element types for fourtune_quantize_block16. */
+#define FT_DTYPE_BF16 0
+#define FT_DTYPE_F32 1
+
+/*
+ * Workspace bytes needed by fourtune_quantize_block16 for a [rows, cols] input with a
+ * fused down-projection of rank r_down (0 for none).
+ */
+size_t fourtune_quantize_workspace_bytes(int64_t rows, int64_t cols, int32_t r_down);
+
+/*
+ * Q(.) of sections 3.1-3.2: quantize x [rows, cols] (row stride ld elements) into
+ * 16x16-block NVFP4 codes and scales, optionally fused with a down-projection
+ * (section 3.3 "LoRA Fusion": the quantizer and the low-rank down-projections read
+ * the same input once).
+ *   x_dev          : bf16 or fp32 (x_dtype = FT_DTYPE_BF16 / FT_DTYPE_F32), device.
+ *   rows, cols     : multiples of 16 (128 and 64 when out->sf_mma or out_t is used).
+ *   amax_or_null   : device float[1] holding max|x| to use for g, or NULL to compute
+ *                    it (one extra read of x).  A caller-supplied value smaller than
+ *                    the true maximum saturates codes; larger values are valid.
+ *   down_dev       : bf16 [r_down, cols] or NULL; down_out_dev: fp32 [rows, r_down]
+ *                    receives x * down^T (exact fp32 accumulation order not specified).
+ *                    bf16 input only.
+ *   out            : codes/scales/g required, sf_mma optional.
+ *   out_t          : optional Q(x)^T (rows = cols, cols = rows), the transpose of the
+ *                    same codes and scales (no requantization); sf_mma required when set.
+ * Errors: FT_ERR_INVALID_ARG, FT_ERR_SHAPE, FT_ERR_ALIGN, FT_ERR_WORKSPACE, FT_ERR_CUDA.
+ */
+ft_status fourtune_quantize_block16(const void* x_dev, int32_t x_dtype, int64_t rows,
+                                    int64_t cols, int64_t ld, const float* amax_or_null,
+                                    const void* down_dev, int32_t r_down, float* down_out_dev,
+                                    const ft_fp4* out, const ft_fp4* out_t, void* ws,
+                                    size_t ws_bytes, void* stream);
+
+/* Workspace bytes for fourtune_linear_fwd / fourtune_linear_bwd with M tokens. */
+size_t fourtune_linear_workspace_bytes(const ft_linear* layer, int64_t M);
+
+/*
+ * Forward pass, Eq. (2): Y = GEMM4(Q(X), Q(R)) + X Ls_down^T Ls_up^T + s X A^T B^T.
+ *   x_dev      : bf16 [M, K].
+ *   amax_or_null : device float[1] = max|X| (see fourtune_quantize_block16) or NULL.
+ *   y_dev      : bf16 [M, N], written.
+ *   t_saved_dev: fp32 [M, r_s + r], written: X [Ls_down; A]^T, kept for the backward.
+ * Shapes: M % 128 == 0, N % 256 == 0, K % 256 == 0.
+ */
+ft_status fourtune_linear_fwd(const ft_linear* layer, const void* x_dev, int64_t M,
+                              const float* amax_or_null, void* y_dev, float* t_saved_dev,
+                              void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Backward pass, Eq. (3) and the adapter gradients of section 3.2.
+ *   x_dev       : bf16 [M, K], the forward input.
+ *   t_saved_dev : fp32 [M, r_s + r] from fourtune_linear_fwd.
+ *   dy_dev      : bf16 [M, N], G = dL/dY.
+ *   amax_or_null: device float[1] = max|G| or NULL.
+ *   dx_dev      : bf16 [M, K], written: GEMM4(Q(G), Q(R)^T) + G Ls_up Ls_down + s G B A.
+ *   da_dev      : fp32 [r, K], written (overwritten, not accumulated): s (G B)^T X.
+ *   db_dev      : fp32 [N, r], written (overwritten, not accumulated): s G^T (X A^T).
+ * Shapes as for the forward.  R and L_stab get no gradient (frozen).
+ */
+ft_status fourtune_linear_bwd(const ft_linear* layer, const void* x_dev, const float* t_saved_dev,
+                              const void* dy_dev, int64_t M, const float* amax_or_null,
+                              void* dx_dev, float* da_dev, float* db_dev, void* ws,
+                              size_t ws_bytes, void* stream);
+
+/*
+ * Reads (synchronously, on `stream`) the device status word that the kernels of the
+ * last call using workspace `ws` left behind: FT_OK or FT_ERR_TIMEOUT.  *status_out is
+ * a HOST pointer.  Clears the word.
+ */
+ft_status fourtune_device_status(void* ws, int32_t* status_out, void* stream);
+
+/*
+ * GELU (tanh form) between the MLP linears (section 3.3 "MLP Fusion" names GeLU):
+ *   fwd: h = bf16(0.5 p (1 + tanh(sqrt(2/pi) (p + 0.044715 p^3))))
+ *   bwd: dp = bf16(dh * gelu'(p))
+ * p, h, dh, dp: bf16 device arrays of n elements (n % 8 == 0).
+ */
+ft_status fourtune_gelu_tanh_fwd(const void* p_dev, void* h_dev, int64_t n, void* stream);
+ft_status fourtune_gelu_tanh_bwd(const void* p_dev, const void* dh_dev, void* dp_dev, int64_t n,
+                                 void* stream);
+
+/*
+ * Codec access for exhaustive checks of the conversions the quantizer uses:
+ * out[i] = E2M1 code (with sign) of v[i], or UE4M3 code of v[i] (v[i] >= 0), both
+ * round-to-nearest-even with saturation.  v: fp32 device [n]; out: uint8 device [n].
+ */
+ft_status fourtune_encode_e2m1(const float* v_dev, int64_t n, uint8_t* out_dev, void* stream);
+ft_status fourtune_encode_ue4m3(const float* v_dev, int64_t n, uint8_t* out_dev, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FOURTUNE_H_ */
