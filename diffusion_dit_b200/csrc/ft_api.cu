@@ -2,6 +2,7 @@
 // Host side only: argument checks, workspace carving, TMA descriptors, launch order.
 #include <cudaTypedefs.h>
 
+#include <atomic>
 #include <mutex>
 
 #include "fourtune.h"
@@ -192,9 +193,47 @@ ft_status run_gemm(const uint8_t* a_codes, const uint8_t* a_sf, const float* ga,
     return FT_OK;
 }
 
+std::atomic<uint64_t> g_launches{0};
+std::mutex g_ev_mu;
+cudaEvent_t g_ev_before[FT_KERNEL_KINDS] = {};
+cudaEvent_t g_ev_after[FT_KERNEL_KINDS] = {};
+
 }  // namespace
 
+namespace ft {
+
+void before_launch(int kind, cudaStream_t stream) {
+    if (kind < 0 || kind >= FT_KERNEL_KINDS) return;
+    std::lock_guard<std::mutex> lock(g_ev_mu);
+    if (g_ev_before[kind]) {
+        cudaEventRecord(g_ev_before[kind], stream);
+        g_ev_before[kind] = nullptr;
+    }
+}
+
+void after_launch(int kind, cudaStream_t stream) {
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    if (kind < 0 || kind >= FT_KERNEL_KINDS) return;
+    std::lock_guard<std::mutex> lock(g_ev_mu);
+    if (g_ev_after[kind]) {
+        cudaEventRecord(g_ev_after[kind], stream);
+        g_ev_after[kind] = nullptr;
+    }
+}
+
+}  // namespace ft
+
 extern "C" {
+
+uint64_t fourtune_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+ft_status fourtune_time_next_launch(int32_t kernel, void* ev_before, void* ev_after) {
+    if (kernel < 0 || kernel >= FT_KERNEL_KINDS) return FT_ERR_INVALID_ARG;
+    std::lock_guard<std::mutex> lock(g_ev_mu);
+    g_ev_before[kernel] = static_cast<cudaEvent_t>(ev_before);
+    g_ev_after[kernel] = static_cast<cudaEvent_t>(ev_after);
+    return FT_OK;
+}
 
 const char* fourtune_status_string(int s) {
     switch (s) {

@@ -269,7 +269,9 @@ cudaError_t launch_gemm_fp4_lowrank(const CUtensorMap& tmA, const CUtensorMap& t
     }
     const int tiles = (args.M / BM) * (args.N / BN);
     const int grid = tiles < num_sms ? tiles : num_sms;
+    before_launch(K_GEMM, stream);
     gemm_fp4_lowrank_kernel<<<grid, THREADS, SMEM_BYTES, stream>>>(tmA, tmB, tmLA, tmLB, args);
+    after_launch(K_GEMM, stream);
     return cudaGetLastError();
 }
 

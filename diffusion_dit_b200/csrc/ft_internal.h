@@ -8,6 +8,13 @@
 
 namespace ft {
 
+// Instrumentation (ft_api.cu): every launcher calls before_launch(kind, stream) and
+// after_launch(kind, stream) around its kernel launch.
+enum KernelKind { K_GEMM = 0, K_QUANT = 1, K_AMAX = 2, K_LOWRANK = 3, K_LORA_DB = 4, K_LORA_DA = 5,
+                  K_OTHER = 6 };
+void before_launch(int kind, cudaStream_t stream);
+void after_launch(int kind, cudaStream_t stream);
+
 struct GemmFp4Args {
     const uint8_t* sfa;     // tensor-core scale layout of A (rows M, cols K)
     const uint8_t* sfb;     // tensor-core scale layout of B (rows N, cols K)

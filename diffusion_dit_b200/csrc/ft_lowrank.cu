@@ -214,7 +214,9 @@ cudaError_t launch_lowrank_down(const LowRankDownArgs& a, cudaStream_t stream) {
         if (e != cudaSuccess) return e;
         attr = true;
     }
+    before_launch(K_LOWRANK, stream);
     lowrank_down_kernel<<<static_cast<unsigned>(a.M / TM), 256, smem, stream>>>(a);
+    after_launch(K_LOWRANK, stream);
     return cudaGetLastError();
 }
 
@@ -223,22 +225,28 @@ cudaError_t launch_build_factors(const __nv_bfloat16* ls_down, const __nv_bfloat
                                  int64_t K, int r_s, int r, int KL, __nv_bfloat16* dn,
                                  __nv_bfloat16* upcat, __nv_bfloat16* upt, __nv_bfloat16* dntcat,
                                  cudaStream_t stream) {
+    before_launch(K_OTHER, stream);
     build_factors_kernel<<<148 * 4, 256, 0, stream>>>(ls_down, lora_a, ls_up, lora_b, N, K, r_s, r, KL,
                                                       dn, upcat, upt, dntcat);
+    after_launch(K_OTHER, stream);
     return cudaGetLastError();
 }
 
 cudaError_t launch_lora_db(const __nv_bfloat16* g, int64_t M, int64_t N, const float* t, int R,
                            int r_s, int r, float s, float* db, cudaStream_t stream) {
     const size_t smem = sizeof(float) * TK * (64 + r);
+    before_launch(K_LORA_DB, stream);
     lora_db_kernel<<<static_cast<unsigned>(N / 64), 256, smem, stream>>>(g, M, N, t, R, r_s, r, s, db);
+    after_launch(K_LORA_DB, stream);
     return cudaGetLastError();
 }
 
 cudaError_t launch_lora_da(const float* u, int R, int r_s, int r, const __nv_bfloat16* x, int64_t M,
                            int64_t K, float s, float* da, cudaStream_t stream) {
     const size_t smem = sizeof(float) * TK * (64 + r);
+    before_launch(K_LORA_DA, stream);
     lora_da_kernel<<<static_cast<unsigned>(K / 64), 256, smem, stream>>>(u, R, r_s, r, x, M, K, s, da);
+    after_launch(K_LORA_DA, stream);
     return cudaGetLastError();
 }
 

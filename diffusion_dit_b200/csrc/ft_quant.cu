@@ -239,12 +239,14 @@ cudaError_t launch_amax(const void* x, bool is_f32, int64_t rows, int64_t cols, 
     cudaError_t e = cudaMemsetAsync(amax_out, 0, sizeof(float), stream);
     if (e != cudaSuccess) return e;
     const int grid = grid_for(rows * cols / 8, 256, num_sms * 4);
+    before_launch(K_AMAX, stream);
     if (is_f32)
         amax_kernel<float><<<grid, 256, 0, stream>>>(static_cast<const float*>(x), rows, cols, ld,
                                                       reinterpret_cast<unsigned*>(amax_out));
     else
         amax_kernel<__nv_bfloat16><<<grid, 256, 0, stream>>>(
             static_cast<const __nv_bfloat16*>(x), rows, cols, ld, reinterpret_cast<unsigned*>(amax_out));
+    after_launch(K_AMAX, stream);
     return cudaGetLastError();
 }
 
@@ -253,52 +255,68 @@ cudaError_t launch_quant_block16(const void* x, bool is_f32, int64_t rows, int64
                                  int num_sms, cudaStream_t stream) {
     const int64_t nblocks = (rows / 16) * (cols / 16);
     const int grid = grid_for(nblocks * 32, 256, num_sms * 8);
+    before_launch(K_QUANT, stream);
     if (is_f32)
         quant_block16_kernel<float><<<grid, 256, 0, stream>>>(static_cast<const float*>(x), rows, cols,
                                                                ld, amax, codes, scales, g_out);
     else
         quant_block16_kernel<__nv_bfloat16><<<grid, 256, 0, stream>>>(
             static_cast<const __nv_bfloat16*>(x), rows, cols, ld, amax, codes, scales, g_out);
+    after_launch(K_QUANT, stream);
     return cudaGetLastError();
 }
 
 cudaError_t launch_expand_scales(const uint8_t* scales, int64_t rows, int64_t cols, uint8_t* sf_mma,
                                  cudaStream_t stream) {
     const int grid = grid_for(rows * cols / 16, 256, 148 * 8);
+    before_launch(K_OTHER, stream);
     expand_scales_kernel<<<grid, 256, 0, stream>>>(scales, rows, cols, sf_mma);
+    after_launch(K_OTHER, stream);
     return cudaGetLastError();
 }
 
 cudaError_t launch_transpose_q(const uint8_t* codes, const uint8_t* scales, int64_t rows, int64_t cols,
                                uint8_t* codes_t, uint8_t* scales_t, cudaStream_t stream) {
     const int grid = grid_for(rows * cols / 2, 256, 148 * 8);
+    before_launch(K_OTHER, stream);
     transpose_q_kernel<<<grid, 256, 0, stream>>>(codes, scales, rows, cols, codes_t, scales_t);
+    after_launch(K_OTHER, stream);
     return cudaGetLastError();
 }
 
 cudaError_t launch_copy_scalar(const float* src, float* dst, cudaStream_t stream) {
+    before_launch(K_OTHER, stream);
     copy_scalar_kernel<<<1, 1, 0, stream>>>(src, dst);
+    after_launch(K_OTHER, stream);
     return cudaGetLastError();
 }
 
 cudaError_t launch_encode_e2m1(const float* v, int64_t n, uint8_t* out, cudaStream_t stream) {
+    before_launch(K_OTHER, stream);
     encode_e2m1_kernel<<<grid_for(n, 256, 148 * 16), 256, 0, stream>>>(v, n, out);
+    after_launch(K_OTHER, stream);
     return cudaGetLastError();
 }
 
 cudaError_t launch_encode_ue4m3(const float* v, int64_t n, uint8_t* out, cudaStream_t stream) {
+    before_launch(K_OTHER, stream);
     encode_ue4m3_kernel<<<grid_for(n, 256, 148 * 16), 256, 0, stream>>>(v, n, out);
+    after_launch(K_OTHER, stream);
     return cudaGetLastError();
 }
 
 cudaError_t launch_gelu_fwd(const __nv_bfloat16* p, __nv_bfloat16* h, int64_t n, cudaStream_t stream) {
+    before_launch(K_OTHER, stream);
     gelu_fwd_kernel<<<grid_for(n / 8, 256, 148 * 8), 256, 0, stream>>>(p, h, n);
+    after_launch(K_OTHER, stream);
     return cudaGetLastError();
 }
 
 cudaError_t launch_gelu_bwd(const __nv_bfloat16* p, const __nv_bfloat16* dh, __nv_bfloat16* dp,
                             int64_t n, cudaStream_t stream) {
+    before_launch(K_OTHER, stream);
     gelu_bwd_kernel<<<grid_for(n / 8, 256, 148 * 8), 256, 0, stream>>>(p, dh, dp, n);
+    after_launch(K_OTHER, stream);
     return cudaGetLastError();
 }
 

@@ -64,7 +64,11 @@ EXPORTS = {
                                 ctypes.c_void_p], ctypes.c_int),
     "fourtune_encode_e2m1": ([ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p], ctypes.c_int),
     "fourtune_encode_ue4m3": ([ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p], ctypes.c_int),
+    "fourtune_launch_count": ([], ctypes.c_uint64),
+    "fourtune_time_next_launch": ([ctypes.c_int32, ctypes.c_void_p, ctypes.c_void_p], ctypes.c_int),
 }
+
+FT_KERNEL_GEMM, FT_KERNEL_QUANT, FT_KERNEL_AMAX, FT_KERNEL_LOWRANK, FT_KERNEL_LORA_DB, FT_KERNEL_LORA_DA = range(6)
 
 _lib = None
 
@@ -279,6 +283,19 @@ def encode_ue4m3(v: torch.Tensor, stream=None) -> torch.Tensor:
     out = torch.empty(v.numel(), dtype=torch.uint8, device=v.device)
     _check("fourtune_encode_ue4m3", lib().fourtune_encode_ue4m3(_p(v), v.numel(), _p(out), _stream(stream)))
     return out
+
+
+def launch_count() -> int:
+    """Kernels the library has launched in this process."""
+    return int(lib().fourtune_launch_count())
+
+
+def time_next_launch(kind: int, before: Optional[torch.cuda.Event], after: Optional[torch.cuda.Event]):
+    """Have the library record ``before``/``after`` (timing events) around its next
+    launch of kernel ``kind`` (FT_KERNEL_*), on that launch's stream."""
+    b = ctypes.c_void_p(before.cuda_event) if before is not None else None
+    a = ctypes.c_void_p(after.cuda_event) if after is not None else None
+    _check("fourtune_time_next_launch", lib().fourtune_time_next_launch(kind, b, a))
 
 
 class FourTuneLinearFunction(torch.autograd.Function):

@@ -200,6 +200,24 @@ ft_status fourtune_gelu_tanh_bwd(const void* p_dev, const void* dh_dev, void* dp
 ft_status fourtune_encode_e2m1(const float* v_dev, int64_t n, uint8_t* out_dev, void* stream);
 ft_status fourtune_encode_ue4m3(const float* v_dev, int64_t n, uint8_t* out_dev, void* stream);
 
+/*
+ * Instrumentation for benchmarks.
+ * fourtune_launch_count: number of kernels this library has launched in this process.
+ * fourtune_time_next_launch: records the caller's CUDA events (cudaEvent_t, created by
+ *   the caller) on the launch stream immediately before and after the NEXT launch of the
+ *   given kernel kind (FT_KERNEL_*), then forgets them.  Either event may be NULL.
+ *   Returns FT_ERR_INVALID_ARG for an unknown kind.
+ */
+#define FT_KERNEL_GEMM 0      /* 4-bit GEMM with the low-rank tail (forward and dX) */
+#define FT_KERNEL_QUANT 1     /* 16x16 block quantizer */
+#define FT_KERNEL_AMAX 2      /* tensor max */
+#define FT_KERNEL_LOWRANK 3   /* low-rank down-projection */
+#define FT_KERNEL_LORA_DB 4   /* adapter gradient dB */
+#define FT_KERNEL_LORA_DA 5   /* adapter gradient dA */
+#define FT_KERNEL_KINDS 6
+uint64_t fourtune_launch_count(void);
+ft_status fourtune_time_next_launch(int32_t kernel, void* ev_before, void* ev_after);
+
 #ifdef __cplusplus
 }
 #endif
