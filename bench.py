@@ -1,0 +1,359 @@
+"""Benchmark of the W4A4G4 triple-branch linear layer (FourTune, arXiv 2607.05711).
+
+One step = the whole hot path once over one batch: the forward (tensor max, 16x16
+block quantization of X, the low-rank down-projection, the 4-bit GEMM with the up-
+projections fused in) and the backward (the same for G, the dX GEMM through Q(R)^T,
+and the adapter gradients dA, dB).  Workload: the FLUX.1-dev attention QKV projection,
+4608 tokens (4096 image + 512 text) x 3072 -> 9216, stabilizer rank 32, LoRA rank 16,
+synthetic inputs and random-init weights of that shape (see workloads.py).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+N > 1 runs data-parallel under torchrun: each rank processes its own 4608 tokens
+(weak scaling) and the adapter gradients are summed with an NCCL all-reduce.  The
+reference arm times the CPU oracle (the only reference this method has) on a bounded
+sample of the same workload.  One JSON line on rank 0.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "W4A4G4 linear fwd+bwd TFLOPS & % FP4 roofline; quantizer GB/s vs HBM"
+NOMINAL_FP4_OVER_BF16 = 4.0   # 9 / 2.25 PFLOP/s dense (B200 spec ratio)
+
+
+def layer_flops(M, K, N, r_s, r):
+    R = r_s + r
+    fp4 = 4.0 * M * N * K                              # forward GEMM + dX GEMM
+    bf16 = 2.0 * R * (2 * M * K + 2 * M * N) + 2.0 * r * (M * N + M * K)
+    return fp4, bf16
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), "measured"
+    except Exception:
+        return 6650.0, 1590.0, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clock and throttle-reason samples during the timed region."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = os.path.join("/tmp", f"ft_clocks_{os.getpid()}.csv")
+
+    def __enter__(self):
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=self.f, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.f.close()
+
+    def summary(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) == 6 and parts[0].isdigit():
+                    rows.append(parts)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[2 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(int(r[0]) for r in rows), "sm_max_mhz": int(rows[0][1]),
+                "reasons": reasons, "samples": len(rows)}
+
+
+def run_reference(args, spec):
+    """The reference arm: the CPU oracle as it stands, on a bounded token sample."""
+    import numpy as np
+    import torch
+
+    from diffusion_dit_b200 import prep, workloads as wl
+    from oracle import fourtune_oracle as ora
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    rows = args.ref_rows
+    inp = wl.make_layer_inputs(spec, seed=0, rows=rows)
+    split = prep.svd_split(inp.w, spec.r_s)
+    layer = ora.Layer(qr=ora.quantize_residual(split.residual), ls_up=split.ls_up, ls_down=split.ls_down,
+                      lora_a=inp.lora_a, lora_b=inp.lora_b, lora_scale=spec.lora_scale)
+    threads = blas_threads()
+
+    def one():
+        ora.linear_fwd(inp.x, layer)
+        ora.linear_bwd(inp.x, inp.dy, layer)
+
+    for _ in range(args.warmup):
+        one()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        one()
+    dt = (time.perf_counter() - t0) / args.steps
+    fp4, bf = layer_flops(rows, spec.K, spec.N, spec.r_s, spec.r)
+    value = (fp4 + bf) / dt / 1e12
+    sample = f"{rows} of {spec.M} tokens, full weights; oracle quantize+fwd+bwd (fp64 products)"
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": workload_config(spec),
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        return max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def workload_config(spec):
+    return {"workload": f"{spec.name} fwd+bwd", "M_tokens_per_gpu": spec.M, "K": spec.K, "N": spec.N,
+            "stabilizer_rank": spec.r_s, "lora_rank": spec.r,
+            "l2": "flushed between steps (512 MiB write, outside the step events)"}
+
+
+def cpu_baseline(spec, budget_s=12.0, rows=512):
+    """The oracle timed on the host cores on a bounded sample (rank 0, N = 1)."""
+    import torch  # noqa: F401
+
+    from diffusion_dit_b200 import prep, workloads as wl
+    from oracle import fourtune_oracle as ora
+    inp = wl.make_layer_inputs(spec, seed=0, rows=rows)
+    split = prep.svd_split(inp.w, spec.r_s)
+    layer = ora.Layer(qr=ora.quantize_residual(split.residual), ls_up=split.ls_up, ls_down=split.ls_down,
+                      lora_a=inp.lora_a, lora_b=inp.lora_b, lora_scale=spec.lora_scale)
+    n, t0 = 0, time.perf_counter()
+    while True:
+        ora.linear_fwd(inp.x, layer)
+        ora.linear_bwd(inp.x, inp.dy, layer)
+        n += 1
+        if time.perf_counter() - t0 >= budget_s:
+            break
+    dt = (time.perf_counter() - t0) / n
+    fp4, bf = layer_flops(rows, spec.K, spec.N, spec.r_s, spec.r)
+    return {"value": (fp4 + bf) / dt / 1e12, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
+            "sample": f"{rows} of {spec.M} tokens with the full weights, {n} oracle passes "
+                      f"(quantize + fwd + bwd, fp64 products) in {time.perf_counter() - t0:.1f} s"}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--ref-rows", type=int, default=256)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    from diffusion_dit_b200 import workloads as wl
+    spec = wl.FLUX_QKV
+    if args.impl == "reference":
+        run_reference(args, spec)
+        return
+
+    import torch
+    import torch.distributed as dist
+
+    from diffusion_dit_b200 import fourtune as ft
+    from diffusion_dit_b200 import dp, prep
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    # --- setup (untimed): inputs of this rank's shard, offline weight prep ------
+    inp = wl.make_layer_inputs(spec, seed=rank)
+    split = prep.svd_split(inp.w, spec.r_s)
+    w = ft.prepare_weights(split.residual.to(dev), split.ls_up.to(dev), split.ls_down.to(dev),
+                           inp.lora_a.to(dev), inp.lora_b.to(dev), spec.lora_scale)
+    M, K, N = spec.M, spec.K, spec.N
+    R = spec.r_s + spec.r
+    ws = ft.Workspace(w, M, dev)
+    x = inp.x.to(dev)
+    dy = inp.dy.to(dev)
+    y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+    t = torch.empty(M, R, dtype=torch.float32, device=dev)
+    dx = torch.empty(M, K, dtype=torch.bfloat16, device=dev)
+    da = torch.empty(spec.r, K, dtype=torch.float32, device=dev)
+    db = torch.empty(N, spec.r, dtype=torch.float32, device=dev)
+    flush = torch.empty(512 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+
+    def step():
+        ft.linear_fwd(w, x, ws, y=y, t_saved=t)
+        ft.linear_bwd(w, x, t, dy, ws, dx=dx, da=da, db=db)
+        if world > 1:
+            dp.allreduce_adapter_grads(da, db)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    if ws.device_status() != 0:
+        raise RuntimeError("device status reports a timeout during warm-up")
+
+    Kst = args.steps
+    E = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+    ev_s, ev_e = [E() for _ in range(Kst)], [E() for _ in range(Kst)]
+    g_s, g_e = [E() for _ in range(2 * Kst)], [E() for _ in range(2 * Kst)]
+    q_s, q_e = [E() for _ in range(2 * Kst)], [E() for _ in range(2 * Kst)]
+    a_s, a_e = [E() for _ in range(2 * Kst)], [E() for _ in range(2 * Kst)]
+    for ev in ev_s + ev_e + g_s + g_e + q_s + q_e + a_s + a_e:
+        ev.record()  # torch creates the CUDA event on first record; the library needs the handle
+    torch.cuda.synchronize()
+
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    launches0 = ft.launch_count()
+    with ClockSampler(local) as clocks:
+        for i in range(Kst):
+            flush.zero_()
+            ev_s[i].record()
+            ft.time_next_launch(ft.FT_KERNEL_GEMM, g_s[2 * i], g_e[2 * i])
+            ft.time_next_launch(ft.FT_KERNEL_QUANT, q_s[2 * i], q_e[2 * i])
+            ft.time_next_launch(ft.FT_KERNEL_AMAX, a_s[2 * i], a_e[2 * i])
+            ft.linear_fwd(w, x, ws, y=y, t_saved=t)
+            ft.time_next_launch(ft.FT_KERNEL_GEMM, g_s[2 * i + 1], g_e[2 * i + 1])
+            ft.time_next_launch(ft.FT_KERNEL_QUANT, q_s[2 * i + 1], q_e[2 * i + 1])
+            ft.time_next_launch(ft.FT_KERNEL_AMAX, a_s[2 * i + 1], a_e[2 * i + 1])
+            ft.linear_bwd(w, x, t, dy, ws, dx=dx, da=da, db=db)
+            if world > 1:
+                dp.allreduce_adapter_grads(da, db)
+            ev_e[i].record()
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+    launches = ft.launch_count() - launches0
+    if ws.device_status() != 0:
+        raise RuntimeError("device status reports a timeout in the timed region")
+
+    total_ms = sum(ev_s[i].elapsed_time(ev_e[i]) for i in range(Kst))
+    gemm_ms = [g_s[j].elapsed_time(g_e[j]) for j in range(2 * Kst)]
+    quant_ms = [q_s[j].elapsed_time(q_e[j]) for j in range(2 * Kst)]
+    amax_ms = [a_s[j].elapsed_time(a_e[j]) for j in range(2 * Kst)]
+    tm = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(tm, op=dist.ReduceOp.MAX)
+    total_ms = float(tm.item())
+    ms_per_step = total_ms / Kst
+    fp4, bf = layer_flops(M, K, N, spec.r_s, spec.r)
+    value = world * (fp4 + bf) * Kst / (total_ms * 1e-3) / 1e12
+
+    # --- end to end through the API with host buffers (pinned), copies timed ---
+    x_h = inp.x.pin_memory()
+    dy_h = inp.dy.pin_memory()
+    da_h = torch.empty(da.shape, dtype=da.dtype).pin_memory()
+    db_h = torch.empty(db.shape, dtype=db.dtype).pin_memory()
+    e_s, e_e = [E() for _ in range(Kst)], [E() for _ in range(Kst)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    for i in range(Kst):
+        flush.zero_()
+        e_s[i].record()
+        x.copy_(x_h, non_blocking=True)
+        dy.copy_(dy_h, non_blocking=True)
+        ft.linear_fwd(w, x, ws, y=y, t_saved=t)
+        ft.linear_bwd(w, x, t, dy, ws, dx=dx, da=da, db=db)
+        if world > 1:
+            dp.allreduce_adapter_grads(da, db)
+        da_h.copy_(da, non_blocking=True)
+        db_h.copy_(db, non_blocking=True)
+        e_e[i].record()
+    torch.cuda.synchronize()
+    e2e_ms = torch.tensor([sum(e_s[i].elapsed_time(e_e[i]) for i in range(Kst))], dtype=torch.float64,
+                          device=dev)
+    if world > 1:
+        dist.all_reduce(e2e_ms, op=dist.ReduceOp.MAX)
+    e2e_value = world * (fp4 + bf) * Kst / (float(e2e_ms.item()) * 1e-3) / 1e12
+    h2d = x.numel() * 2 + dy.numel() * 2
+    d2h = da.numel() * 4 + db.numel() * 4
+
+    if rank == 0:
+        hbm, bf16_peak, src = peaks()
+        fp4_peak = bf16_peak * NOMINAL_FP4_OVER_BF16
+        gemm_avg = statistics.mean(gemm_ms)
+        achieved = 2.0 * M * N * K / (gemm_avg * 1e-3) / 1e12
+        traffic = None
+        # quantizer: X [M, K] and G [M, N] alternate; algorithmic bytes per element:
+        # 2 (read bf16) + 0.5 (codes) + 1/256 (block scales); the tensor max is one more read.
+        elems = [M * K, M * N] * Kst
+        qbytes = sum(e * (2.0 + 0.5 + 1.0 / 256) for e in elems)
+        q_gbs = qbytes / (sum(quant_ms) * 1e-3) / 1e9
+        qa_gbs = (qbytes + sum(2.0 * e for e in elems)) / ((sum(quant_ms) + sum(amax_ms)) * 1e-3) / 1e9
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": Kst,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "nvfp4(e2m1,ue4m3)+bf16", "data": "synthetic",
+            "config": dict(workload_config(spec), parallelism=f"dp{world}",
+                           flops_per_step={"fp4": fp4, "bf16": bf}),
+            "roofline": {"bound": "tensor", "kernel": "gemm_fp4_lowrank_kernel (fwd and dX)",
+                         "achieved": achieved, "peak": fp4_peak, "unit": "TFLOP/s",
+                         "frac": achieved / fp4_peak, "traffic": traffic,
+                         "peak_source": f"{src} bf16 {bf16_peak} TFLOP/s x {NOMINAL_FP4_OVER_BF16} "
+                                        f"(nominal fp4/bf16 ratio)",
+                         "avg_launch_ms": gemm_avg},
+            "quantizer": {"kernel": "quant_block16_kernel", "achieved_gbs": q_gbs,
+                          "with_amax_pass_gbs": qa_gbs, "peak_gbs": hbm, "frac": q_gbs / hbm,
+                          "frac_with_amax": qa_gbs / hbm, "avg_launch_ms": statistics.mean(quant_ms)},
+            "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "gpu_launches": launches,
+            "clocks": clocks.summary(),
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(spec)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

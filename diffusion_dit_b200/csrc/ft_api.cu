@@ -84,14 +84,29 @@ ft_status cuda_status(cudaError_t e) { return e == cudaSuccess ? FT_OK : FT_ERR_
 
 int low_rank_width(int R) { return R == 0 ? 0 : static_cast<int>(align_up(2 * static_cast<size_t>(R), 64)); }
 
+// Width of the tensor-core down-projection: the rank rounded up to the MMA's N step.
+int padded_rank(int R) { return R == 0 ? 0 : static_cast<int>(align_up(static_cast<size_t>(R), 16)); }
+
+uint32_t tmem_cols_for(int Rp) {
+    uint32_t c = 32;
+    while (c < static_cast<uint32_t>(Rp)) c <<= 1;
+    return c;
+}
+
+constexpr int kMaxSplits = 16;  // upper bound of quant_down_splits()
+
 // Workspace of the layer calls.  Regions are 256-byte aligned.
 struct LinearWs {
-    size_t status, scal, qx_codes, qx_scales, qx_sf, dn, upcat, tcat;
-    size_t qg_codes, qg_scales, qg_sf, upt, dntcat, u, ucat, total;
+    size_t status, scal, qx_codes, qx_scales, qx_sf, dn, upcat, tcat, partial;
+    size_t qg_codes, qg_scales, qg_sf, upt, dntcat, u, ucat, vcat, gpartial, total;
 };
 
-LinearWs linear_ws(int64_t M, int64_t N, int64_t K, int R) {
+// Width of the adapter-gradient operand [hi, lo, 0]: 2r rounded up to 64.
+int lora_width(int r) { return r == 0 ? 0 : static_cast<int>(align_up(2 * static_cast<size_t>(r), 64)); }
+
+LinearWs linear_ws(int64_t M, int64_t N, int64_t K, int R, int r) {
     const int KL = low_rank_width(R);
+    const int Rp = padded_rank(R);
     LinearWs w{};
     size_t o = 0;
     auto take = [&](size_t bytes) {
@@ -104,16 +119,19 @@ LinearWs linear_ws(int64_t M, int64_t N, int64_t K, int R) {
     w.qx_codes = take(static_cast<size_t>(M) * K / 2);
     w.qx_scales = take(static_cast<size_t>(M) * K / 256);
     w.qx_sf = take(static_cast<size_t>(M) * K / 16);
-    w.dn = take(static_cast<size_t>(R) * K * 2);
+    w.dn = take(static_cast<size_t>(Rp) * K * 2);
     w.upcat = take(static_cast<size_t>(N) * KL * 2);
     w.tcat = take(static_cast<size_t>(M) * KL * 2);
+    w.partial = take(static_cast<size_t>(kMaxSplits) * M * Rp * 4);
     w.qg_codes = take(static_cast<size_t>(M) * N / 2);
     w.qg_scales = take(static_cast<size_t>(M) * N / 256);
     w.qg_sf = take(static_cast<size_t>(M) * N / 16);
-    w.upt = take(static_cast<size_t>(R) * N * 2);
+    w.upt = take(static_cast<size_t>(Rp) * N * 2);
     w.dntcat = take(static_cast<size_t>(K) * KL * 2);
     w.u = take(static_cast<size_t>(M) * R * 4);
     w.ucat = take(static_cast<size_t>(M) * KL * 2);
+    w.vcat = take(static_cast<size_t>(M) * lora_width(r) * 2);
+    w.gpartial = take(static_cast<size_t>(kMaxSplits) * (N > K ? N : K) * lora_width(r) * 4);
     w.total = o;
     return w;
 }
@@ -149,17 +167,40 @@ ft_status check_layer(const ft_linear* L) {
 const __nv_bfloat16* bf(const void* p) { return static_cast<const __nv_bfloat16*>(p); }
 __nv_bfloat16* bfm(void* p) { return static_cast<__nv_bfloat16*>(p); }
 
-// Quantize a bf16 [rows, cols] operand into (codes, scales, g, sf_mma) held in the workspace.
-ft_status quantize_operand(const void* x, int64_t rows, int64_t cols, const float* amax_or_null,
+// Quantize a bf16 [rows, cols] operand into (codes, scales, g, sf_mma) and, when
+// Rp > 0, its down-projection partials x w^T (w: bf16 [Rp, cols]) in one fused kernel.
+// Returns the number of column slices (partials) through *splits.
+ft_status quantize_operand(const void* x, int64_t rows, int64_t cols, int64_t ld, const float* amax_or_null,
                            float* amax_slot, uint8_t* codes, uint8_t* scales, uint8_t* sf, float* g,
+                           const void* w, int Rp, float* partial, int* splits, int* status,
                            const DeviceInfo& dev, cudaStream_t st) {
     const float* amax = amax_or_null;
     if (!amax) {
-        FT_CUDA(ft::launch_amax(x, false, rows, cols, cols, amax_slot, dev.num_sms, st));
+        FT_CUDA(ft::launch_amax(x, false, rows, cols, ld, amax_slot, dev.num_sms, st));
         amax = amax_slot;
     }
-    FT_CUDA(ft::launch_quant_block16(x, false, rows, cols, cols, amax, codes, scales, g, dev.num_sms, st));
-    FT_CUDA(ft::launch_expand_scales(scales, rows, cols, sf, st));
+    CUtensorMap tX, tW;
+    FT_TRY(make_tmap(&tX, x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, cols, rows, ld * 2, 64, 128));
+    if (Rp > 0)
+        FT_TRY(make_tmap(&tW, w, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, cols, Rp, cols * 2, 64, Rp));
+    else
+        tW = tX;
+    const int s = ft::quant_down_splits(rows, cols, dev.num_sms);
+    ft::QuantDownArgs a{};
+    a.rows = rows;
+    a.cols = cols;
+    a.cols_per_split = static_cast<int>(cols / s);
+    a.Rp = Rp;
+    a.tmem_cols = tmem_cols_for(Rp);
+    a.amax = amax;
+    a.codes = codes;
+    a.scales = scales;
+    a.sf_mma = sf;
+    a.g_out = g;
+    a.partial = partial;
+    a.status = status;
+    FT_CUDA(ft::launch_quant_down(tX, tW, a, s, st));
+    *splits = s;
     return FT_OK;
 }
 
@@ -191,6 +232,29 @@ ft_status run_gemm(const uint8_t* a_codes, const uint8_t* a_sf, const float* ga,
     g.status = status;
     FT_CUDA(ft::launch_gemm_fp4_lowrank(tA, tB, tLA, tLB, g, dev.num_sms, st));
     return FT_OK;
+}
+
+// Quantize workspace: status word, amax slot, the down factor padded to Rp rows, and
+// the split partials of the down-projection.
+struct QuantWs {
+    size_t status, amax, down, partial, total;
+};
+
+QuantWs quant_ws(int64_t rows, int64_t cols, int r_down) {
+    const int Rp = padded_rank(r_down);
+    QuantWs w{};
+    size_t o = 0;
+    auto take = [&](size_t bytes) {
+        size_t at = o;
+        o = align_up(o + bytes, kAlign);
+        return at;
+    };
+    w.status = take(16);
+    w.amax = take(16);
+    w.down = take(static_cast<size_t>(Rp) * cols * 2);
+    w.partial = take(static_cast<size_t>(kMaxSplits) * rows * Rp * 4);
+    w.total = o;
+    return w;
 }
 
 std::atomic<uint64_t> g_launches{0};
@@ -250,10 +314,8 @@ const char* fourtune_status_string(int s) {
 }
 
 size_t fourtune_quantize_workspace_bytes(int64_t rows, int64_t cols, int32_t r_down) {
-    (void)rows;
-    (void)cols;
-    (void)r_down;
-    return 2 * kAlign;  // status word + amax slot
+    if (rows < 0 || cols < 0 || r_down < 0) return 0;
+    return quant_ws(rows, cols, r_down).total;
 }
 
 ft_status fourtune_quantize_block16(const void* x_dev, int32_t x_dtype, int64_t rows, int64_t cols,
@@ -264,57 +326,66 @@ ft_status fourtune_quantize_block16(const void* x_dev, int32_t x_dtype, int64_t 
     if (rows <= 0 || cols <= 0 || ld < cols || r_down < 0 || r_down > 256) return FT_ERR_INVALID_ARG;
     if (rows % 16 || cols % 16 || ld % 8) return FT_ERR_SHAPE;
     if (r_down > 0 && (!down_dev || !down_out_dev || x_dtype != FT_DTYPE_BF16)) return FT_ERR_INVALID_ARG;
-    if (r_down > 0 && rows % 32) return FT_ERR_SHAPE;
     FT_TRY(check_fp4(*out, rows, cols, false));
     const bool want_sf = out->sf_mma != nullptr;
+    const bool fused_ok = x_dtype == FT_DTYPE_BF16 && rows % 128 == 0 && cols % 64 == 0;
+    if (r_down > 0 && !fused_ok) return FT_ERR_SHAPE;
     if ((want_sf || out_t) && (rows % 128 || cols % 128)) return FT_ERR_SHAPE;
     if (out_t) FT_TRY(check_fp4(*out_t, cols, rows, true));
     if (!aligned16(x_dev) || (down_dev && !aligned16(down_dev)) || (down_out_dev && !aligned16(down_out_dev)))
         return FT_ERR_ALIGN;
-    if (!ws || ws_bytes < fourtune_quantize_workspace_bytes(rows, cols, r_down)) return FT_ERR_WORKSPACE;
+    const QuantWs qw = quant_ws(rows, cols, r_down);
+    if (!ws || ws_bytes < qw.total) return FT_ERR_WORKSPACE;
     if (reinterpret_cast<uintptr_t>(ws) % kAlign) return FT_ERR_ALIGN;
     DeviceInfo dev;
     FT_TRY(device_info(&dev));
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    float* amax_slot = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + kAlign);
+    uint8_t* W = static_cast<uint8_t*>(ws);
+    float* amax_slot = reinterpret_cast<float*>(W + qw.amax);
+    int* status = reinterpret_cast<int*>(W + qw.status);
     const bool f32 = x_dtype == FT_DTYPE_F32;
-    const float* amax = amax_or_null;
-    if (!amax) {
-        FT_CUDA(ft::launch_amax(x_dev, f32, rows, cols, ld, amax_slot, dev.num_sms, st));
-        amax = amax_slot;
+    if (fused_ok) {
+        const int Rp = padded_rank(r_down);
+        if (Rp > 0)
+            FT_CUDA(ft::launch_build_factors(bf(down_dev), nullptr, nullptr, nullptr, 0, cols, r_down, 0, Rp, 0,
+                                             bfm(W + qw.down), nullptr, nullptr, nullptr, st));
+        int splits = 1;
+        float* partial = reinterpret_cast<float*>(W + qw.partial);
+        FT_TRY(quantize_operand(x_dev, rows, cols, ld, amax_or_null, amax_slot, out->codes, out->scales,
+                                out->sf_mma, out->g, W + qw.down, Rp, partial, &splits, status, dev, st));
+        if (Rp > 0) {
+            ft::LowRankFinalizeArgs f{};
+            f.partial = partial;
+            f.splits = splits;
+            f.rows = rows;
+            f.Rp = Rp;
+            f.R = r_down;
+            f.r_s = r_down;
+            f.s = 1.0f;
+            f.out = down_out_dev;
+            FT_CUDA(ft::launch_lowrank_finalize(f, st));
+        }
+    } else {
+        const float* amax = amax_or_null;
+        if (!amax) {
+            FT_CUDA(ft::launch_amax(x_dev, f32, rows, cols, ld, amax_slot, dev.num_sms, st));
+            amax = amax_slot;
+        }
+        FT_CUDA(ft::launch_quant_block16(x_dev, f32, rows, cols, ld, amax, out->codes, out->scales, out->g,
+                                         dev.num_sms, st));
+        if (want_sf) FT_CUDA(ft::launch_expand_scales(out->scales, rows, cols, out->sf_mma, st));
     }
-    FT_CUDA(ft::launch_quant_block16(x_dev, f32, rows, cols, ld, amax, out->codes, out->scales, out->g,
-                                     dev.num_sms, st));
-    if (want_sf) FT_CUDA(ft::launch_expand_scales(out->scales, rows, cols, out->sf_mma, st));
     if (out_t) {
         FT_CUDA(ft::launch_transpose_q(out->codes, out->scales, rows, cols, out_t->codes, out_t->scales, st));
         FT_CUDA(ft::launch_copy_scalar(out->g, out_t->g, st));
         FT_CUDA(ft::launch_expand_scales(out_t->scales, cols, rows, out_t->sf_mma, st));
-    }
-    if (r_down > 0) {
-        // the down-projection alone: out = x down^T (fp32); its bf16 split is not needed
-        ft::LowRankDownArgs a{};
-        a.x = bf(x_dev);
-        a.ldx = ld;
-        a.M = rows;
-        a.K = cols;
-        a.w = bf(down_dev);
-        a.R = r_down;
-        a.r_s = r_down;
-        a.s = 1.0f;
-        a.ga = nullptr;
-        a.gb = nullptr;
-        a.out = down_out_dev;
-        a.cat = nullptr;
-        a.KL = 0;
-        FT_CUDA(ft::launch_lowrank_down(a, st));
     }
     return FT_OK;
 }
 
 size_t fourtune_linear_workspace_bytes(const ft_linear* L, int64_t M) {
     if (!L || M <= 0) return 0;
-    return linear_ws(M, L->N, L->K, L->r_s + L->r).total;
+    return linear_ws(M, L->N, L->K, L->r_s + L->r, L->r).total;
 }
 
 ft_status fourtune_linear_fwd(const ft_linear* L, const void* x_dev, int64_t M, const float* amax_or_null,
@@ -324,7 +395,7 @@ ft_status fourtune_linear_fwd(const ft_linear* L, const void* x_dev, int64_t M, 
     if (!x_dev || !y_dev || (R > 0 && !t_saved_dev) || M <= 0) return FT_ERR_INVALID_ARG;
     if (M % 128) return FT_ERR_SHAPE;
     if (!aligned16(x_dev) || !aligned16(y_dev) || (t_saved_dev && !aligned16(t_saved_dev))) return FT_ERR_ALIGN;
-    const LinearWs w = linear_ws(M, L->N, L->K, R);
+    const LinearWs w = linear_ws(M, L->N, L->K, R, L->r);
     if (!ws || ws_bytes < w.total) return FT_ERR_WORKSPACE;
     if (reinterpret_cast<uintptr_t>(ws) % kAlign) return FT_ERR_ALIGN;
     DeviceInfo dev;
@@ -335,28 +406,34 @@ ft_status fourtune_linear_fwd(const ft_linear* L, const void* x_dev, int64_t M, 
     int* status = reinterpret_cast<int*>(W + w.status);
     const int64_t N = L->N, K = L->K;
     const int KL = low_rank_width(R);
+    const int Rp = padded_rank(R);
+    float* partial = reinterpret_cast<float*>(W + w.partial);
 
-    FT_TRY(quantize_operand(x_dev, M, K, amax_or_null, scal + SC_AMAX_X, W + w.qx_codes, W + w.qx_scales,
-                            W + w.qx_sf, scal + SC_G_X, dev, st));
-    if (R > 0) {
+    // Eq. (2): the factors of this step ([Ls_down; A] and [Ls_up, B]; A, B train),
+    // then Q(X) fused with T = X [Ls_down; A]^T, then the 4-bit GEMM with the
+    // up-projections in its accumulator.
+    if (R > 0)
         FT_CUDA(ft::launch_build_factors(bf(L->ls_down), bf(L->lora_a), bf(L->ls_up), bf(L->lora_b), N, K,
-                                         L->r_s, L->r, KL, bfm(W + w.dn), bfm(W + w.upcat), nullptr, nullptr,
-                                         st));
-        ft::LowRankDownArgs a{};
-        a.x = bf(x_dev);
-        a.ldx = K;
-        a.M = M;
-        a.K = K;
-        a.w = bf(W + w.dn);
-        a.R = R;
-        a.r_s = L->r_s;
-        a.s = L->lora_scale;
-        a.ga = scal + SC_G_X;
-        a.gb = L->qr.g;
-        a.out = t_saved_dev;
-        a.cat = bfm(W + w.tcat);
-        a.KL = KL;
-        FT_CUDA(ft::launch_lowrank_down(a, st));
+                                         L->r_s, L->r, Rp, KL, bfm(W + w.dn), bfm(W + w.upcat), nullptr,
+                                         nullptr, st));
+    int splits = 1;
+    FT_TRY(quantize_operand(x_dev, M, K, K, amax_or_null, scal + SC_AMAX_X, W + w.qx_codes, W + w.qx_scales,
+                            W + w.qx_sf, scal + SC_G_X, W + w.dn, Rp, partial, &splits, status, dev, st));
+    if (R > 0) {
+        ft::LowRankFinalizeArgs f{};
+        f.partial = partial;
+        f.splits = splits;
+        f.rows = M;
+        f.Rp = Rp;
+        f.R = R;
+        f.r_s = L->r_s;
+        f.s = L->lora_scale;
+        f.ga = scal + SC_G_X;
+        f.gb = L->qr.g;
+        f.out = t_saved_dev;
+        f.cat = bfm(W + w.tcat);
+        f.KL = KL;
+        FT_CUDA(ft::launch_lowrank_finalize(f, st));
     }
     return run_gemm(W + w.qx_codes, W + w.qx_sf, scal + SC_G_X, L->qr, bf(W + w.tcat), bf(W + w.upcat), KL, M,
                     N, K, y_dev, status, dev, st);
@@ -374,7 +451,7 @@ ft_status fourtune_linear_bwd(const ft_linear* L, const void* x_dev, const float
         (t_saved_dev && !aligned16(t_saved_dev)) || (da_dev && !aligned16(da_dev)) ||
         (db_dev && !aligned16(db_dev)))
         return FT_ERR_ALIGN;
-    const LinearWs w = linear_ws(M, L->N, L->K, R);
+    const LinearWs w = linear_ws(M, L->N, L->K, R, L->r);
     if (!ws || ws_bytes < w.total) return FT_ERR_WORKSPACE;
     if (reinterpret_cast<uintptr_t>(ws) % kAlign) return FT_ERR_ALIGN;
     DeviceInfo dev;
@@ -385,35 +462,66 @@ ft_status fourtune_linear_bwd(const ft_linear* L, const void* x_dev, const float
     int* status = reinterpret_cast<int*>(W + w.status);
     const int64_t N = L->N, K = L->K;
     const int KL = low_rank_width(R);
-
-    FT_TRY(quantize_operand(dy_dev, M, N, amax_or_null, scal + SC_AMAX_G, W + w.qg_codes, W + w.qg_scales,
-                            W + w.qg_sf, scal + SC_G_G, dev, st));
+    const int Rp = padded_rank(R);
+    float* partial = reinterpret_cast<float*>(W + w.partial);
     float* U = reinterpret_cast<float*>(W + w.u);
-    if (R > 0) {
+
+    // Eq. (3): Q(G) fused with U = G [Ls_up, B], the dX GEMM through Q(R)^T with
+    // U [Ls_down; A] in its accumulator, then the adapter gradients.
+    if (R > 0)
         FT_CUDA(ft::launch_build_factors(bf(L->ls_down), bf(L->lora_a), bf(L->ls_up), bf(L->lora_b), N, K,
-                                         L->r_s, L->r, KL, nullptr, nullptr, bfm(W + w.upt),
+                                         L->r_s, L->r, Rp, KL, nullptr, nullptr, bfm(W + w.upt),
                                          bfm(W + w.dntcat), st));
-        ft::LowRankDownArgs a{};
-        a.x = bf(dy_dev);
-        a.ldx = N;
-        a.M = M;
-        a.K = N;
-        a.w = bf(W + w.upt);
-        a.R = R;
-        a.r_s = L->r_s;
-        a.s = L->lora_scale;
-        a.ga = scal + SC_G_G;
-        a.gb = L->qr_t.g;
-        a.out = U;
-        a.cat = bfm(W + w.ucat);
-        a.KL = KL;
-        FT_CUDA(ft::launch_lowrank_down(a, st));
+    int splits = 1;
+    FT_TRY(quantize_operand(dy_dev, M, N, N, amax_or_null, scal + SC_AMAX_G, W + w.qg_codes, W + w.qg_scales,
+                            W + w.qg_sf, scal + SC_G_G, W + w.upt, Rp, partial, &splits, status, dev, st));
+    if (R > 0) {
+        ft::LowRankFinalizeArgs f{};
+        f.partial = partial;
+        f.splits = splits;
+        f.rows = M;
+        f.Rp = Rp;
+        f.R = R;
+        f.r_s = L->r_s;
+        f.s = L->lora_scale;
+        f.ga = scal + SC_G_G;
+        f.gb = L->qr_t.g;
+        f.out = U;
+        f.cat = bfm(W + w.ucat);
+        f.KL = KL;
+        FT_CUDA(ft::launch_lowrank_finalize(f, st));
     }
     FT_TRY(run_gemm(W + w.qg_codes, W + w.qg_sf, scal + SC_G_G, L->qr_t, bf(W + w.ucat), bf(W + w.dntcat), KL,
                     M, K, N, dx_dev, status, dev, st));
     if (L->r > 0) {
-        FT_CUDA(ft::launch_lora_db(bf(dy_dev), M, N, t_saved_dev, R, L->r_s, L->r, L->lora_scale, db_dev, st));
-        FT_CUDA(ft::launch_lora_da(U, R, L->r_s, L->r, bf(x_dev), M, K, L->lora_scale, da_dev, st));
+        // Section 3.2 adapter gradients: dB = s G^T T_lora, dA = s U_lora^T X, on the
+        // tensor cores, reading G and X straight (MN-major operands).
+        const int NBW = lora_width(L->r);
+        __nv_bfloat16* vcat = bfm(W + w.vcat);
+        float* gpart = reinterpret_cast<float*>(W + w.gpartial);
+        CUtensorMap tP, tV;
+        FT_TRY(make_tmap(&tV, vcat, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, NBW, M, NBW * 2, 64, 64));
+        ft::LoraGradArgs g{};
+        g.NBW = NBW;
+        g.tmem_cols = tmem_cols_for(NBW);
+        g.partial = gpart;
+        g.status = status;
+        // dB over the output features n
+        FT_CUDA(ft::launch_build_hilo(t_saved_dev, R, L->r_s, L->r, M, NBW, vcat, st));
+        FT_TRY(make_tmap(&tP, dy_dev, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, N, M, N * 2, 64, 64));
+        int sp = ft::lora_grad_splits(M, N, dev.num_sms);
+        g.F = N;
+        g.tokens_per_split = static_cast<int>(M / sp);
+        FT_CUDA(ft::launch_lora_grad(tP, tV, g, sp, ft::K_LORA_DB, st));
+        FT_CUDA(ft::launch_lora_grad_finalize(gpart, sp, N, NBW, L->r, L->lora_scale, false, db_dev, st));
+        // dA over the input features k
+        FT_CUDA(ft::launch_build_hilo(U, R, L->r_s, L->r, M, NBW, vcat, st));
+        FT_TRY(make_tmap(&tP, x_dev, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, K, M, K * 2, 64, 64));
+        sp = ft::lora_grad_splits(M, K, dev.num_sms);
+        g.F = K;
+        g.tokens_per_split = static_cast<int>(M / sp);
+        FT_CUDA(ft::launch_lora_grad(tP, tV, g, sp, ft::K_LORA_DA, st));
+        FT_CUDA(ft::launch_lora_grad_finalize(gpart, sp, K, NBW, L->r, L->lora_scale, true, da_dev, st));
     }
     return FT_OK;
 }

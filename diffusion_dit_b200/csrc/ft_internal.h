@@ -64,17 +64,65 @@ struct LowRankDownArgs {
 };
 cudaError_t launch_lowrank_down(const LowRankDownArgs& a, cudaStream_t stream);
 
+// Fused quantizer + down-projection (ft_quant_fused.cu).
+struct QuantDownArgs {
+    int64_t rows, cols;      // input [rows, cols]; rows % 128 == 0, cols % 64 == 0
+    int cols_per_split;      // columns per CTA slice (multiple of 64)
+    int Rp;                  // down-projection width (multiple of 16, <= 256; 0 = none)
+    uint32_t tmem_cols;      // TMEM columns to allocate (power of two >= max(32, Rp))
+    const float* amax;       // tensor max used for g
+    uint8_t* codes;          // [rows, cols/2]
+    uint8_t* scales;         // [rows/16, cols/16]
+    uint8_t* sf_mma;         // tensor-core scale layout or null
+    float* g_out;
+    float* partial;          // [splits, rows, Rp] fp32
+    int* status;
+};
+int quant_down_splits(int64_t rows, int64_t cols, int num_sms);
+size_t quant_down_smem_bytes(int Rp);
+cudaError_t launch_quant_down(const CUtensorMap& tmX, const CUtensorMap& tmW, const QuantDownArgs& a,
+                              int splits, cudaStream_t stream);
+
+// Sums the split partials in a fixed order and emits out (fp32 [rows, R], may be null)
+// and the 4-bit GEMM's low-rank operand cat (bf16 [rows, KL], may be null).
+struct LowRankFinalizeArgs {
+    const float* partial;    // [splits, rows, Rp]
+    int splits;
+    int64_t rows;
+    int Rp, R, r_s;
+    float s;
+    const float* ga;
+    const float* gb;
+    float* out;
+    __nv_bfloat16* cat;
+    int KL;
+};
+cudaError_t launch_lowrank_finalize(const LowRankFinalizeArgs& a, cudaStream_t stream);
+
 // Build the concatenated low-rank factors used by the forward and backward GEMMs.
+// dn and upt get Rp rows (rows R..Rp-1 zero) so they can feed an MMA of width Rp.
 cudaError_t launch_build_factors(const __nv_bfloat16* ls_down, const __nv_bfloat16* lora_a,
                                  const __nv_bfloat16* ls_up, const __nv_bfloat16* lora_b, int64_t N,
-                                 int64_t K, int r_s, int r, int KL, __nv_bfloat16* dn,
+                                 int64_t K, int r_s, int r, int Rp, int KL, __nv_bfloat16* dn,
                                  __nv_bfloat16* upcat, __nv_bfloat16* upt, __nv_bfloat16* dntcat,
                                  cudaStream_t stream);
 
-// adapter gradients (ft_lowrank.cu)
-cudaError_t launch_lora_db(const __nv_bfloat16* g, int64_t M, int64_t N, const float* t, int R,
-                           int r_s, int r, float s, float* db, cudaStream_t stream);
-cudaError_t launch_lora_da(const float* u, int R, int r_s, int r, const __nv_bfloat16* x, int64_t M,
-                           int64_t K, float s, float* da, cudaStream_t stream);
+// adapter gradients on the tensor cores (ft_lora_grad.cu):
+//   partial[split][f][c] = sum over the split's tokens m of P[m, f] V'[m, c]
+struct LoraGradArgs {
+    int64_t F;               // features of P [M, F] (multiple of 128)
+    int tokens_per_split;    // multiple of 64
+    int NBW;                 // width of V' = [hi, lo, 0] (multiple of 64, <= 256)
+    uint32_t tmem_cols;      // power of two >= max(32, NBW)
+    float* partial;          // [splits, F, NBW]
+    int* status;
+};
+int lora_grad_splits(int64_t M, int64_t F, int num_sms);
+cudaError_t launch_lora_grad(const CUtensorMap& tmP, const CUtensorMap& tmV, const LoraGradArgs& a, int splits,
+                             int kind, cudaStream_t stream);
+cudaError_t launch_lora_grad_finalize(const float* partial, int splits, int64_t F, int NBW, int r, float s,
+                                      bool transpose_out, float* out, cudaStream_t stream);
+cudaError_t launch_build_hilo(const float* src, int64_t ld, int c0, int r, int64_t M, int NBW,
+                              __nv_bfloat16* dst, cudaStream_t stream);
 
 }  // namespace ft

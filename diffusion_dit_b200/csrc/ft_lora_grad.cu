@@ -1,0 +1,250 @@
+// Adapter weight gradients on the tensor cores (FourTune, arXiv 2607.05711, section
+// 3.2: weight gradients exist only for the adapter branch):
+//   dB [N, r] = s G^T T_lora          (T_lora = X A^T, saved by the forward)
+//   dA [r, K] = s U_lora^T X          (U_lora = G B, from the backward down-projection)
+// Both are contractions over the tokens m of a big bf16 operand P [M, F] (G or X,
+// row-major: F contiguous) with a small operand V [M, r]:
+//   D[f, c] = sum_m P[m, f] V'[m, c]
+// The 128 x 64 tile of P that TMA puts in shared memory (rows = tokens) is exactly
+// the MN-major layout the MMA wants for an A operand indexed (f, m), so P is read once,
+// straight, with no transpose.  V' = [hi(V), lo(V), 0] (bf16, width NBW = 2r rounded
+// up to 64) is MN-major too; the hi and lo halves land in separate accumulator
+// columns and are added in the final sum, keeping ~16 mantissa bits of V.
+//
+// One CTA = 128 features x a slice of the tokens; partials[split][f][NBW] fp32 are
+// summed in a fixed order by lora_grad_finalize_kernel (deterministic).
+#include "ft_internal.h"
+#include "ft_ptx.cuh"
+
+namespace ft {
+namespace lg {
+
+constexpr int BF = 128;                 // features per CTA (MMA M)
+constexpr int BMT = 64;                 // tokens per stage
+constexpr int A_BYTES = BMT * BF * 2;   // 16 KB: two 64-feature boxes of [64 tokens x 128 B]
+constexpr int THREADS = 192;            // producer, MMA, 4 epilogue warps
+constexpr int MAX_STAGES = 8;
+constexpr int BAR_BYTES = 256;
+
+struct Layout {
+    int stages, stage_bytes, smem_bytes;
+};
+
+__host__ __device__ inline Layout layout_for(int NBW) {
+    Layout L;
+    L.stage_bytes = A_BYTES + BMT * NBW * 2;
+    int s = (192 * 1024) / L.stage_bytes;
+    if (s > 6) s = 6;
+    if (s < 2) s = 2;
+    L.stages = s;
+    L.smem_bytes = s * L.stage_bytes + BAR_BYTES + 1024;
+    return L;
+}
+
+__global__ void __launch_bounds__(THREADS, 1)
+    lora_grad_kernel(const __grid_constant__ CUtensorMap tmP, const __grid_constant__ CUtensorMap tmV,
+                     const LoraGradArgs p) {
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw_u32 = smem_u32(smem_raw);
+    const uint32_t pad = (1024 - (raw_u32 & 1023)) & 1023;
+    const uint32_t base_u32 = raw_u32 + pad;
+    uint8_t* base = smem_raw + pad;
+    const Layout L = layout_for(p.NBW);
+    const int S = L.stages;
+    uint8_t* bar_area = base + S * L.stage_bytes;
+    auto bar = [&](int i) { return base_u32 + S * L.stage_bytes + 8 * i; };
+    volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(bar_area + 8 * (2 * MAX_STAGES + 2));
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(bar_area + 8 * (2 * MAX_STAGES + 2) + 4);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int f0 = blockIdx.x * BF;
+    const int split = blockIdx.y;
+    const int m0 = split * p.tokens_per_split;
+    const int nk = p.tokens_per_split / BMT;
+    const int nchunk = p.NBW / 64;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < S; ++i) {
+            mbar_init(bar(i), 1);
+            mbar_init(bar(S + i), 1);
+        }
+        mbar_init(bar(2 * S), 1);
+        mbar_init(bar(2 * S + 1), 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+        fence_proxy_async_smem();
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&tmP);
+        tma_prefetch_desc(&tmV);
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_u32(const_cast<uint32_t*>(tmem_slot)), p.tmem_cols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            const uint32_t tx = L.stage_bytes;
+            int k = 0;
+            for (; k < nk; ++k) {
+                const int s = k % S;
+                if (!mbar_wait(bar(S + s), ((k / S) & 1) ^ 1, abort_flag, p.status)) break;
+                const uint32_t st = base_u32 + s * L.stage_bytes;
+                mbar_arrive_expect_tx(bar(s), tx);
+                const int mm = m0 + k * BMT;
+                tma_load_2d(st, &tmP, bar(s), f0, mm);
+                tma_load_2d(st + A_BYTES / 2, &tmP, bar(s), f0 + 64, mm);
+                for (int c = 0; c < nchunk; ++c)
+                    tma_load_2d(st + A_BYTES + c * (BMT * 128), &tmV, bar(s), 64 * c, mm);
+            }
+            for (int j = k - 1; j >= 0 && j >= k - S; --j) {
+                volatile int no_abort = 0;
+                mbar_wait(bar(j % S), (j / S) & 1, &no_abort, p.status);
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            const uint32_t idesc = idesc_bf16(BF, p.NBW, /*a_mn=*/true, /*b_mn=*/true);
+            for (int k = 0; k < nk; ++k) {
+                const int s = k % S;
+                if (!mbar_wait(bar(s), (k / S) & 1, abort_flag, p.status)) break;
+                tc_fence_after();
+                const uint32_t st = base_u32 + s * L.stage_bytes;
+                // MN-major, 128-byte swizzle: 8-token groups 1024 B apart (SBO); the two
+                // 64-feature halves of A (and the 64-column chunks of V) 8 KB apart (LBO).
+                const uint64_t ad = sdesc_mnmajor_sw128(st, A_BYTES / 2, 1024);
+                const uint64_t bd = sdesc_mnmajor_sw128(st + A_BYTES, BMT * 128, 1024);
+#pragma unroll
+                for (int i = 0; i < BMT / 16; ++i)  // 16 tokens per MMA = two 8-row groups
+                    mma_bf16(tmem, ad + (2048 >> 4) * i, bd + (2048 >> 4) * i, idesc, (k | i) != 0);
+                tc_commit(bar(S + s));
+            }
+            tc_commit(bar(2 * S));
+            tc_commit(bar(2 * S + 1));
+            volatile int no_abort = 0;
+            mbar_wait(bar(2 * S + 1), 0, &no_abort, p.status);
+        }
+    } else {
+        const int q = warp & 3;
+        if (mbar_wait(bar(2 * S), 0, abort_flag, p.status)) {
+            tc_fence_after();
+            const int f = f0 + 32 * q + lane;
+            float* dst = p.partial + (static_cast<int64_t>(split) * p.F + f) * p.NBW;
+            for (int c = 0; c < p.NBW; c += 32) {
+                uint32_t v[32];
+                tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(32 * q) << 16) + c, v);
+                tmem_ld_wait();
+#pragma unroll
+                for (int e = 0; e < 32; e += 4)
+                    *reinterpret_cast<float4*>(dst + c + e) =
+                        make_float4(__uint_as_float(v[e]), __uint_as_float(v[e + 1]),
+                                    __uint_as_float(v[e + 2]), __uint_as_float(v[e + 3]));
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tmem, p.tmem_cols);
+}
+
+// out = s * sum_split (D[f][j] + D[f][r + j]); transposed (out[j][f]) for dA.
+__global__ void lora_grad_finalize_kernel(const float* __restrict__ partial, int splits, int64_t F, int NBW,
+                                          int r, float s, bool transpose_out, float* __restrict__ out) {
+    const int64_t total = F * r;
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        int64_t f, j;
+        if (transpose_out) {  // consecutive threads walk f for coalesced stores into out[j][f]
+            j = i / F;
+            f = i % F;
+        } else {
+            f = i / r;
+            j = i % r;
+        }
+        float v = 0.0f;
+        for (int sp = 0; sp < splits; ++sp) {
+            const float* d = partial + (static_cast<int64_t>(sp) * F + f) * NBW;
+            v += d[j] + d[r + j];
+        }
+        v *= s;
+        if (transpose_out)
+            out[j * F + f] = v;
+        else
+            out[f * r + j] = v;
+    }
+}
+
+// V' [M, NBW] bf16 = [hi(V), lo(V), 0] from fp32 V = src[:, c0 : c0 + r] (row stride ld).
+__global__ void build_hilo_kernel(const float* __restrict__ src, int64_t ld, int c0, int r, int64_t M, int NBW,
+                                  __nv_bfloat16* __restrict__ dst) {
+    const int64_t total = M * NBW;
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t m = i / NBW;
+        const int c = static_cast<int>(i % NBW);
+        __nv_bfloat16 o = __float2bfloat16_rn(0.0f);
+        if (c < 2 * r) {
+            const float v = src[m * ld + c0 + (c < r ? c : c - r)];
+            const __nv_bfloat16 hi = __float2bfloat16_rn(v);
+            o = c < r ? hi : __float2bfloat16_rn(v - __bfloat162float(hi));
+        }
+        dst[i] = o;
+    }
+}
+
+}  // namespace lg
+
+int lora_grad_splits(int64_t M, int64_t F, int num_sms) {
+    const int64_t tiles = F / lg::BF;
+    const int64_t chunks = M / lg::BMT;
+    // as many token slices as fill the SMs once, dividing the token chunks evenly
+    int64_t s = tiles > 0 ? num_sms / tiles : 1;
+    if (s < 1) s = 1;
+    if (s > 16) s = 16;
+    while (s > 1 && chunks % s) --s;
+    return static_cast<int>(s);
+}
+
+cudaError_t launch_lora_grad(const CUtensorMap& tmP, const CUtensorMap& tmV, const LoraGradArgs& a, int splits,
+                             int kind, cudaStream_t stream) {
+    const lg::Layout L = lg::layout_for(a.NBW);
+    cudaError_t e = cudaFuncSetAttribute(lg::lora_grad_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         L.smem_bytes);
+    if (e != cudaSuccess) return e;
+    dim3 grid(static_cast<unsigned>(a.F / lg::BF), static_cast<unsigned>(splits));
+    before_launch(kind, stream);
+    lg::lora_grad_kernel<<<grid, lg::THREADS, L.smem_bytes, stream>>>(tmP, tmV, a);
+    after_launch(kind, stream);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_lora_grad_finalize(const float* partial, int splits, int64_t F, int NBW, int r, float s,
+                                      bool transpose_out, float* out, cudaStream_t stream) {
+    int64_t g = (F * r + 255) / 256;
+    if (g > 148 * 8) g = 148 * 8;
+    before_launch(K_OTHER, stream);
+    lg::lora_grad_finalize_kernel<<<static_cast<unsigned>(g), 256, 0, stream>>>(partial, splits, F, NBW, r, s,
+                                                                                 transpose_out, out);
+    after_launch(K_OTHER, stream);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_build_hilo(const float* src, int64_t ld, int c0, int r, int64_t M, int NBW,
+                              __nv_bfloat16* dst, cudaStream_t stream) {
+    int64_t g = (M * NBW + 255) / 256;
+    if (g > 148 * 8) g = 148 * 8;
+    before_launch(K_OTHER, stream);
+    lg::build_hilo_kernel<<<static_cast<unsigned>(g), 256, 0, stream>>>(src, ld, c0, r, M, NBW, dst);
+    after_launch(K_OTHER, stream);
+    return cudaGetLastError();
+}
+
+}  // namespace ft

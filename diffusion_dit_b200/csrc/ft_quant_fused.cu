@@ -1,0 +1,266 @@
+// Fused 16x16-block quantizer + low-rank down-projection (FourTune, arXiv 2607.05711,
+// section 3.3 "LoRA Fusion": the quantizer and the stabilizer / LoRA down-projections
+// share the same input, so they run as one kernel that reads it once).
+//
+// For a bf16 input X [rows, cols] and a bf16 down factor W [Rp, cols] (Rp = the rank
+// rounded up to 16, extra rows zero) one CTA takes a 128-row band and a slice of the
+// columns.  Each 128 x 64 tile arrives by TMA (128-byte swizzle) into a shared-memory
+// ring and is consumed twice:
+//   * the MMA warp multiplies it with the matching W tile on the tensor cores
+//     (tcgen05.mma kind::f16, accumulator [128 x Rp] fp32 in TMEM), giving this CTA's
+//     partial of T = X W^T;
+//   * eight quantizer warps read the same tile from shared memory and emit the E2M1
+//     codes, the compact block scales and the tensor-core scale layout (same
+//     arithmetic, bit for bit, as quant_block16_kernel in ft_quant.cu).
+// A stage is released when the MMA has finished reading it (tcgen05.commit) and all
+// eight quantizer warps have arrived.  At the end four warps drain the accumulator
+// into partials[split][row][Rp]; ft_lowrank.cu sums the splits in a fixed order.
+#include "ft_internal.h"
+#include "ft_ptx.cuh"
+
+namespace ft {
+namespace qf {
+
+constexpr int BM = 128;
+constexpr int BKE = 64;                 // bf16 columns per stage (one 128-byte row)
+constexpr int X_BYTES = BM * 128;       // 16 KB
+constexpr int NQ = 8;                   // quantizer warps
+constexpr int THREADS = 32 * (2 + NQ);  // producer, MMA, quantizers
+constexpr int MAX_STAGES = 8;
+constexpr int BAR_BYTES = 256;
+
+struct Layout {
+    int stages;
+    int stage_bytes;
+    int smem_bytes;
+};
+
+__host__ __device__ inline Layout layout_for(int Rp) {
+    Layout L;
+    L.stage_bytes = X_BYTES + Rp * 128;
+    int s = (200 * 1024) / L.stage_bytes;
+    if (s > 6) s = 6;
+    if (s < 2) s = 2;
+    L.stages = s;
+    L.smem_bytes = s * L.stage_bytes + BAR_BYTES + 1024;
+    return L;
+}
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
+}
+
+__global__ void __launch_bounds__(THREADS, 1)
+    quant_down_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
+                      const QuantDownArgs p) {
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw_u32 = smem_u32(smem_raw);
+    const uint32_t pad = (1024 - (raw_u32 & 1023)) & 1023;
+    uint8_t* base = smem_raw + pad;
+    const uint32_t base_u32 = raw_u32 + pad;
+    const Layout L = layout_for(p.Rp);
+    const int S = L.stages;
+    uint8_t* bar_area = base + S * L.stage_bytes;
+    auto bar = [&](int i) { return base_u32 + S * L.stage_bytes + 8 * i; };
+    // barriers: full[0..S), empty[S..2S), tmem_full 2S, final 2S+1
+    volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(bar_area + 8 * (2 * MAX_STAGES + 2));
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(bar_area + 8 * (2 * MAX_STAGES + 2) + 4);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int band = blockIdx.x;
+    const int split = blockIdx.y;
+    const int64_t row0 = static_cast<int64_t>(band) * BM;
+    const int64_t col0 = static_cast<int64_t>(split) * p.cols_per_split;
+    const int nk = p.cols_per_split / BKE;
+    const bool has_mma = p.Rp > 0;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < S; ++i) {
+            mbar_init(bar(i), 1);
+            mbar_init(bar(S + i), NQ + (has_mma ? 1 : 0));
+        }
+        mbar_init(bar(2 * S), 1);
+        mbar_init(bar(2 * S + 1), 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+        fence_proxy_async_smem();
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&tmX);
+        if (has_mma) tma_prefetch_desc(&tmW);
+    }
+    if (warp == 1 && has_mma) {
+        tmem_alloc(smem_u32(const_cast<uint32_t*>(tmem_slot)), p.tmem_cols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = has_mma ? *tmem_slot : 0;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            const uint32_t tx = X_BYTES + p.Rp * 128;
+            int k = 0;
+            for (; k < nk; ++k) {
+                const int s = k % S;
+                if (!mbar_wait(bar(S + s), ((k / S) & 1) ^ 1, abort_flag, p.status)) break;
+                const uint32_t st = base_u32 + s * L.stage_bytes;
+                mbar_arrive_expect_tx(bar(s), tx);
+                const int c = static_cast<int>(col0) + k * BKE;
+                tma_load_2d(st, &tmX, bar(s), c, static_cast<int>(row0));
+                if (has_mma) tma_load_2d(st + X_BYTES, &tmW, bar(s), c, 0);
+            }
+            for (int j = k - 1; j >= 0 && j >= k - S; --j) {
+                volatile int no_abort = 0;
+                mbar_wait(bar(j % S), (j / S) & 1, &no_abort, p.status);
+            }
+        }
+    } else if (warp == 1) {
+        if (has_mma && lane == 0) {
+            const uint32_t idesc = idesc_bf16(BM, p.Rp);
+            for (int k = 0; k < nk; ++k) {
+                const int s = k % S;
+                if (!mbar_wait(bar(s), (k / S) & 1, abort_flag, p.status)) break;
+                tc_fence_after();
+                const uint32_t st = base_u32 + s * L.stage_bytes;
+                const uint64_t ad = sdesc_kmajor_sw128(st);
+                const uint64_t bd = sdesc_kmajor_sw128(st + X_BYTES);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) mma_bf16(tmem, ad + 2 * i, bd + 2 * i, idesc, (k | i) != 0);
+                tc_commit(bar(S + s));
+            }
+            tc_commit(bar(2 * S));
+            tc_commit(bar(2 * S + 1));
+            volatile int no_abort = 0;
+            mbar_wait(bar(2 * S + 1), 0, &no_abort, p.status);
+        }
+    } else {
+        // ---------------------------------------------------------------- quantizers
+        const int qw = warp - 2;  // block-row of 16 inside the 128-row band
+        float g = 1.0f;
+        bool degenerate = true;
+        {
+            const float amax = *p.amax;
+            if (amax > 0.0f) {
+                const float gg = __fdiv_rn(2688.0f, amax);
+                if (isfinite(gg) && gg > 0.0f) {
+                    g = gg;
+                    degenerate = false;
+                }
+            }
+        }
+        if (band == 0 && split == 0 && threadIdx.x == 64) *p.g_out = g;
+        const int rr = qw * 16 + (lane >> 1);  // row inside the band
+        const int h = lane & 1;
+        const int64_t row = row0 + rr;
+        const int64_t cbs = p.cols / 16;
+        const int64_t atoms_per_band = p.cols / 64;
+        for (int k = 0; k < nk; ++k) {
+            const int s = k % S;
+            if (!mbar_wait(bar(s), (k / S) & 1, abort_flag, p.status)) break;
+            const uint8_t* tile = base + s * L.stage_bytes;
+            const int64_t c0 = col0 + k * BKE;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int chunk = (2 * j + h) ^ (rr & 7);
+                const uint4 w = *reinterpret_cast<const uint4*>(tile + rr * 128 + chunk * 16);
+                float v[8];
+                v[0] = bf16lo_to_f32(w.x); v[1] = bf16hi_to_f32(w.x);
+                v[2] = bf16lo_to_f32(w.y); v[3] = bf16hi_to_f32(w.y);
+                v[4] = bf16lo_to_f32(w.z); v[5] = bf16hi_to_f32(w.z);
+                v[6] = bf16lo_to_f32(w.w); v[7] = bf16hi_to_f32(w.w);
+                float am = 0.0f;
+#pragma unroll
+                for (int e = 0; e < 8; ++e) am = fmaxf(am, fabsf(v[e]));
+                am = warp_max(am);
+                uint32_t sb = 0, packed = 0;
+                if (!degenerate) {
+                    sb = cvt_ue4m3(__fmul_rn(__fdiv_rn(am, 6.0f), g));
+                    if (sb != 0) {
+                        const float inv = __fdiv_rn(g, ue4m3_to_f32(sb));
+#pragma unroll
+                        for (int e = 0; e < 4; ++e)
+                            packed |= cvt_e2m1x2(__fmul_rn(v[2 * e], inv), __fmul_rn(v[2 * e + 1], inv))
+                                      << (8 * e);
+                    }
+                }
+                const int64_t col = c0 + 16 * j + 8 * h;
+                *reinterpret_cast<uint32_t*>(p.codes + row * (p.cols / 2) + col / 2) = packed;
+                const int64_t cb = c0 / 16 + j;
+                if (lane == 0) p.scales[(row / 16) * cbs + cb] = static_cast<uint8_t>(sb);
+                if (p.sf_mma && h == 0) {
+                    const int m = rr;  // row inside the 128-row band
+                    const int64_t atom = static_cast<int64_t>(band) * atoms_per_band + c0 / 64;
+                    p.sf_mma[atom * 512 + 16 * (m % 32) + 4 * (m / 32) + (cb % 4)] = static_cast<uint8_t>(sb);
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(S + s));
+        }
+        // ------------------------------------------------------------ T partial epilogue
+        if (has_mma && qw < 4) {
+            const int q = warp & 3;
+            if (mbar_wait(bar(2 * S), 0, abort_flag, p.status)) {
+                tc_fence_after();
+                const int64_t orow = row0 + 32 * q + lane;
+                float* dst = p.partial + (static_cast<int64_t>(split) * p.rows + orow) * p.Rp;
+                for (int c = 0; c < p.Rp; c += 16) {
+                    uint32_t v[16];
+                    asm volatile(
+                        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+                        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+                        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]),
+                          "=r"(v[6]), "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]),
+                          "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
+                        : "r"(tmem + (static_cast<uint32_t>(32 * q) << 16) + c));
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int e = 0; e < 16; e += 4)
+                        *reinterpret_cast<float4*>(dst + c + e) =
+                            make_float4(__uint_as_float(v[e]), __uint_as_float(v[e + 1]),
+                                        __uint_as_float(v[e + 2]), __uint_as_float(v[e + 3]));
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1 && has_mma) tmem_dealloc(tmem, p.tmem_cols);
+}
+
+}  // namespace qf
+
+int quant_down_splits(int64_t rows, int64_t cols, int num_sms) {
+    // Enough CTAs to cover the SMs once: split the columns of each 128-row band into
+    // slices of whole 64-column tiles.
+    const int64_t bands = rows / 128;
+    const int64_t tiles = cols / 64;
+    int64_t s = bands > 0 ? num_sms / bands : 1;
+    if (s < 1) s = 1;
+    if (s > 16) s = 16;
+    while (s > 1 && tiles % s) --s;
+    return static_cast<int>(s);
+}
+
+size_t quant_down_smem_bytes(int Rp) { return static_cast<size_t>(qf::layout_for(Rp).smem_bytes); }
+
+cudaError_t launch_quant_down(const CUtensorMap& tmX, const CUtensorMap& tmW, const QuantDownArgs& a,
+                              int splits, cudaStream_t stream) {
+    const qf::Layout L = qf::layout_for(a.Rp);
+    cudaError_t e = cudaFuncSetAttribute(qf::quant_down_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         L.smem_bytes);
+    if (e != cudaSuccess) return e;
+    dim3 grid(static_cast<unsigned>(a.rows / 128), static_cast<unsigned>(splits));
+    before_launch(K_QUANT, stream);
+    qf::quant_down_kernel<<<grid, qf::THREADS, L.smem_bytes, stream>>>(tmX, tmW, a);
+    after_launch(K_QUANT, stream);
+    return cudaGetLastError();
+}
+
+}  // namespace ft

@@ -292,7 +292,11 @@ def launch_count() -> int:
 
 def time_next_launch(kind: int, before: Optional[torch.cuda.Event], after: Optional[torch.cuda.Event]):
     """Have the library record ``before``/``after`` (timing events) around its next
-    launch of kernel ``kind`` (FT_KERNEL_*), on that launch's stream."""
+    launch of kernel ``kind`` (FT_KERNEL_*), on that launch's stream.  The events must
+    already exist (torch creates a CUDA event at its first record())."""
+    for e in (before, after):
+        if e is not None and not e.cuda_event:
+            raise ValueError("record the event once before handing it to the library")
     b = ctypes.c_void_p(before.cuda_event) if before is not None else None
     a = ctypes.c_void_p(after.cuda_event) if after is not None else None
     _check("fourtune_time_next_launch", lib().fourtune_time_next_launch(kind, b, a))
