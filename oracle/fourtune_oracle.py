@@ -335,18 +335,27 @@ _C = math.sqrt(2.0 / math.pi)
 
 
 def gelu_tanh(p: np.ndarray) -> np.ndarray:
-    """0.5 p (1 + tanh(sqrt(2/pi) (p + 0.044715 p^3))), fp64."""
+    """0.5 p (1 + tanh(sqrt(2/pi) (p + 0.044715 p^3))), fp64.
+
+    Evaluated as p * sigmoid(2u), the same function (0.5 (1 + tanh u) = 1 / (1 + e^{-2u})):
+    written as printed, 1 + tanh(u) cancels for p below about -6.5 and loses all relative
+    precision even in fp64."""
     p = np.asarray(p, dtype=np.float64)
-    return 0.5 * p * (1.0 + np.tanh(_C * (p + 0.044715 * p ** 3)))
+    u = _C * (p + 0.044715 * p ** 3)
+    with np.errstate(over="ignore"):
+        return p / (1.0 + np.exp(-2.0 * u))
 
 
 def gelu_tanh_grad(p: np.ndarray) -> np.ndarray:
-    """d/dp of gelu_tanh, fp64 (product and chain rule of the formula above)."""
+    """d/dp of gelu_tanh, fp64: with s = sigmoid(2u), s + 2 p s (1 - s) u' (the product and
+    chain rule of the formula above; 1 - s = sigmoid(-2u) evaluated directly)."""
     p = np.asarray(p, dtype=np.float64)
     u = _C * (p + 0.044715 * p ** 3)
-    t = np.tanh(u)
     du = _C * (1.0 + 3.0 * 0.044715 * p ** 2)
-    return 0.5 * (1.0 + t) + 0.5 * p * (1.0 - t * t) * du
+    with np.errstate(over="ignore"):
+        s = 1.0 / (1.0 + np.exp(-2.0 * u))
+        one_minus = 1.0 / (1.0 + np.exp(2.0 * u))
+    return s + 2.0 * p * s * one_minus * du
 
 
 def to_bf16(a: np.ndarray) -> torch.Tensor:
