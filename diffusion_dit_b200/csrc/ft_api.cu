@@ -2,6 +2,7 @@
 // Host side only: argument checks, workspace carving, TMA descriptors, launch order.
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <atomic>
 #include <mutex>
 
@@ -58,9 +59,10 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     return fn;
 }
 
-// 2-D row-major tensor map with a 128-byte swizzle.
+// 2-D row-major tensor map (128-byte swizzle unless told otherwise).
 ft_status make_tmap(CUtensorMap* map, const void* base, CUtensorMapDataType dt, uint64_t inner_elems,
-                    uint64_t rows, uint64_t row_bytes, uint32_t box_inner, uint32_t box_rows) {
+                    uint64_t rows, uint64_t row_bytes, uint32_t box_inner, uint32_t box_rows,
+                    CUtensorMapSwizzle swz = CU_TENSOR_MAP_SWIZZLE_128B) {
     auto fn = encode_fn();
     if (!fn) return FT_ERR_CUDA;
     cuuint64_t dims[2] = {inner_elems, rows};
@@ -68,7 +70,7 @@ ft_status make_tmap(CUtensorMap* map, const void* base, CUtensorMapDataType dt, 
     cuuint32_t box[2] = {box_inner, box_rows};
     cuuint32_t estr[2] = {1, 1};
     CUresult r = fn(map, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
-                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? FT_OK : FT_ERR_CUDA;
 }
@@ -93,7 +95,18 @@ uint32_t tmem_cols_for(int Rp) {
     return c;
 }
 
-constexpr int kMaxSplits = 16;  // upper bound of quant_down_splits()
+// Upper bound of the column / token slices the fused quantizer and the adapter-gradient
+// kernels use: one CTA per SM at most (the heuristics see at most kMaxSms SMs), and
+// never more than 16 slices.
+constexpr int kMaxSplits = 16;
+constexpr int kMaxSms = 160;
+
+size_t max_splits(int64_t units) {
+    int64_t s = units > 0 ? kMaxSms / units : kMaxSplits;
+    if (s < 1) s = 1;
+    if (s > kMaxSplits) s = kMaxSplits;
+    return static_cast<size_t>(s);
+}
 
 // Workspace of the layer calls.  Regions are 256-byte aligned.
 struct LinearWs {
@@ -122,7 +135,7 @@ LinearWs linear_ws(int64_t M, int64_t N, int64_t K, int R, int r) {
     w.dn = take(static_cast<size_t>(Rp) * K * 2);
     w.upcat = take(static_cast<size_t>(N) * KL * 2);
     w.tcat = take(static_cast<size_t>(M) * KL * 2);
-    w.partial = take(static_cast<size_t>(kMaxSplits) * M * Rp * 4);
+    w.partial = take(std::max(max_splits(M / 128), static_cast<size_t>(1)) * M * Rp * 4);
     w.qg_codes = take(static_cast<size_t>(M) * N / 2);
     w.qg_scales = take(static_cast<size_t>(M) * N / 256);
     w.qg_sf = take(static_cast<size_t>(M) * N / 16);
@@ -131,7 +144,7 @@ LinearWs linear_ws(int64_t M, int64_t N, int64_t K, int R, int r) {
     w.u = take(static_cast<size_t>(M) * R * 4);
     w.ucat = take(static_cast<size_t>(M) * KL * 2);
     w.vcat = take(static_cast<size_t>(M) * lora_width(r) * 2);
-    w.gpartial = take(static_cast<size_t>(kMaxSplits) * (N > K ? N : K) * lora_width(r) * 4);
+    w.gpartial = take(std::max(max_splits(N / 128) * N, max_splits(K / 128) * K) * lora_width(r) * 4);
     w.total = o;
     return w;
 }
@@ -153,6 +166,7 @@ ft_status check_layer(const ft_linear* L) {
     if (!L) return FT_ERR_INVALID_ARG;
     if (L->N <= 0 || L->K <= 0 || L->r_s < 0 || L->r < 0) return FT_ERR_INVALID_ARG;
     if (L->r_s + L->r > 256 || L->r > 64) return FT_ERR_SHAPE;
+    if (L->r_s % 8 || L->r % 8) return FT_ERR_SHAPE;  // factor rows move in 16-byte pieces
     if (L->N % 256 || L->K % 256) return FT_ERR_SHAPE;
     FT_TRY(check_fp4(L->qr, L->N, L->K, true));
     FT_TRY(check_fp4(L->qr_t, L->K, L->N, true));
@@ -218,6 +232,8 @@ ft_status run_gemm(const uint8_t* a_codes, const uint8_t* a_sf, const float* ga,
         tLA = tA;
         tLB = tB;
     }
+    CUtensorMap tOut;
+    FT_TRY(make_tmap(&tOut, out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, N, M, N * 2, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B));
     GemmFp4Args g{};
     g.sfa = a_sf;
     g.sfb = b.sf_mma;
@@ -230,7 +246,7 @@ ft_status run_gemm(const uint8_t* a_codes, const uint8_t* a_sf, const float* ga,
     g.K = static_cast<int>(K);
     g.KL = KL;
     g.status = status;
-    FT_CUDA(ft::launch_gemm_fp4_lowrank(tA, tB, tLA, tLB, g, dev.num_sms, st));
+    FT_CUDA(ft::launch_gemm_fp4_lowrank(tA, tB, tLA, tLB, tOut, g, dev.num_sms, st));
     return FT_OK;
 }
 
@@ -252,7 +268,7 @@ QuantWs quant_ws(int64_t rows, int64_t cols, int r_down) {
     w.status = take(16);
     w.amax = take(16);
     w.down = take(static_cast<size_t>(Rp) * cols * 2);
-    w.partial = take(static_cast<size_t>(kMaxSplits) * rows * Rp * 4);
+    w.partial = take(max_splits(rows / 128) * rows * Rp * 4);
     w.total = o;
     return w;
 }
@@ -523,6 +539,16 @@ ft_status fourtune_linear_bwd(const ft_linear* L, const void* x_dev, const float
         FT_CUDA(ft::launch_lora_grad(tP, tV, g, sp, ft::K_LORA_DA, st));
         FT_CUDA(ft::launch_lora_grad_finalize(gpart, sp, K, NBW, L->r, L->lora_scale, true, da_dev, st));
     }
+    return FT_OK;
+}
+
+ft_status fourtune_selftest_bounded_wait(int64_t limit_ns, void* ws, void* stream) {
+    if (!ws || limit_ns <= 0 || limit_ns > 1000000000LL) return FT_ERR_INVALID_ARG;
+    if (reinterpret_cast<uintptr_t>(ws) % kAlign) return FT_ERR_ALIGN;
+    DeviceInfo dev;
+    FT_TRY(device_info(&dev));
+    FT_CUDA(ft::launch_bounded_wait_selftest(static_cast<uint64_t>(limit_ns), static_cast<int*>(ws),
+                                             static_cast<cudaStream_t>(stream)));
     return FT_OK;
 }
 

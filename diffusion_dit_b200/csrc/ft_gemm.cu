@@ -36,8 +36,10 @@ constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;  // 55296
 constexpr int OFF_B = A_BYTES;
 constexpr int OFF_SFA = A_BYTES + B_BYTES;
 constexpr int OFF_SFB = OFF_SFA + SFA_BYTES;
+constexpr int EPI_BYTES = 32 * 64;        // per epilogue warp: 32 rows x 32 bf16 columns
+constexpr int OFF_EPI = STAGES * STAGE_BYTES;
 constexpr int BAR_BYTES = 256;
-constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + BAR_BYTES + 1024;  // + alignment slack
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 4 * EPI_BYTES + BAR_BYTES + 1024;  // + alignment slack
 constexpr int THREADS = 192;
 
 // Tensor memory columns: accumulator [0,256), scale slots per stage after it.
@@ -53,7 +55,7 @@ struct Smem {
     uint8_t* base;    // 1024-aligned
     uint32_t base_u32;
     __device__ uint32_t stage(int s) const { return base_u32 + s * STAGE_BYTES; }
-    __device__ uint32_t bar(int i) const { return base_u32 + STAGES * STAGE_BYTES + 8 * i; }
+    __device__ uint32_t bar(int i) const { return base_u32 + OFF_EPI + 4 * EPI_BYTES + 8 * i; }
 };
 // barrier indices
 __host__ __device__ constexpr int BAR_FULL(int s) { return s; }
@@ -69,12 +71,13 @@ __global__ void __launch_bounds__(THREADS, 1)
     gemm_fp4_lowrank_kernel(const __grid_constant__ CUtensorMap tmA,
                             const __grid_constant__ CUtensorMap tmB,
                             const __grid_constant__ CUtensorMap tmLA,
-                            const __grid_constant__ CUtensorMap tmLB, const GemmFp4Args p) {
+                            const __grid_constant__ CUtensorMap tmLB,
+                            const __grid_constant__ CUtensorMap tmOut, const GemmFp4Args p) {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_u32 = smem_u32(smem_raw);
     const uint32_t pad = (1024 - (raw_u32 & 1023)) & 1023;
     Smem sm{smem_raw + pad, raw_u32 + pad};
-    uint8_t* bar_area = sm.base + STAGES * STAGE_BYTES;
+    uint8_t* bar_area = sm.base + OFF_EPI + 4 * EPI_BYTES;
     volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(bar_area + OFF_TMEM_SLOT);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(bar_area + OFF_ABORT);
 
@@ -225,27 +228,48 @@ __global__ void __launch_bounds__(THREADS, 1)
             const int mb = t % MB, nb = t / MB;
             if (!mbar_wait(sm.bar(BAR_TMEM_FULL), ti & 1, abort_flag, p.status)) break;
             tc_fence_after();
-            uint32_t pk[BN / 2];
+            // Drain the accumulator into registers (scaled, rounded to bf16) and give the
+            // tensor memory back to the MMA warp at once; then stage each 32 x 32 block in
+            // shared memory (64-byte swizzle, the layout of the output tensor map) and
+            // hand it to a TMA store while the next tile's MMAs already run.
             const uint32_t lane_addr = tmem + COL_ACC + (static_cast<uint32_t>(32 * q) << 16);
+            const uint32_t stage_u32 = sm.base_u32 + OFF_EPI + (warp - 2) * EPI_BYTES;
+            uint8_t* stage_ptr = sm.base + OFF_EPI + (warp - 2) * EPI_BYTES;
+            uint32_t pk[BN / 2];
 #pragma unroll
             for (int ch = 0; ch < BN / 32; ++ch) {
                 uint32_t v[32];
                 tmem_ld_32x32b_x32(lane_addr + ch * 32, v);
                 tmem_ld_wait();
 #pragma unroll
-                for (int j = 0; j < 16; ++j)
-                    pk[ch * 16 + j] = pack_bf16x2(__uint_as_float(v[2 * j]) * c,
-                                                  __uint_as_float(v[2 * j + 1]) * c);
+                for (int jj = 0; jj < 16; ++jj)
+                    pk[ch * 16 + jj] = pack_bf16x2(__uint_as_float(v[2 * jj]) * c,
+                                                   __uint_as_float(v[2 * jj + 1]) * c);
             }
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(sm.bar(BAR_TMEM_EMPTY));
-            const int row = mb * BM + 32 * q + lane;
-            uint4* dst = reinterpret_cast<uint4*>(p.out + static_cast<size_t>(row) * p.ldo + nb * BN);
 #pragma unroll
-            for (int j = 0; j < BN / 8; ++j)
-                dst[j] = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+            for (int ch = 0; ch < BN / 32; ++ch) {
+                if (lane == 0) bulk_wait_group_read0();  // previous store has read the buffer
+                __syncwarp();
+#pragma unroll
+                for (int c4 = 0; c4 < 4; ++c4) {
+                    const int phys = c4 ^ ((lane >> 1) & 3);
+                    *reinterpret_cast<uint4*>(stage_ptr + lane * 64 + phys * 16) =
+                        make_uint4(pk[ch * 16 + 4 * c4], pk[ch * 16 + 4 * c4 + 1], pk[ch * 16 + 4 * c4 + 2],
+                                   pk[ch * 16 + 4 * c4 + 3]);
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    tma_store_2d(&tmOut, stage_u32, nb * BN + ch * 32, mb * BM + 32 * q);
+                    bulk_commit_group();
+                }
+            }
         }
+        if (lane == 0) bulk_wait_group0();
+        __syncwarp();
     }
 
     tc_fence_before();
@@ -258,7 +282,8 @@ __global__ void __launch_bounds__(THREADS, 1)
 
 cudaError_t launch_gemm_fp4_lowrank(const CUtensorMap& tmA, const CUtensorMap& tmB,
                                     const CUtensorMap& tmLA, const CUtensorMap& tmLB,
-                                    const GemmFp4Args& args, int num_sms, cudaStream_t stream) {
+                                    const CUtensorMap& tmOut, const GemmFp4Args& args, int num_sms,
+                                    cudaStream_t stream) {
     using namespace gemm;
     static bool attr_set = false;
     if (!attr_set) {
@@ -270,7 +295,7 @@ cudaError_t launch_gemm_fp4_lowrank(const CUtensorMap& tmA, const CUtensorMap& t
     const int tiles = (args.M / BM) * (args.N / BN);
     const int grid = tiles < num_sms ? tiles : num_sms;
     before_launch(K_GEMM, stream);
-    gemm_fp4_lowrank_kernel<<<grid, THREADS, SMEM_BYTES, stream>>>(tmA, tmB, tmLA, tmLB, args);
+    gemm_fp4_lowrank_kernel<<<grid, THREADS, SMEM_BYTES, stream>>>(tmA, tmB, tmLA, tmLB, tmOut, args);
     after_launch(K_GEMM, stream);
     return cudaGetLastError();
 }

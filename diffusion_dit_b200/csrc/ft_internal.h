@@ -27,9 +27,11 @@ struct GemmFp4Args {
     int* status;            // device status word
 };
 
+// tmOut: bf16 [M, N] output, box 32 x 32, 64-byte swizzle.
 cudaError_t launch_gemm_fp4_lowrank(const CUtensorMap& tmA, const CUtensorMap& tmB,
                                     const CUtensorMap& tmLA, const CUtensorMap& tmLB,
-                                    const GemmFp4Args& args, int num_sms, cudaStream_t stream);
+                                    const CUtensorMap& tmOut, const GemmFp4Args& args, int num_sms,
+                                    cudaStream_t stream);
 
 // quantizer and helpers (ft_quant.cu)
 cudaError_t launch_amax(const void* x, bool is_f32, int64_t rows, int64_t cols, int64_t ld,
@@ -48,21 +50,7 @@ cudaError_t launch_gelu_fwd(const __nv_bfloat16* p, __nv_bfloat16* h, int64_t n,
 cudaError_t launch_gelu_bwd(const __nv_bfloat16* p, const __nv_bfloat16* dh, __nv_bfloat16* dp,
                             int64_t n, cudaStream_t stream);
 
-// low-rank branches (ft_lowrank.cu)
-struct LowRankDownArgs {
-    const __nv_bfloat16* x;  // [M, ldx], reduction over K columns
-    int64_t ldx;
-    int64_t M, K;
-    const __nv_bfloat16* w;  // [R, K] down factor (rows = output columns)
-    int R, r_s;              // columns >= r_s are scaled by `s` before the split
-    float s;
-    const float* ga;         // g of the quantized operand of the following GEMM
-    const float* gb;
-    float* out;              // fp32 [M, R] unscaled product (may be null)
-    __nv_bfloat16* cat;      // bf16 [M, KL]: hi(g v'), lo(g v'), zeros
-    int KL;
-};
-cudaError_t launch_lowrank_down(const LowRankDownArgs& a, cudaStream_t stream);
+cudaError_t launch_bounded_wait_selftest(uint64_t limit_ns, int* status, cudaStream_t stream);
 
 // Fused quantizer + down-projection (ft_quant_fused.cu).
 struct QuantDownArgs {

@@ -206,6 +206,7 @@ int lora_grad_splits(int64_t M, int64_t F, int num_sms) {
     const int64_t tiles = F / lg::BF;
     const int64_t chunks = M / lg::BMT;
     // as many token slices as fill the SMs once, dividing the token chunks evenly
+    if (num_sms > 160) num_sms = 160;  // the workspace queries size partials for at most 160 SMs
     int64_t s = tiles > 0 ? num_sms / tiles : 1;
     if (s < 1) s = 1;
     if (s > 16) s = 16;

@@ -56,40 +56,52 @@ __global__ void lowrank_finalize_kernel(const LowRankFinalizeArgs a) {
 __global__ void build_factors_kernel(const __nv_bfloat16* __restrict__ ls_down,
                                      const __nv_bfloat16* __restrict__ lora_a,
                                      const __nv_bfloat16* __restrict__ ls_up,
-                                     const __nv_bfloat16* __restrict__ lora_b, int64_t N, int64_t K,
-                                     int r_s, int r, int Rp, int KL, __nv_bfloat16* __restrict__ dn,
+                                     const __nv_bfloat16* __restrict__ lora_b, int N, int K, int r_s,
+                                     int r, int Rp, int KL, __nv_bfloat16* __restrict__ dn,
                                      __nv_bfloat16* __restrict__ upcat, __nv_bfloat16* __restrict__ upt,
                                      __nv_bfloat16* __restrict__ dntcat) {
     const int R = r_s + r;
     const __nv_bfloat16 zero = __float2bfloat16_rn(0.0f);
-    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-    const int64_t t0 = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
-    auto dn_at = [&](int j, int64_t k) {
-        return j < r_s ? ls_down[(int64_t)j * K + k] : lora_a[(int64_t)(j - r_s) * K + k];
-    };
-    auto up_at = [&](int64_t n, int j) {
-        return j < r_s ? ls_up[n * r_s + j] : lora_b[n * r + (j - r_s)];
-    };
-    if (dn)
-        for (int64_t i = t0; i < (int64_t)Rp * K; i += stride) {
-            const int j = static_cast<int>(i / K);
-            dn[i] = j < R ? dn_at(j, i % K) : zero;
+    const int stride = gridDim.x * blockDim.x;
+    const int t0 = blockIdx.x * blockDim.x + threadIdx.x;
+    auto dn_at = [&](int j, int k) { return j < r_s ? ls_down[j * K + k] : lora_a[(j - r_s) * K + k]; };
+    auto up_at = [&](int n, int j) { return j < r_s ? ls_up[n * r_s + j] : lora_b[n * r + (j - r_s)]; };
+    // Row-wise pieces move 8 elements (16 bytes) per thread; the 8-element chunks never
+    // straddle two sources because r_s, r and K are multiples of 8 (checked by the host).
+    if (dn) {
+        const int kc = K / 8;
+        for (int i = t0; i < Rp * kc; i += stride) {
+            const int j = i / kc, k = (i % kc) * 8;
+            uint4 v = make_uint4(0, 0, 0, 0);
+            if (j < r_s) v = *reinterpret_cast<const uint4*>(ls_down + j * K + k);
+            else if (j < R) v = *reinterpret_cast<const uint4*>(lora_a + (j - r_s) * K + k);
+            *reinterpret_cast<uint4*>(dn + j * K + k) = v;
         }
-    if (upcat)
-        for (int64_t i = t0; i < N * KL; i += stride) {
-            const int64_t n = i / KL;
-            const int c = static_cast<int>(i % KL);
-            upcat[i] = c < R ? up_at(n, c) : (c < 2 * R ? up_at(n, c - R) : zero);
+    }
+    if (upcat) {
+        const int cc = KL / 8;
+        for (int i = t0; i < N * cc; i += stride) {
+            const int n = i / cc;
+            int c = (i % cc) * 8;
+            uint4 v = make_uint4(0, 0, 0, 0);
+            if (c < 2 * R) {
+                if (c >= R) c -= R;
+                v = c < r_s ? *reinterpret_cast<const uint4*>(ls_up + n * r_s + c)
+                            : *reinterpret_cast<const uint4*>(lora_b + n * r + (c - r_s));
+            }
+            *reinterpret_cast<uint4*>(upcat + n * KL + (i % cc) * 8) = v;
         }
+    }
+    // Transposed pieces: one element per thread, consecutive threads along the
+    // destination row (the sources are small and stay in L2).
     if (upt)
-        for (int64_t i = t0; i < (int64_t)Rp * N; i += stride) {
-            const int j = static_cast<int>(i / N);
-            upt[i] = j < R ? up_at(i % N, j) : zero;
+        for (int i = t0; i < Rp * N; i += stride) {
+            const int j = i / N, n = i % N;
+            upt[i] = j < R ? up_at(n, j) : zero;
         }
     if (dntcat)
-        for (int64_t i = t0; i < K * KL; i += stride) {
-            const int64_t k = i / KL;
-            const int c = static_cast<int>(i % KL);
+        for (int i = t0; i < K * KL; i += stride) {
+            const int k = i / KL, c = i % KL;
             dntcat[i] = c < R ? dn_at(c, k) : (c < 2 * R ? dn_at(c - R, k) : zero);
         }
 }
@@ -116,8 +128,9 @@ cudaError_t launch_build_factors(const __nv_bfloat16* ls_down, const __nv_bfloat
                                  __nv_bfloat16* upcat, __nv_bfloat16* upt, __nv_bfloat16* dntcat,
                                  cudaStream_t stream) {
     before_launch(K_OTHER, stream);
-    build_factors_kernel<<<148 * 4, 256, 0, stream>>>(ls_down, lora_a, ls_up, lora_b, N, K, r_s, r, Rp, KL,
-                                                      dn, upcat, upt, dntcat);
+    build_factors_kernel<<<148 * 4, 256, 0, stream>>>(ls_down, lora_a, ls_up, lora_b, static_cast<int>(N),
+                                                      static_cast<int>(K), r_s, r, Rp, KL, dn, upcat, upt,
+                                                      dntcat);
     after_launch(K_OTHER, stream);
     return cudaGetLastError();
 }

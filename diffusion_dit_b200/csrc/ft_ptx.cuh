@@ -71,7 +71,7 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 // longer) if `abort_flag` becomes non-zero or FT_WAIT_NS elapses; in the timeout case
 // it also raises the CTA's abort flag and the global status word.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
-                                          int* status) {
+                                          int* status, uint64_t limit_ns = FT_WAIT_NS) {
 #pragma unroll 1
     for (int i = 0; i < 256; ++i)
         if (mbar_try_wait(bar, parity)) return true;
@@ -80,7 +80,7 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
     while (true) {
         if (mbar_try_wait(bar, parity)) return true;
         if (*abort_flag) return false;
-        if (globaltimer() - t0 > FT_WAIT_NS) {
+        if (globaltimer() - t0 > limit_ns) {
             *abort_flag = 1;
             if (status) atomicExch(status, kStatusTimeout);
             return false;
@@ -293,6 +293,33 @@ __device__ __forceinline__ uint32_t cvt_e2m1x2(float lo, float hi) {
         : "=r"(out)
         : "f"(hi), "f"(lo));
     return out;
+}
+
+// Eight fp32 -> eight E2M1 codes in one 32-bit word (element i in nibble i), each
+// round-to-nearest-even and saturating.
+__device__ __forceinline__ uint32_t cvt_e2m1x8(const float (&v)[8]) {
+    uint32_t out;
+    asm volatile(
+        "{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+        "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+        : "=r"(out)
+        : "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7]));
+    return out;
+}
+
+// The IEEE fp32 quotient a / 6 for a = any finite bf16 value, without a division: the
+// product with RN(1/6) plus one Markstein correction step (the residual a - 6 q0 is
+// exact in an FMA).  Identical to a / 6 for all 2^15 non-negative bf16 inputs (checked
+// exhaustively against the IEEE division).
+__device__ __forceinline__ float div6_bf16(float a) {
+    const float r6 = 0.16666667163372040f;  // RN(1/6)
+    const float q0 = __fmul_rn(a, r6);
+    const float res = __fmaf_rn(-6.0f, q0, a);
+    return __fmaf_rn(res, r6, q0);
 }
 
 // fp32 (non-negative) -> UE4M3 code, round-to-nearest-even, saturating at 448.

@@ -59,12 +59,25 @@ __global__ void __launch_bounds__(256) amax_kernel(const T* __restrict__ x, int6
                                                    int64_t ld, unsigned* __restrict__ out) {
     const int64_t vec_per_row = cols / 8;
     const int64_t nvec = rows * vec_per_row;
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
     float m = 0.0f;
-    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < nvec;
-         i += (int64_t)gridDim.x * blockDim.x) {
-        const int64_t r = i / vec_per_row, c = (i % vec_per_row) * 8;
+    int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+    // four independent 8-element loads in flight per thread per trip
+    for (; i + 3 * stride < nvec; i += 4 * stride) {
+        float v[4][8];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int64_t iu = i + u * stride;
+            load8(x + (iu / vec_per_row) * ld + (iu % vec_per_row) * 8, v[u]);
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+#pragma unroll
+            for (int j = 0; j < 8; ++j) m = fmaxf(m, fabsf(v[u][j]));
+    }
+    for (; i < nvec; i += stride) {
         float v[8];
-        load8(x + r * ld + c, v);
+        load8(x + (i / vec_per_row) * ld + (i % vec_per_row) * 8, v);
 #pragma unroll
         for (int j = 0; j < 8; ++j) m = fmaxf(m, fabsf(v[j]));
     }
@@ -179,19 +192,24 @@ __global__ void encode_ue4m3_kernel(const float* __restrict__ v, int64_t n, uint
         out[i] = static_cast<uint8_t>(cvt_ue4m3(v[i]));
 }
 
-// GELU, tanh form, fp32 arithmetic with the library tanhf, bf16 round-to-nearest-even.
+// GELU, tanh form: 0.5 p (1 + tanh(u)), u = sqrt(2/pi) (p + 0.044715 p^3).  Evaluated
+// as p * sigmoid(2u), the same function (0.5 (1 + tanh u) = 1 / (1 + exp(-2u))), which
+// keeps full relative accuracy for large negative p where 1 + tanh(u) cancels; fp32
+// with the library expf, result rounded to bf16 (nearest even).
 __device__ __forceinline__ float gelu_tanh_f(float p) {
     const float k = 0.7978845608028654f;  // sqrt(2 / pi)
     const float u = k * (p + 0.044715f * p * p * p);
-    return 0.5f * p * (1.0f + tanhf(u));
+    return p / (1.0f + expf(-2.0f * u));
 }
 
+// d/dp: with s = sigmoid(2u), gelu' = s + 2 p s (1 - s) u'.
 __device__ __forceinline__ float gelu_tanh_grad_f(float p) {
     const float k = 0.7978845608028654f;
     const float u = k * (p + 0.044715f * p * p * p);
-    const float t = tanhf(u);
+    const float sg = 1.0f / (1.0f + expf(-2.0f * u));
+    const float one_minus = 1.0f / (1.0f + expf(2.0f * u));  // sigmoid(-2u), no inf / inf
     const float du = k * (1.0f + 3.0f * 0.044715f * p * p);
-    return 0.5f * (1.0f + t) + 0.5f * p * (1.0f - t * t) * du;
+    return sg + 2.0f * p * sg * one_minus * du;
 }
 
 __global__ void gelu_fwd_kernel(const __nv_bfloat16* __restrict__ p, __nv_bfloat16* __restrict__ h,
@@ -238,7 +256,7 @@ cudaError_t launch_amax(const void* x, bool is_f32, int64_t rows, int64_t cols, 
                         float* amax_out, int num_sms, cudaStream_t stream) {
     cudaError_t e = cudaMemsetAsync(amax_out, 0, sizeof(float), stream);
     if (e != cudaSuccess) return e;
-    const int grid = grid_for(rows * cols / 8, 256, num_sms * 4);
+    const int grid = grid_for(rows * cols / 32, 256, num_sms * 4);
     before_launch(K_AMAX, stream);
     if (is_f32)
         amax_kernel<float><<<grid, 256, 0, stream>>>(static_cast<const float*>(x), rows, cols, ld,
@@ -316,6 +334,35 @@ cudaError_t launch_gelu_bwd(const __nv_bfloat16* p, const __nv_bfloat16* dh, __n
                             int64_t n, cudaStream_t stream) {
     before_launch(K_OTHER, stream);
     gelu_bwd_kernel<<<grid_for(n / 8, 256, 148 * 8), 256, 0, stream>>>(p, dh, dp, n);
+    after_launch(K_OTHER, stream);
+    return cudaGetLastError();
+}
+
+}  // namespace ft
+
+namespace ft {
+namespace {
+
+// Self-test of the bounded wait every pipelined kernel uses: wait on an mbarrier that
+// nothing will ever complete, give up after limit_ns, report FT_ERR_TIMEOUT.
+__global__ void bounded_wait_selftest_kernel(uint64_t limit_ns, int* status) {
+    __shared__ __align__(8) uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        mbar_init(smem_u32(&bar), 1);
+        abort_flag = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) mbar_wait(smem_u32(&bar), 0, &abort_flag, status, limit_ns);
+    __syncthreads();
+}
+
+}  // namespace
+
+cudaError_t launch_bounded_wait_selftest(uint64_t limit_ns, int* status, cudaStream_t stream) {
+    before_launch(K_OTHER, stream);
+    bounded_wait_selftest_kernel<<<1, 32, 0, stream>>>(limit_ns, status);
     after_launch(K_OTHER, stream);
     return cudaGetLastError();
 }

@@ -27,7 +27,7 @@ constexpr int X_BYTES = BM * 128;       // 16 KB
 constexpr int NQ = 8;                   // quantizer warps
 constexpr int THREADS = 32 * (2 + NQ);  // producer, MMA, quantizers
 constexpr int MAX_STAGES = 8;
-constexpr int BAR_BYTES = 256;
+constexpr int BAR_BYTES = 768;           // barriers, TMEM slot, abort flag, inv table at +160
 
 struct Layout {
     int stages;
@@ -140,7 +140,13 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
     } else {
         // ---------------------------------------------------------------- quantizers
-        const int qw = warp - 2;  // block-row of 16 inside the 128-row band
+        // Warp qw owns the 16-row block-row qw of the band; in each 128 x 64 stage it
+        // has four 16x16 blocks.  Lane L works on block j = L / 8 and holds rows
+        // l8 and l8 + 8 (l8 = L % 8) of it, 16 elements each: the block max needs three
+        // shuffle steps inside the 8-lane group, and each lane derives its block's scale
+        // once.  The per-tensor table inv[sb] = fl32(g / val(sb)) replaces the division
+        // per block; the block max / 6 uses div6_bf16 (exact for bf16 inputs).
+        const int qw = warp - 2;
         float g = 1.0f;
         bool degenerate = true;
         {
@@ -154,9 +160,16 @@ __global__ void __launch_bounds__(THREADS, 1)
             }
         }
         if (band == 0 && split == 0 && threadIdx.x == 64) *p.g_out = g;
-        const int rr = qw * 16 + (lane >> 1);  // row inside the band
-        const int h = lane & 1;
-        const int64_t row = row0 + rr;
+        float* inv_lut = reinterpret_cast<float*>(bar_area + 160);  // 128 floats
+        {
+            const int t = threadIdx.x - 64;
+            if (t < 128) inv_lut[t] = (t > 0 && t < 127) ? __fdiv_rn(g, ue4m3_to_f32(t)) : 0.0f;
+            asm volatile("bar.sync 1, %0;" ::"n"(32 * NQ) : "memory");  // quantizer warps only
+        }
+        const int j = lane >> 3;       // block of the stage
+        const int l8 = lane & 7;
+        const int rA = qw * 16 + l8;   // the lane's two rows inside the band
+        const int rB = rA + 8;
         const int64_t cbs = p.cols / 16;
         const int64_t atoms_per_band = p.cols / 64;
         for (int k = 0; k < nk; ++k) {
@@ -164,39 +177,47 @@ __global__ void __launch_bounds__(THREADS, 1)
             if (!mbar_wait(bar(s), (k / S) & 1, abort_flag, p.status)) break;
             const uint8_t* tile = base + s * L.stage_bytes;
             const int64_t c0 = col0 + k * BKE;
+            uint4 w[4];  // rows rA, rA, rB, rB; 16-byte chunks 2j, 2j + 1
+            w[0] = *reinterpret_cast<const uint4*>(tile + rA * 128 + (((2 * j) ^ (rA & 7)) << 4));
+            w[1] = *reinterpret_cast<const uint4*>(tile + rA * 128 + (((2 * j + 1) ^ (rA & 7)) << 4));
+            w[2] = *reinterpret_cast<const uint4*>(tile + rB * 128 + (((2 * j) ^ (rB & 7)) << 4));
+            w[3] = *reinterpret_cast<const uint4*>(tile + rB * 128 + (((2 * j + 1) ^ (rB & 7)) << 4));
+            // block max |x| on the bf16 bit patterns (sign cleared: integer order = numeric order)
+            uint32_t m2 = 0;
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const int chunk = (2 * j + h) ^ (rr & 7);
-                const uint4 w = *reinterpret_cast<const uint4*>(tile + rr * 128 + chunk * 16);
+            for (int q2 = 0; q2 < 4; ++q2)
+                m2 = __vmaxu2(m2, __vmaxu2(__vmaxu2(w[q2].x & 0x7FFF7FFFu, w[q2].y & 0x7FFF7FFFu),
+                                           __vmaxu2(w[q2].z & 0x7FFF7FFFu, w[q2].w & 0x7FFF7FFFu)));
+            uint32_t amb = max(m2 & 0xFFFFu, m2 >> 16);
+            amb = max(amb, __shfl_xor_sync(0xffffffffu, amb, 1));
+            amb = max(amb, __shfl_xor_sync(0xffffffffu, amb, 2));
+            amb = max(amb, __shfl_xor_sync(0xffffffffu, amb, 4));
+            const uint32_t sb =
+                degenerate ? 0u : cvt_ue4m3(__fmul_rn(div6_bf16(__uint_as_float(amb << 16)), g));
+            const float inv = inv_lut[sb];
+            uint32_t code[4];  // row rA: words 0, 1; row rB: words 2, 3
+#pragma unroll
+            for (int q2 = 0; q2 < 4; ++q2) {
                 float v[8];
-                v[0] = bf16lo_to_f32(w.x); v[1] = bf16hi_to_f32(w.x);
-                v[2] = bf16lo_to_f32(w.y); v[3] = bf16hi_to_f32(w.y);
-                v[4] = bf16lo_to_f32(w.z); v[5] = bf16hi_to_f32(w.z);
-                v[6] = bf16lo_to_f32(w.w); v[7] = bf16hi_to_f32(w.w);
-                float am = 0.0f;
-#pragma unroll
-                for (int e = 0; e < 8; ++e) am = fmaxf(am, fabsf(v[e]));
-                am = warp_max(am);
-                uint32_t sb = 0, packed = 0;
-                if (!degenerate) {
-                    sb = cvt_ue4m3(__fmul_rn(__fdiv_rn(am, 6.0f), g));
-                    if (sb != 0) {
-                        const float inv = __fdiv_rn(g, ue4m3_to_f32(sb));
-#pragma unroll
-                        for (int e = 0; e < 4; ++e)
-                            packed |= cvt_e2m1x2(__fmul_rn(v[2 * e], inv), __fmul_rn(v[2 * e + 1], inv))
-                                      << (8 * e);
-                    }
-                }
-                const int64_t col = c0 + 16 * j + 8 * h;
-                *reinterpret_cast<uint32_t*>(p.codes + row * (p.cols / 2) + col / 2) = packed;
-                const int64_t cb = c0 / 16 + j;
-                if (lane == 0) p.scales[(row / 16) * cbs + cb] = static_cast<uint8_t>(sb);
-                if (p.sf_mma && h == 0) {
-                    const int m = rr;  // row inside the 128-row band
-                    const int64_t atom = static_cast<int64_t>(band) * atoms_per_band + c0 / 64;
-                    p.sf_mma[atom * 512 + 16 * (m % 32) + 4 * (m / 32) + (cb % 4)] = static_cast<uint8_t>(sb);
-                }
+                v[0] = __fmul_rn(bf16lo_to_f32(w[q2].x), inv); v[1] = __fmul_rn(bf16hi_to_f32(w[q2].x), inv);
+                v[2] = __fmul_rn(bf16lo_to_f32(w[q2].y), inv); v[3] = __fmul_rn(bf16hi_to_f32(w[q2].y), inv);
+                v[4] = __fmul_rn(bf16lo_to_f32(w[q2].z), inv); v[5] = __fmul_rn(bf16hi_to_f32(w[q2].z), inv);
+                v[6] = __fmul_rn(bf16lo_to_f32(w[q2].w), inv); v[7] = __fmul_rn(bf16hi_to_f32(w[q2].w), inv);
+                code[q2] = sb ? cvt_e2m1x8(v) : 0u;
+            }
+            uint8_t* crow = p.codes + (row0 + rA) * (p.cols / 2) + c0 / 2 + 8 * j;
+            *reinterpret_cast<uint2*>(crow) = make_uint2(code[0], code[1]);
+            *reinterpret_cast<uint2*>(crow + 8 * (p.cols / 2)) = make_uint2(code[2], code[3]);
+            // the four blocks' scales, gathered from lanes l8, l8 + 8, l8 + 16, l8 + 24
+            const uint32_t sb4 = __shfl_sync(0xffffffffu, sb, l8) | (__shfl_sync(0xffffffffu, sb, l8 + 8) << 8) |
+                                 (__shfl_sync(0xffffffffu, sb, l8 + 16) << 16) |
+                                 (__shfl_sync(0xffffffffu, sb, l8 + 24) << 24);
+            if (lane == 0)
+                *reinterpret_cast<uint32_t*>(p.scales + (row0 / 16 + qw) * cbs + c0 / 16) = sb4;
+            if (p.sf_mma && j == 0) {
+                uint8_t* atom = p.sf_mma + (static_cast<int64_t>(band) * atoms_per_band + c0 / 64) * 512;
+                *reinterpret_cast<uint32_t*>(atom + 16 * (rA % 32) + 4 * (rA / 32)) = sb4;
+                *reinterpret_cast<uint32_t*>(atom + 16 * (rB % 32) + 4 * (rB / 32)) = sb4;
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(S + s));
@@ -241,6 +262,7 @@ int quant_down_splits(int64_t rows, int64_t cols, int num_sms) {
     // slices of whole 64-column tiles.
     const int64_t bands = rows / 128;
     const int64_t tiles = cols / 64;
+    if (num_sms > 160) num_sms = 160;  // the workspace queries size partials for at most 160 SMs
     int64_t s = bands > 0 ? num_sms / bands : 1;
     if (s < 1) s = 1;
     if (s > 16) s = 16;

@@ -65,6 +65,7 @@ EXPORTS = {
     "fourtune_encode_e2m1": ([ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p], ctypes.c_int),
     "fourtune_encode_ue4m3": ([ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p], ctypes.c_int),
     "fourtune_launch_count": ([], ctypes.c_uint64),
+    "fourtune_selftest_bounded_wait": ([ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p], ctypes.c_int),
     "fourtune_time_next_launch": ([ctypes.c_int32, ctypes.c_void_p, ctypes.c_void_p], ctypes.c_int),
 }
 

@@ -183,6 +183,15 @@ ft_status fourtune_linear_bwd(const ft_linear* layer, const void* x_dev, const f
 ft_status fourtune_device_status(void* ws, int32_t* status_out, void* stream);
 
 /*
+ * Failure-detection self-test: launches one kernel that waits, with the bounded wait
+ * every pipelined kernel of this library uses, on an mbarrier that nothing completes;
+ * after limit_ns nanoseconds (1 .. 1e9) it gives up and writes FT_ERR_TIMEOUT into the
+ * status word at the start of `ws` (the same place fourtune_device_status reads).
+ * The kernel then returns normally and the CUDA context stays usable.
+ */
+ft_status fourtune_selftest_bounded_wait(int64_t limit_ns, void* ws, void* stream);
+
+/*
  * GELU (tanh form) between the MLP linears (section 3.3 "MLP Fusion" names GeLU):
  *   fwd: h = bf16(0.5 p (1 + tanh(sqrt(2/pi) (p + 0.044715 p^3))))
  *   bwd: dp = bf16(dh * gelu'(p))

@@ -67,7 +67,7 @@ def test_quantize_rejects_bad_arguments_on_host(lib):
     assert q(0x10000, 0, 32, 32, 32, None, None, 0, None, ctypes.byref(with_sf), None, None, 0, None) == 2
 
 
-def _layer(N=256, K=256, r_s=4, r=4):
+def _layer(N=256, K=256, r_s=8, r=8):
     return ft.FtLinear(N, K, r_s, r, 1.0, _fp4(N, K, 0x100000), _fp4(K, N, 0x200000),
                        0x300000, 0x310000, 0x320000, 0x330000)
 

@@ -97,3 +97,25 @@ def test_fused_down_projection_of_the_quantizer():
     _check_equal(q, ora.quantize_block16(x))
     ref = x.double().numpy() @ down.double().numpy().T
     assert ora.rel_frobenius(t.cpu().double().numpy(), ref) < 1e-5
+
+
+@pytest.mark.parametrize("amax_t", [1e-30, 3e-4, 1.0, 250.0, 3e5, 1e30])
+def test_every_bf16_block_max(amax_t):
+    # Each 16x16 block is the constant v for one of the 32639 positive finite bf16 values
+    # (plus one zero block), so the block-scale arithmetic fl32(fl32(v / 6) * g) and the
+    # UE4M3 rounding are exercised on every possible block max, for several g
+    # (amax_t is supplied; blocks above it saturate, as in the oracle).
+    ft = _ft()
+    vals = (np.arange(1, 0x7F80, dtype=np.uint32) << 16).view(np.float32)
+    vals = np.concatenate([vals, np.zeros(1, np.float32)])
+    nb = vals.size + (-vals.size) % 8          # pad to a multiple of 8 blocks (128 columns)
+    vals = np.concatenate([vals, np.full(nb - vals.size, 1.0, np.float32)])
+    row = np.repeat(vals, 16)
+    x = torch.from_numpy(np.tile(row, (128, 1))).to(torch.bfloat16)   # 128 rows x 16*nb columns
+    q, _, _ = ft.quantize_block16(x.cuda(), amax=torch.tensor([amax_t], dtype=torch.float32, device="cuda"),
+                                  with_sf=True)
+    qo = ora.quantize_block16(x[:16].contiguous(), float(np.float32(amax_t)))
+    got_scales = q.scales.cpu().numpy()
+    for band in range(8):
+        assert np.array_equal(got_scales[band], qo.scales[0])
+    assert np.array_equal(q.codes[:16].cpu().numpy(), qo.codes)
