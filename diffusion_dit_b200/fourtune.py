@@ -19,6 +19,8 @@ LIB_PATH = os.path.join(_HERE, "_lib", "libfourtune.so")
 
 FT_DTYPE_BF16 = 0
 FT_DTYPE_F32 = 1
+# size of the fixed scratch array behind fourtune_quantize_block16_noalloc
+NOALLOC_SCRATCH_BYTES = 8 << 20
 
 STATUS = {0: "FT_OK", 1: "FT_ERR_INVALID_ARG", 2: "FT_ERR_SHAPE", 3: "FT_ERR_ALIGN",
           4: "FT_ERR_WORKSPACE", 5: "FT_ERR_CUDA", 6: "FT_ERR_UNSUPPORTED", 7: "FT_ERR_TIMEOUT"}
@@ -64,6 +66,10 @@ EXPORTS = {
                                 ctypes.c_void_p], ctypes.c_int),
     "fourtune_encode_e2m1": ([ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p], ctypes.c_int),
     "fourtune_encode_ue4m3": ([ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p], ctypes.c_int),
+    "fourtune_quantize_block16_noalloc": ([ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_int64,
+                                           ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int32,
+                                           ctypes.c_void_p, ctypes.POINTER(FtFp4), ctypes.POINTER(FtFp4),
+                                           ctypes.c_void_p], ctypes.c_int),
     "fourtune_launch_count": ([], ctypes.c_uint64),
     "fourtune_selftest_bounded_wait": ([ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p], ctypes.c_int),
     "fourtune_time_next_launch": ([ctypes.c_int32, ctypes.c_void_p, ctypes.c_void_p], ctypes.c_int),

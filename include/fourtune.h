@@ -144,6 +144,37 @@ ft_status fourtune_quantize_block16(const void* x_dev, int32_t x_dtype, int64_t 
                                     const ft_fp4* out, const ft_fp4* out_t, void* ws,
                                     size_t ws_bytes, void* stream);
 
+/*
+ * fourtune_quantize_block16_noalloc -- fourtune_quantize_block16 for callers that cannot
+ * allocate device memory.  The paper has no counterpart; this is a library convenience.
+ *
+ * Who needs it: code that is handed only its input and output buffers and has no way to
+ * obtain scratch memory -- for example a plugin running inside a host framework whose
+ * interface passes just the tensors, or a process whose device memory is budgeted up
+ * front and owned by another runtime, so a cudaMalloc here would fail or is not allowed.
+ *
+ * Instead of a caller workspace, the quantizer's scratch (status word, tensor max, the
+ * down factor padded to the MMA width, the per-slice partial sums of the down-projection)
+ * lives in one fixed array of FT_NOALLOC_SCRATCH_BYTES in the library's own device
+ * memory.  Every GPU that loads the library holds that array until the process exits.
+ * Arguments, shapes, results and errors are those of fourtune_quantize_block16; inputs
+ * and outputs are still the caller's.
+ *  - A problem whose scratch (fourtune_quantize_workspace_bytes) exceeds
+ *    FT_NOALLOC_SCRATCH_BYTES is refused with FT_ERR_WORKSPACE before anything runs.
+ *  - The first call on a device looks up the array's device address (that device must
+ *    be current) and keeps it; make that first call before any stream capture.
+ *  - All calls share the one array and it keeps the previous call's contents (the call
+ *    clears what must start at zero).  Calls whose kernels can overlap on the GPU --
+ *    different streams with no ordering between them -- race and give wrong results.
+ *  - It allocates nothing: no cudaMalloc, cudaFree or allocating library routine.
+ */
+#define FT_NOALLOC_SCRATCH_BYTES (8u << 20)
+ft_status fourtune_quantize_block16_noalloc(const void* x_dev, int32_t x_dtype, int64_t rows,
+                                            int64_t cols, int64_t ld, const float* amax_or_null,
+                                            const void* down_dev, int32_t r_down,
+                                            float* down_out_dev, const ft_fp4* out,
+                                            const ft_fp4* out_t, void* stream);
+
 /* Workspace bytes for fourtune_linear_fwd / fourtune_linear_bwd with M tokens. */
 size_t fourtune_linear_workspace_bytes(const ft_linear* layer, int64_t M);
 
