@@ -184,6 +184,9 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--ref-rows", type=int, default=256)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--graph", dest="graph", action="store_true", default=True,
+                    help="replay each step as a captured CUDA graph (default)")
+    ap.add_argument("--no-graph", dest="graph", action="store_false")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -240,13 +243,38 @@ def main():
     Kst = args.steps
     E = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
     ev_s, ev_e = [E() for _ in range(Kst)], [E() for _ in range(Kst)]
-    g_s, g_e = [E() for _ in range(2 * Kst)], [E() for _ in range(2 * Kst)]
-    q_s, q_e = [E() for _ in range(2 * Kst)], [E() for _ in range(2 * Kst)]
-    a_s, a_e = [E() for _ in range(2 * Kst)], [E() for _ in range(2 * Kst)]
-    for ev in ev_s + ev_e + g_s + g_e + q_s + q_e + a_s + a_e:
+    # per-launch events of the dominant kernel (the 4-bit GEMM: forward and dX), the
+    # quantizer and the tensor max; the library records them on the launch stream
+    kev = {k: ([E(), E()], [E(), E()]) for k in (ft.FT_KERNEL_GEMM, ft.FT_KERNEL_QUANT, ft.FT_KERNEL_AMAX)}
+    for ev in ev_s + ev_e + [e for b_, a_ in kev.values() for e in b_ + a_]:
         ev.record()  # torch creates the CUDA event on first record; the library needs the handle
     torch.cuda.synchronize()
 
+    def one_step_with_events():
+        for k, (b_, a_) in kev.items():
+            ft.time_next_launch(k, b_[0], a_[0])
+        ft.linear_fwd(w, x, ws, y=y, t_saved=t)
+        for k, (b_, a_) in kev.items():
+            ft.time_next_launch(k, b_[1], a_[1])
+        ft.linear_bwd(w, x, t, dy, ws, dx=dx, da=da, db=db)
+
+    graph = None
+    launches_per_step = None
+    if args.graph:
+        # One step (forward + backward, all of the library's kernels and its timing-event
+        # records) captured once as a CUDA graph and replayed: the same kernels, without
+        # the host launch gaps between them.
+        c0 = ft.launch_count()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            one_step_with_events()
+        launches_per_step = ft.launch_count() - c0
+        for _ in range(args.warmup):
+            flush.zero_()
+            graph.replay()
+        torch.cuda.synchronize()
+
+    gemm_ms, quant_ms, amax_ms = [], [], []
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
@@ -255,29 +283,27 @@ def main():
         for i in range(Kst):
             flush.zero_()
             ev_s[i].record()
-            ft.time_next_launch(ft.FT_KERNEL_GEMM, g_s[2 * i], g_e[2 * i])
-            ft.time_next_launch(ft.FT_KERNEL_QUANT, q_s[2 * i], q_e[2 * i])
-            ft.time_next_launch(ft.FT_KERNEL_AMAX, a_s[2 * i], a_e[2 * i])
-            ft.linear_fwd(w, x, ws, y=y, t_saved=t)
-            ft.time_next_launch(ft.FT_KERNEL_GEMM, g_s[2 * i + 1], g_e[2 * i + 1])
-            ft.time_next_launch(ft.FT_KERNEL_QUANT, q_s[2 * i + 1], q_e[2 * i + 1])
-            ft.time_next_launch(ft.FT_KERNEL_AMAX, a_s[2 * i + 1], a_e[2 * i + 1])
-            ft.linear_bwd(w, x, t, dy, ws, dx=dx, da=da, db=db)
+            if graph is not None:
+                graph.replay()
+            else:
+                one_step_with_events()
             if world > 1:
                 dp.allreduce_adapter_grads(da, db)
             ev_e[i].record()
+            # the per-launch events are reused by every step: read them before the next one
+            torch.cuda.synchronize()
+            for k, dst in ((ft.FT_KERNEL_GEMM, gemm_ms), (ft.FT_KERNEL_QUANT, quant_ms), (ft.FT_KERNEL_AMAX, amax_ms)):
+                b_, a_ = kev[k]
+                dst.extend([b_[0].elapsed_time(a_[0]), b_[1].elapsed_time(a_[1])])
         torch.cuda.synchronize()
         if world > 1:
             dist.barrier()
         torch.cuda.synchronize()
-    launches = ft.launch_count() - launches0
+    launches = (launches_per_step * Kst) if graph is not None else ft.launch_count() - launches0
     if ws.device_status() != 0:
         raise RuntimeError("device status reports a timeout in the timed region")
 
     total_ms = sum(ev_s[i].elapsed_time(ev_e[i]) for i in range(Kst))
-    gemm_ms = [g_s[j].elapsed_time(g_e[j]) for j in range(2 * Kst)]
-    quant_ms = [q_s[j].elapsed_time(q_e[j]) for j in range(2 * Kst)]
-    amax_ms = [a_s[j].elapsed_time(a_e[j]) for j in range(2 * Kst)]
     tm = torch.tensor([total_ms], dtype=torch.float64, device=dev)
     if world > 1:
         dist.all_reduce(tm, op=dist.ReduceOp.MAX)
@@ -345,6 +371,7 @@ def main():
                           "frac_with_amax": qa_gbs / hbm, "avg_launch_ms": statistics.mean(quant_ms)},
             "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
             "gpu_launches": launches,
+            "launch_mode": "cuda_graph_replay" if graph is not None else "stream",
             "clocks": clocks.summary(),
         }
         if world == 1 and not args.no_cpu_baseline:

@@ -111,7 +111,7 @@ size_t max_splits(int64_t units) {
 // Workspace of the layer calls.  Regions are 256-byte aligned.
 struct LinearWs {
     size_t status, scal, qx_codes, qx_scales, qx_sf, dn, upcat, tcat, partial;
-    size_t qg_codes, qg_scales, qg_sf, upt, dntcat, u, ucat, vcat, gpartial, total;
+    size_t qg_codes, qg_scales, qg_sf, upt, dntcat, ucat, vcat, ucat_lora, gpartial, total;
 };
 
 // Width of the adapter-gradient operand [hi, lo, 0]: 2r rounded up to 64.
@@ -141,9 +141,9 @@ LinearWs linear_ws(int64_t M, int64_t N, int64_t K, int R, int r) {
     w.qg_sf = take(static_cast<size_t>(M) * N / 16);
     w.upt = take(static_cast<size_t>(Rp) * N * 2);
     w.dntcat = take(static_cast<size_t>(K) * KL * 2);
-    w.u = take(static_cast<size_t>(M) * R * 4);
     w.ucat = take(static_cast<size_t>(M) * KL * 2);
     w.vcat = take(static_cast<size_t>(M) * lora_width(r) * 2);
+    w.ucat_lora = take(static_cast<size_t>(M) * lora_width(r) * 2);
     w.gpartial = take(std::max(max_splits(N / 128) * N, max_splits(K / 128) * K) * lora_width(r) * 4);
     w.total = o;
     return w;
@@ -282,11 +282,22 @@ cudaEvent_t g_ev_after[FT_KERNEL_KINDS] = {};
 
 namespace ft {
 
+// Records a caller's timing event on the launch stream.  Inside a stream capture the
+// record becomes an external event node of the graph, which is recorded at every
+// replay and can be timed.
+static void record_event(cudaEvent_t ev, cudaStream_t stream) {
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(stream, &cs) == cudaSuccess && cs == cudaStreamCaptureStatusActive)
+        cudaEventRecordWithFlags(ev, stream, cudaEventRecordExternal);
+    else
+        cudaEventRecord(ev, stream);
+}
+
 void before_launch(int kind, cudaStream_t stream) {
     if (kind < 0 || kind >= FT_KERNEL_KINDS) return;
     std::lock_guard<std::mutex> lock(g_ev_mu);
     if (g_ev_before[kind]) {
-        cudaEventRecord(g_ev_before[kind], stream);
+        record_event(g_ev_before[kind], stream);
         g_ev_before[kind] = nullptr;
     }
 }
@@ -296,7 +307,7 @@ void after_launch(int kind, cudaStream_t stream) {
     if (kind < 0 || kind >= FT_KERNEL_KINDS) return;
     std::lock_guard<std::mutex> lock(g_ev_mu);
     if (g_ev_after[kind]) {
-        cudaEventRecord(g_ev_after[kind], stream);
+        record_event(g_ev_after[kind], stream);
         g_ev_after[kind] = nullptr;
     }
 }
@@ -480,7 +491,6 @@ ft_status fourtune_linear_bwd(const ft_linear* L, const void* x_dev, const float
     const int KL = low_rank_width(R);
     const int Rp = padded_rank(R);
     float* partial = reinterpret_cast<float*>(W + w.partial);
-    float* U = reinterpret_cast<float*>(W + w.u);
 
     // Eq. (3): Q(G) fused with U = G [Ls_up, B], the dX GEMM through Q(R)^T with
     // U [Ls_down; A] in its accumulator, then the adapter gradients.
@@ -502,9 +512,13 @@ ft_status fourtune_linear_bwd(const ft_linear* L, const void* x_dev, const float
         f.s = L->lora_scale;
         f.ga = scal + SC_G_G;
         f.gb = L->qr_t.g;
-        f.out = U;
+        f.out = nullptr;  // U itself is not needed: only its GEMM and dA operands
         f.cat = bfm(W + w.ucat);
         f.KL = KL;
+        if (L->r > 0) {  // U_lora's hi/lo operand for dA, written by the same pass
+            f.lora_cat = bfm(W + w.ucat_lora);
+            f.NBW = lora_width(L->r);
+        }
         FT_CUDA(ft::launch_lowrank_finalize(f, st));
     }
     FT_TRY(run_gemm(W + w.qg_codes, W + w.qg_sf, scal + SC_G_G, L->qr_t, bf(W + w.ucat), bf(W + w.dntcat), KL,
@@ -530,8 +544,8 @@ ft_status fourtune_linear_bwd(const ft_linear* L, const void* x_dev, const float
         g.tokens_per_split = static_cast<int>(M / sp);
         FT_CUDA(ft::launch_lora_grad(tP, tV, g, sp, ft::K_LORA_DB, st));
         FT_CUDA(ft::launch_lora_grad_finalize(gpart, sp, N, NBW, L->r, L->lora_scale, false, db_dev, st));
-        // dA over the input features k
-        FT_CUDA(ft::launch_build_hilo(U, R, L->r_s, L->r, M, NBW, vcat, st));
+        // dA over the input features k (V' = U_lora's hi/lo, written by the split sum)
+        FT_TRY(make_tmap(&tV, W + w.ucat_lora, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, NBW, M, NBW * 2, 64, 64));
         FT_TRY(make_tmap(&tP, x_dev, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, K, M, K * 2, 64, 64));
         sp = ft::lora_grad_splits(M, K, dev.num_sms);
         g.F = K;

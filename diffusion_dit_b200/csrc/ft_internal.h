@@ -84,6 +84,8 @@ struct LowRankFinalizeArgs {
     float* out;
     __nv_bfloat16* cat;
     int KL;
+    __nv_bfloat16* lora_cat;  // optional [rows, NBW] = [hi, lo, 0] of the LoRA columns (unscaled)
+    int NBW;
 };
 cudaError_t launch_lowrank_finalize(const LowRankFinalizeArgs& a, cudaStream_t stream);
 

@@ -156,22 +156,21 @@ __global__ void __launch_bounds__(THREADS, 1)
 }
 
 // out = s * sum_split (D[f][j] + D[f][r + j]); transposed (out[j][f]) for dA.
-__global__ void lora_grad_finalize_kernel(const float* __restrict__ partial, int splits, int64_t F, int NBW,
-                                          int r, float s, bool transpose_out, float* __restrict__ out) {
-    const int64_t total = F * r;
-    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total;
-         i += (int64_t)gridDim.x * blockDim.x) {
-        int64_t f, j;
-        if (transpose_out) {  // consecutive threads walk f for coalesced stores into out[j][f]
+__global__ void lora_grad_finalize_kernel(const float* __restrict__ partial, int splits, int F, int NBW, int r,
+                                          float s, bool transpose_out, float* __restrict__ out) {
+    const int total = F * r;
+    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < total; i += gridDim.x * blockDim.x) {
+        int f, j;
+        if (transpose_out) {  // consecutive threads walk f: coalesced stores into out[j][f]
             j = i / F;
-            f = i % F;
+            f = i - j * F;
         } else {
             f = i / r;
-            j = i % r;
+            j = i - f * r;
         }
         float v = 0.0f;
         for (int sp = 0; sp < splits; ++sp) {
-            const float* d = partial + (static_cast<int64_t>(sp) * F + f) * NBW;
+            const float* d = partial + (sp * F + f) * NBW;
             v += d[j] + d[r + j];
         }
         v *= s;
@@ -183,13 +182,12 @@ __global__ void lora_grad_finalize_kernel(const float* __restrict__ partial, int
 }
 
 // V' [M, NBW] bf16 = [hi(V), lo(V), 0] from fp32 V = src[:, c0 : c0 + r] (row stride ld).
-__global__ void build_hilo_kernel(const float* __restrict__ src, int64_t ld, int c0, int r, int64_t M, int NBW,
+__global__ void build_hilo_kernel(const float* __restrict__ src, int ld, int c0, int r, int M, int NBW,
                                   __nv_bfloat16* __restrict__ dst) {
-    const int64_t total = M * NBW;
-    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total;
-         i += (int64_t)gridDim.x * blockDim.x) {
-        const int64_t m = i / NBW;
-        const int c = static_cast<int>(i % NBW);
+    const int total = M * NBW;
+    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < total; i += gridDim.x * blockDim.x) {
+        const int m = i / NBW;
+        const int c = i - m * NBW;
         __nv_bfloat16 o = __float2bfloat16_rn(0.0f);
         if (c < 2 * r) {
             const float v = src[m * ld + c0 + (c < r ? c : c - r)];
@@ -217,9 +215,10 @@ int lora_grad_splits(int64_t M, int64_t F, int num_sms) {
 cudaError_t launch_lora_grad(const CUtensorMap& tmP, const CUtensorMap& tmV, const LoraGradArgs& a, int splits,
                              int kind, cudaStream_t stream) {
     const lg::Layout L = lg::layout_for(a.NBW);
-    cudaError_t e = cudaFuncSetAttribute(lg::lora_grad_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         L.smem_bytes);
-    if (e != cudaSuccess) return e;
+    // the opt-in limit is raised once to the device maximum (no per-launch host calls)
+    static const cudaError_t attr = cudaFuncSetAttribute(
+        lg::lora_grad_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 232448);
+    if (attr != cudaSuccess) return attr;
     dim3 grid(static_cast<unsigned>(a.F / lg::BF), static_cast<unsigned>(splits));
     before_launch(kind, stream);
     lg::lora_grad_kernel<<<grid, lg::THREADS, L.smem_bytes, stream>>>(tmP, tmV, a);
@@ -232,8 +231,8 @@ cudaError_t launch_lora_grad_finalize(const float* partial, int splits, int64_t 
     int64_t g = (F * r + 255) / 256;
     if (g > 148 * 8) g = 148 * 8;
     before_launch(K_OTHER, stream);
-    lg::lora_grad_finalize_kernel<<<static_cast<unsigned>(g), 256, 0, stream>>>(partial, splits, F, NBW, r, s,
-                                                                                 transpose_out, out);
+    lg::lora_grad_finalize_kernel<<<static_cast<unsigned>(g), 256, 0, stream>>>(
+        partial, splits, static_cast<int>(F), NBW, r, s, transpose_out, out);
     after_launch(K_OTHER, stream);
     return cudaGetLastError();
 }
@@ -243,7 +242,8 @@ cudaError_t launch_build_hilo(const float* src, int64_t ld, int c0, int r, int64
     int64_t g = (M * NBW + 255) / 256;
     if (g > 148 * 8) g = 148 * 8;
     before_launch(K_OTHER, stream);
-    lg::build_hilo_kernel<<<static_cast<unsigned>(g), 256, 0, stream>>>(src, ld, c0, r, M, NBW, dst);
+    lg::build_hilo_kernel<<<static_cast<unsigned>(g), 256, 0, stream>>>(src, static_cast<int>(ld), c0, r,
+                                                                        static_cast<int>(M), NBW, dst);
     after_launch(K_OTHER, stream);
     return cudaGetLastError();
 }

@@ -20,31 +20,39 @@
 namespace ft {
 namespace {
 
-// One thread per (row, j < R): fixed-order sum over the splits, then the hi/lo operand.
+// One thread per (row, j < R): fixed-order sum over the splits, then the hi/lo operands.
 __global__ void lowrank_finalize_kernel(const LowRankFinalizeArgs a) {
-    const int64_t total = a.rows * a.R;
+    const int rows = static_cast<int>(a.rows);
+    const int total = rows * a.R;
     const float g = (a.cat != nullptr) ? __fmul_rn(*a.ga, *a.gb) : 1.0f;
-    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total;
-         i += (int64_t)gridDim.x * blockDim.x) {
-        const int64_t m = i / a.R;
-        const int j = static_cast<int>(i % a.R);
+    const __nv_bfloat16 zero = __float2bfloat16_rn(0.0f);
+    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < total; i += gridDim.x * blockDim.x) {
+        const int m = i / a.R;
+        const int j = i - m * a.R;
         float v = 0.0f;
-        for (int sp = 0; sp < a.splits; ++sp) v += a.partial[(sp * a.rows + m) * a.Rp + j];
+        for (int sp = 0; sp < a.splits; ++sp) v += a.partial[(sp * rows + m) * a.Rp + j];
         if (a.out) a.out[m * a.R + j] = v;
         if (a.cat) {
             const float vs = (j >= a.r_s) ? __fmul_rn(v, a.s) : v;
             const float gv = __fmul_rn(vs, g);
             const __nv_bfloat16 hi = __float2bfloat16_rn(gv);
-            const __nv_bfloat16 lo = __float2bfloat16_rn(gv - __bfloat162float(hi));
             a.cat[m * a.KL + j] = hi;
-            a.cat[m * a.KL + a.R + j] = lo;
+            a.cat[m * a.KL + a.R + j] = __float2bfloat16_rn(gv - __bfloat162float(hi));
+            if (j < a.KL - 2 * a.R) a.cat[m * a.KL + 2 * a.R + j] = zero;
+        }
+        if (a.lora_cat && j >= a.r_s) {  // adapter-gradient operand [hi(v), lo(v), 0] of the LoRA columns
+            const int c = j - a.r_s;
+            const int r = a.R - a.r_s;
+            const __nv_bfloat16 hi = __float2bfloat16_rn(v);
+            a.lora_cat[m * a.NBW + c] = hi;
+            a.lora_cat[m * a.NBW + r + c] = __float2bfloat16_rn(v - __bfloat162float(hi));
+            for (int z = 2 * r + c; z < a.NBW; z += r) a.lora_cat[m * a.NBW + z] = zero;
         }
     }
-    if (a.cat && a.KL > 2 * a.R) {  // zero padding
+    if (a.cat && a.KL - 2 * a.R > a.R) {  // zero padding wider than R columns
         const int w = a.KL - 2 * a.R;
-        for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < a.rows * w;
-             i += (int64_t)gridDim.x * blockDim.x)
-            a.cat[(i / w) * a.KL + 2 * a.R + (i % w)] = __float2bfloat16_rn(0.0f);
+        for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < rows * w; i += gridDim.x * blockDim.x)
+            a.cat[(i / w) * a.KL + 2 * a.R + (i % w)] = zero;
     }
 }
 

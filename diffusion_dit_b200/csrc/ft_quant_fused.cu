@@ -275,9 +275,10 @@ size_t quant_down_smem_bytes(int Rp) { return static_cast<size_t>(qf::layout_for
 cudaError_t launch_quant_down(const CUtensorMap& tmX, const CUtensorMap& tmW, const QuantDownArgs& a,
                               int splits, cudaStream_t stream) {
     const qf::Layout L = qf::layout_for(a.Rp);
-    cudaError_t e = cudaFuncSetAttribute(qf::quant_down_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         L.smem_bytes);
-    if (e != cudaSuccess) return e;
+    // the opt-in limit is raised once to the device maximum (no per-launch host calls)
+    static const cudaError_t attr = cudaFuncSetAttribute(
+        qf::quant_down_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 232448);
+    if (attr != cudaSuccess) return attr;
     dim3 grid(static_cast<unsigned>(a.rows / 128), static_cast<unsigned>(splits));
     before_launch(K_QUANT, stream);
     qf::quant_down_kernel<<<grid, qf::THREADS, L.smem_bytes, stream>>>(tmX, tmW, a);
