@@ -12,12 +12,15 @@
 //
 // B200 design: persistent CTAs (one per SM), 128x256 output tile per CTA, a 4-stage
 // shared-memory ring fed by TMA (128-byte swizzle), tcgen05.mma with the fp32
-// accumulator in tensor memory, scale factors copied smem -> TMEM with tcgen05.cp, and
-// an epilogue that drains TMEM into registers before storing so the next tile's MMAs
-// start while the stores are still in flight.
+// accumulator in tensor memory, scale factors written into tensor memory by four scale
+// warps with tcgen05.st (a tcgen05.cp costs the tensor pipe about as much as half an MMA,
+// and a stage would need twelve of them), and an epilogue that drains TMEM into
+// registers before storing so the next tile's MMAs start while the stores are still in
+// flight.
 //
-// Warp roles (192 threads): warp 0 = TMA producer, warp 1 = MMA issuer (and TMEM
-// owner), warps 2..5 = epilogue (warp w reads TMEM lanes 32 (w % 4) .. +31).
+// Warp roles (320 threads): warp 0 = TMA producer, warp 1 = MMA issuer (and TMEM
+// owner), warps 2..5 = epilogue, warps 6..9 = scale writers (warp w reaches TMEM lanes
+// 32 (w % 4) .. +31).
 #include "ft_internal.h"
 #include "ft_ptx.cuh"
 
@@ -40,7 +43,7 @@ constexpr int EPI_BYTES = 32 * 64;        // per epilogue warp: 32 rows x 32 bf1
 constexpr int OFF_EPI = STAGES * STAGE_BYTES;
 constexpr int BAR_BYTES = 256;
 constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 4 * EPI_BYTES + BAR_BYTES + 1024;  // + alignment slack
-constexpr int THREADS = 192;
+constexpr int THREADS = 320;
 
 // Tensor memory columns: accumulator [0,256), scale slots per stage after it.
 constexpr uint32_t TMEM_COLS = 512;
@@ -63,7 +66,8 @@ __host__ __device__ constexpr int BAR_EMPTY(int s) { return STAGES + s; }
 constexpr int BAR_TMEM_FULL = 2 * STAGES;
 constexpr int BAR_TMEM_EMPTY = 2 * STAGES + 1;
 constexpr int BAR_FINAL = 2 * STAGES + 2;
-constexpr int NUM_BARS = 2 * STAGES + 3;
+__host__ __device__ constexpr int BAR_SF_READY(int s) { return 2 * STAGES + 3 + s; }
+constexpr int NUM_BARS = 3 * STAGES + 3;
 constexpr int OFF_TMEM_SLOT = 8 * 16;   // inside the barrier area
 constexpr int OFF_ABORT = 8 * 16 + 4;
 
@@ -94,6 +98,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         for (int i = 0; i < STAGES; ++i) {
             mbar_init(sm.bar(BAR_FULL(i)), 1);
             mbar_init(sm.bar(BAR_EMPTY(i)), 1);
+            mbar_init(sm.bar(BAR_SF_READY(i)), 4);
         }
         mbar_init(sm.bar(BAR_TMEM_FULL), 1);
         mbar_init(sm.bar(BAR_TMEM_EMPTY), 4);
@@ -176,19 +181,15 @@ __global__ void __launch_bounds__(THREADS, 1)
                 for (int kt = 0; kt < KT; ++kt, ++it) {
                     const int s = it % STAGES;
                     const uint32_t ph = (it / STAGES) & 1;
-                    if (!mbar_wait(sm.bar(BAR_FULL(s)), ph, abort_flag, p.status)) { ok = false; break; }
+                    if (!mbar_wait(sm.bar(BAR_FULL(s)), ph, abort_flag, p.status) ||
+                        !mbar_wait(sm.bar(BAR_SF_READY(s)), ph, abort_flag, p.status)) {
+                        ok = false;
+                        break;
+                    }
                     tc_fence_after();
                     const uint32_t st = sm.stage(s);
                     const uint32_t sfa_t = tmem + COL_SFA + 16 * s;
                     const uint32_t sfb_t = tmem + COL_SFB + 32 * s;
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        tmem_cp_32x128b_x4(sfa_t + 4 * i, sdesc_scale_32x16(st + OFF_SFA + 512 * i));
-#pragma unroll
-                        for (int rb = 0; rb < 2; ++rb)
-                            tmem_cp_32x128b_x4(sfb_t + 8 * i + 4 * rb,
-                                               sdesc_scale_32x16(st + OFF_SFB + rb * 2048 + 512 * i));
-                    }
                     const uint64_t ad = sdesc_kmajor_sw128(st);
                     const uint64_t bd = sdesc_kmajor_sw128(st + OFF_B);
 #pragma unroll
@@ -201,7 +202,11 @@ __global__ void __launch_bounds__(THREADS, 1)
                 for (int kl = 0; kl < KLS; ++kl, ++it) {
                     const int s = it % STAGES;
                     const uint32_t ph = (it / STAGES) & 1;
-                    if (!mbar_wait(sm.bar(BAR_FULL(s)), ph, abort_flag, p.status)) { ok = false; break; }
+                    if (!mbar_wait(sm.bar(BAR_FULL(s)), ph, abort_flag, p.status) ||
+                        !mbar_wait(sm.bar(BAR_SF_READY(s)), ph, abort_flag, p.status)) {
+                        ok = false;
+                        break;
+                    }
                     tc_fence_after();
                     const uint32_t st = sm.stage(s);
                     const uint64_t ad = sdesc_kmajor_sw128(st);
@@ -217,6 +222,48 @@ __global__ void __launch_bounds__(THREADS, 1)
             tc_commit(sm.bar(BAR_FINAL));
             volatile int no_abort = 0;
             mbar_wait(sm.bar(BAR_FINAL), 0, &no_abort, p.status);
+        }
+    } else if (warp >= 6) {
+        // ------------------------------------------------------------ scale writers
+        // Lane l of warp w owns TMEM lane 32 (w % 4) + l.  The block-scaled MMA reads the
+        // scales of a 64-wide k block from 4 columns (A) and 8 columns (B) per lane, holding
+        // the 16-byte row (l) of each 512-byte scale atom (the tcgen05.cp 32x128b.warpx4
+        // layout: the same 32 x 16 bytes in every 32-lane quarter).  Every ring item gets an
+        // arrival, so the MMA issuer can wait on SF_READY with the ring's own phase.
+        const int q = warp & 3;
+        const uint32_t lane_base = tmem + (static_cast<uint32_t>(32 * q) << 16);
+        int it = 0;
+        for (int t = blockIdx.x; t < num_tiles && !*abort_flag; t += gridDim.x) {
+            bool ok = true;
+            for (int j = 0; j < KT + KLS; ++j, ++it) {
+                const int s = it % STAGES;
+                const uint32_t ph = (it / STAGES) & 1;
+                if (!mbar_wait(sm.bar(BAR_FULL(s)), ph, abort_flag, p.status)) { ok = false; break; }
+                if (j < KT) {
+                    const uint8_t* st = sm.base + s * STAGE_BYTES;
+                    uint32_t va[16], vb0[16], vb1[16];
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const uint4 a = *reinterpret_cast<const uint4*>(st + OFF_SFA + 512 * i + 16 * lane);
+                        const uint4 b0 = *reinterpret_cast<const uint4*>(st + OFF_SFB + 512 * i + 16 * lane);
+                        const uint4 b1 =
+                            *reinterpret_cast<const uint4*>(st + OFF_SFB + 2048 + 512 * i + 16 * lane);
+                        uint32_t* vb = i < 2 ? vb0 : vb1;
+                        const int o = 8 * (i & 1);
+                        va[4 * i] = a.x; va[4 * i + 1] = a.y; va[4 * i + 2] = a.z; va[4 * i + 3] = a.w;
+                        vb[o] = b0.x; vb[o + 1] = b0.y; vb[o + 2] = b0.z; vb[o + 3] = b0.w;
+                        vb[o + 4] = b1.x; vb[o + 5] = b1.y; vb[o + 6] = b1.z; vb[o + 7] = b1.w;
+                    }
+                    tmem_st_32x32b_x16(lane_base + COL_SFA + 16 * s, va);
+                    tmem_st_32x32b_x16(lane_base + COL_SFB + 32 * s, vb0);
+                    tmem_st_32x32b_x16(lane_base + COL_SFB + 32 * s + 16, vb1);
+                    tmem_st_wait();
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(sm.bar(BAR_SF_READY(s)));
+            }
+            if (!ok) break;
         }
     } else {
         // ------------------------------------------------------------ epilogue
