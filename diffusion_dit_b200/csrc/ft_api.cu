@@ -222,12 +222,15 @@ ft_status quantize_operand(const void* x, int64_t rows, int64_t cols, int64_t ld
 ft_status run_gemm(const uint8_t* a_codes, const uint8_t* a_sf, const float* ga, const ft_fp4& b,
                    const __nv_bfloat16* la, const __nv_bfloat16* lb, int KL, int64_t M, int64_t N,
                    int64_t K, void* out, int* status, const DeviceInfo& dev, cudaStream_t st) {
+    // CTA pairs (256 x 256 tiles) when M allows, single CTAs (128 x 256) otherwise.
+    const bool pair = (M % 256) == 0 && dev.num_sms >= 2;
+    const uint32_t b_rows = pair ? 128 : 256;
     CUtensorMap tA, tB, tLA, tLB;
     FT_TRY(make_tmap(&tA, a_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, K / 2, M, K / 2, 128, 128));
-    FT_TRY(make_tmap(&tB, b.codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, K / 2, N, K / 2, 128, 256));
+    FT_TRY(make_tmap(&tB, b.codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, K / 2, N, K / 2, 128, b_rows));
     if (KL > 0) {
         FT_TRY(make_tmap(&tLA, la, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, KL, M, KL * 2, 64, 128));
-        FT_TRY(make_tmap(&tLB, lb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, KL, N, KL * 2, 64, 256));
+        FT_TRY(make_tmap(&tLB, lb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, KL, N, KL * 2, 64, b_rows));
     } else {
         tLA = tA;
         tLB = tB;
@@ -246,7 +249,10 @@ ft_status run_gemm(const uint8_t* a_codes, const uint8_t* a_sf, const float* ga,
     g.K = static_cast<int>(K);
     g.KL = KL;
     g.status = status;
-    FT_CUDA(ft::launch_gemm_fp4_lowrank(tA, tB, tLA, tLB, tOut, g, dev.num_sms, st));
+    if (pair)
+        FT_CUDA(ft::launch_gemm_fp4_lowrank_pair(tA, tB, tLA, tLB, tOut, g, dev.num_sms, st));
+    else
+        FT_CUDA(ft::launch_gemm_fp4_lowrank(tA, tB, tLA, tLB, tOut, g, dev.num_sms, st));
     return FT_OK;
 }
 

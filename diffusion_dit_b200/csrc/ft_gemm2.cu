@@ -1,0 +1,345 @@
+// Block-scaled FP4 GEMM with the low-rank tail, computed by CTA pairs (cta_group::2).
+//
+// Same result as gemm_fp4_lowrank_kernel (ft_gemm.cu: FourTune Eq. (2) forward and the
+// backbone pathway of Eq. (3), low-rank branches added in the same accumulator), with
+// less data moved per SM: two CTAs on neighbouring SMs form a cluster and compute one
+// 256 x 256 output tile with tcgen05.mma.cta_group::2, issued by the even CTA.  Each CTA
+// loads its own 128 rows of A and its own 128 rows of B (the MMA reads the pair's shared
+// memories together), so per stage a CTA moves 38 KB instead of the 54 KB a 128 x 256
+// tile needs alone; the single-CTA kernel is bound by operand delivery into shared memory.
+//
+// Per CTA and stage: A [128 x 128 B], B [128 x 128 B] (its half of the tile's N), the
+// scale atoms of its A rows (2 KB) and of all 256 B rows (4 KB: every CTA's part of the
+// MMA reads the scales of the full N from its own tensor memory).  Each CTA's loads
+// complete on its own FULL barrier; its four scale warps write the scale factors into its
+// own tensor memory (tcgen05.st) and arrive on the even CTA's SF_READY barrier, which the
+// MMA issuer waits on, so SF_READY also certifies that both CTAs' operands have landed.
+// The MMA issuer's commits arrive on both CTAs' EMPTY barriers (one commit per CTA) and
+// on both TMEM_FULL barriers; each CTA drains its own 128 x 256 accumulator and releases
+// it on the even CTA's TMEM_EMPTY.  No load is multicast.
+//
+// Warp roles (320 threads per CTA): warp 0 = TMA producer, warp 1 = MMA issuer (even CTA)
+// and TMEM owner, warps 2..5 = epilogue, warps 6..9 = scale writers.
+#include "ft_internal.h"
+#include "ft_ptx.cuh"
+
+namespace ft {
+namespace gemm2 {
+
+constexpr int BM = 128;                  // rows per CTA (256 per pair)
+constexpr int BN = 256;                  // output columns per pair
+constexpr int BN_CTA = 128;              // B rows held by one CTA
+constexpr int BK_BYTES = 128;
+constexpr int STAGES = 5;
+constexpr int A_BYTES = BM * BK_BYTES;      // 16 KB
+constexpr int B_BYTES = BN_CTA * BK_BYTES;  // 16 KB
+constexpr int SFA_BYTES = 4 * 512;
+constexpr int SFB_BYTES = 2 * 4 * 512;
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;  // 38912
+constexpr int OFF_B = A_BYTES;
+constexpr int OFF_SFA = A_BYTES + B_BYTES;
+constexpr int OFF_SFB = OFF_SFA + SFA_BYTES;
+constexpr int EPI_BYTES = 32 * 64;
+constexpr int OFF_EPI = STAGES * STAGE_BYTES;
+constexpr int BAR_BYTES = 256;
+constexpr int SMEM_BYTES = OFF_EPI + 4 * EPI_BYTES + BAR_BYTES + 1024;
+constexpr int THREADS = 320;
+
+constexpr uint32_t TMEM_COLS = 512;
+constexpr uint32_t COL_ACC = 0;
+constexpr uint32_t COL_SFA = 256;                    // STAGES x 16 columns
+constexpr uint32_t COL_SFB = COL_SFA + STAGES * 16;  // STAGES x 32 columns
+
+static_assert(STAGE_BYTES % 1024 == 0, "stage must keep 1024-byte alignment");
+static_assert(SMEM_BYTES <= 232448, "exceeds 227 KB of dynamic shared memory");
+static_assert(COL_SFB + STAGES * 32 <= TMEM_COLS, "tensor memory overflow");
+
+__host__ __device__ constexpr int BAR_FULL(int s) { return s; }
+__host__ __device__ constexpr int BAR_EMPTY(int s) { return STAGES + s; }
+__host__ __device__ constexpr int BAR_SF_READY(int s) { return 2 * STAGES + s; }
+constexpr int BAR_TMEM_FULL = 3 * STAGES;
+constexpr int BAR_TMEM_EMPTY = 3 * STAGES + 1;
+constexpr int BAR_FINAL = 3 * STAGES + 2;
+constexpr int NUM_BARS = 3 * STAGES + 3;
+constexpr int OFF_TMEM_SLOT = 8 * NUM_BARS;
+constexpr int OFF_ABORT = OFF_TMEM_SLOT + 4;
+static_assert(OFF_ABORT + 4 <= BAR_BYTES, "barrier area overflow");
+
+__global__ void __launch_bounds__(THREADS, 1)
+    gemm_fp4_lowrank_pair_kernel(const __grid_constant__ CUtensorMap tmA,
+                                 const __grid_constant__ CUtensorMap tmB,
+                                 const __grid_constant__ CUtensorMap tmLA,
+                                 const __grid_constant__ CUtensorMap tmLB,
+                                 const __grid_constant__ CUtensorMap tmOut, const GemmFp4Args p) {
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw_u32 = smem_u32(smem_raw);
+    const uint32_t pad = (1024 - (raw_u32 & 1023)) & 1023;
+    uint8_t* base = smem_raw + pad;
+    const uint32_t base_u32 = raw_u32 + pad;
+    uint8_t* bar_area = base + OFF_EPI + 4 * EPI_BYTES;
+    auto bar = [&](int i) { return base_u32 + OFF_EPI + 4 * EPI_BYTES + 8 * i; };
+    auto stage = [&](int s) { return base_u32 + s * STAGE_BYTES; };
+    volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(bar_area + OFF_TMEM_SLOT);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(bar_area + OFF_ABORT);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();  // 0: the pair's MMA issuer
+    const int pair = blockIdx.x >> 1;
+    const int num_pairs = gridDim.x >> 1;
+    const int MB2 = p.M / (2 * BM);
+    const int NB = p.N / BN;
+    const int num_tiles = MB2 * NB;
+    const int KT = p.K / 256;
+    const int KLS = p.KL / 64;
+    const int k64 = p.K / 64;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < STAGES; ++i) {
+            mbar_init(bar(BAR_FULL(i)), 1);       // this CTA's producer (+ its bytes)
+            mbar_init(bar(BAR_EMPTY(i)), 1);      // the MMA issuer's commit
+            mbar_init(bar(BAR_SF_READY(i)), 8);   // 4 scale warps x 2 CTAs (even CTA's copy used)
+        }
+        mbar_init(bar(BAR_TMEM_FULL), 1);
+        mbar_init(bar(BAR_TMEM_EMPTY), 8);        // 4 epilogue warps x 2 CTAs (even CTA's copy used)
+        mbar_init(bar(BAR_FINAL), 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+        fence_proxy_async_smem();
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&tmA);
+        tma_prefetch_desc(&tmB);
+        if (KLS > 0) {
+            tma_prefetch_desc(&tmLA);
+            tma_prefetch_desc(&tmLB);
+        }
+    }
+    if (warp == 1) {
+        tmem_alloc_pair(smem_u32(const_cast<uint32_t*>(tmem_slot)), TMEM_COLS);
+        tmem_relinquish_pair();
+    }
+    tc_fence_before();
+    cluster_sync();  // barriers initialised and TMEM allocated in both CTAs
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        // ---------------------------------------------------------------- producer
+        if (lane == 0) {
+            int it = 0;
+            for (int t = pair; t < num_tiles && !*abort_flag; t += num_pairs) {
+                const int mb2 = t % MB2, nb = t / MB2;
+                const int m_band = mb2 * 2 + static_cast<int>(rank);            // this CTA's A rows
+                const int n_rows = nb * BN + BN_CTA * static_cast<int>(rank);  // this CTA's B rows
+                for (int kt = 0; kt < KT; ++kt, ++it) {
+                    const int s = it % STAGES;
+                    if (!mbar_wait(bar(BAR_EMPTY(s)), ((it / STAGES) & 1) ^ 1, abort_flag, p.status)) break;
+                    const uint32_t full = bar(BAR_FULL(s));
+                    const uint32_t st = stage(s);
+                    mbar_arrive_expect_tx(full, STAGE_BYTES);
+                    tma_load_2d(st, &tmA, full, kt * BK_BYTES, m_band * BM);
+                    tma_load_2d(st + OFF_B, &tmB, full, kt * BK_BYTES, n_rows);
+                    bulk_load(st + OFF_SFA, p.sfa + (static_cast<size_t>(m_band) * k64 + kt * 4) * 512,
+                              SFA_BYTES, full);
+#pragma unroll
+                    for (int rb = 0; rb < 2; ++rb)
+                        bulk_load(st + OFF_SFB + rb * 2048,
+                                  p.sfb + (static_cast<size_t>(nb * 2 + rb) * k64 + kt * 4) * 512, 2048,
+                                  full);
+                }
+                if (*abort_flag) break;
+                for (int kl = 0; kl < KLS; ++kl, ++it) {
+                    const int s = it % STAGES;
+                    if (!mbar_wait(bar(BAR_EMPTY(s)), ((it / STAGES) & 1) ^ 1, abort_flag, p.status)) break;
+                    const uint32_t full = bar(BAR_FULL(s));
+                    const uint32_t st = stage(s);
+                    mbar_arrive_expect_tx(full, A_BYTES + B_BYTES);
+                    tma_load_2d(st, &tmLA, full, kl * 64, m_band * BM);
+                    tma_load_2d(st + OFF_B, &tmLB, full, kl * 64, n_rows);
+                }
+            }
+            // Drain: every copy this thread issued has landed before the CTA may exit.
+            for (int j = it - 1; j >= 0 && j >= it - STAGES; --j) {
+                volatile int no_abort = 0;
+                mbar_wait(bar(BAR_FULL(j % STAGES)), (j / STAGES) & 1, &no_abort, p.status);
+            }
+        }
+    } else if (warp == 1) {
+        // ---------------------------------------------------------------- MMA issuer (even CTA)
+        if (rank == 0 && lane == 0) {
+            const uint32_t idesc4 = idesc_fp4_block16(2 * BM, BN);
+            const uint32_t idesc16 = idesc_bf16(2 * BM, BN);
+            int it = 0, ti = 0;
+            for (int t = pair; t < num_tiles && !*abort_flag; t += num_pairs, ++ti) {
+                if (!mbar_wait(bar(BAR_TMEM_EMPTY), (ti & 1) ^ 1, abort_flag, p.status)) break;
+                tc_fence_after();
+                bool ok = true;
+                for (int j = 0; j < KT + KLS; ++j, ++it) {
+                    const int s = it % STAGES;
+                    if (!mbar_wait(bar(BAR_SF_READY(s)), (it / STAGES) & 1, abort_flag, p.status)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t st = stage(s);
+                    const uint64_t ad = sdesc_kmajor_sw128(st);
+                    const uint64_t bd = sdesc_kmajor_sw128(st + OFF_B);
+                    if (j < KT) {
+                        const uint32_t sfa_t = tmem + COL_SFA + 16 * s;
+                        const uint32_t sfb_t = tmem + COL_SFB + 32 * s;
+#pragma unroll
+                        for (int i = 0; i < 4; ++i)
+                            mma_fp4_block16_pair(tmem + COL_ACC, ad + 2 * i, bd + 2 * i, idesc4, sfa_t + 4 * i,
+                                                 sfb_t + 8 * i, (j | i) != 0);
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < 4; ++i)
+                            mma_bf16_pair(tmem + COL_ACC, ad + 2 * i, bd + 2 * i, idesc16, 1);
+                    }
+                    tc_commit_pair(bar(BAR_EMPTY(s)));
+                    tc_commit_pair(mapa_shared(bar(BAR_EMPTY(s)), 1));
+                }
+                if (!ok) break;
+                tc_commit_pair(bar(BAR_TMEM_FULL));
+                tc_commit_pair(mapa_shared(bar(BAR_TMEM_FULL), 1));
+            }
+            // every MMA has retired (in both CTAs' tensor memory) before the pair tears down
+            tc_commit_pair(bar(BAR_FINAL));
+            volatile int no_abort = 0;
+            mbar_wait(bar(BAR_FINAL), 0, &no_abort, p.status);
+        }
+    } else if (warp >= 6) {
+        // ---------------------------------------------------------------- scale writers
+        // Same tensor-memory layout as the single-CTA kernel: lane l of quarter q holds row
+        // l of every 512-byte scale atom (4 columns per A k-block, 8 per B k-block).
+        const int q = warp & 3;
+        const uint32_t lane_base = tmem + (static_cast<uint32_t>(32 * q) << 16);
+        int it = 0;
+        for (int t = pair; t < num_tiles && !*abort_flag; t += num_pairs) {
+            bool ok = true;
+            for (int j = 0; j < KT + KLS; ++j, ++it) {
+                const int s = it % STAGES;
+                const uint32_t ph = (it / STAGES) & 1;
+                if (!mbar_wait(bar(BAR_FULL(s)), ph, abort_flag, p.status)) { ok = false; break; }
+                if (j < KT) {
+                    const uint8_t* st = base + s * STAGE_BYTES;
+                    uint32_t va[16], vb0[16], vb1[16];
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const uint4 a = *reinterpret_cast<const uint4*>(st + OFF_SFA + 512 * i + 16 * lane);
+                        const uint4 b0 = *reinterpret_cast<const uint4*>(st + OFF_SFB + 512 * i + 16 * lane);
+                        const uint4 b1 =
+                            *reinterpret_cast<const uint4*>(st + OFF_SFB + 2048 + 512 * i + 16 * lane);
+                        uint32_t* vb = i < 2 ? vb0 : vb1;
+                        const int o = 8 * (i & 1);
+                        va[4 * i] = a.x; va[4 * i + 1] = a.y; va[4 * i + 2] = a.z; va[4 * i + 3] = a.w;
+                        vb[o] = b0.x; vb[o + 1] = b0.y; vb[o + 2] = b0.z; vb[o + 3] = b0.w;
+                        vb[o + 4] = b1.x; vb[o + 5] = b1.y; vb[o + 6] = b1.z; vb[o + 7] = b1.w;
+                    }
+                    tmem_st_32x32b_x16(lane_base + COL_SFA + 16 * s, va);
+                    tmem_st_32x32b_x16(lane_base + COL_SFB + 32 * s, vb0);
+                    tmem_st_32x32b_x16(lane_base + COL_SFB + 32 * s + 16, vb1);
+                    tmem_st_wait();
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive_cluster(mapa_shared(bar(BAR_SF_READY(s)), 0));
+            }
+            if (!ok) break;
+        }
+    } else {
+        // ---------------------------------------------------------------- epilogue (both CTAs)
+        const int q = warp & 3;
+        const float ga = *p.ga, gb = *p.gb;
+        const float c = 1.0f / (ga * gb);
+        const uint32_t empty_even = mapa_shared(bar(BAR_TMEM_EMPTY), 0);
+        int ti = 0;
+        for (int t = pair; t < num_tiles && !*abort_flag; t += num_pairs, ++ti) {
+            const int mb2 = t % MB2, nb = t / MB2;
+            if (!mbar_wait(bar(BAR_TMEM_FULL), ti & 1, abort_flag, p.status)) break;
+            tc_fence_after();
+            const uint32_t lane_addr = tmem + COL_ACC + (static_cast<uint32_t>(32 * q) << 16);
+            const uint32_t stage_u32 = base_u32 + OFF_EPI + (warp - 2) * EPI_BYTES;
+            uint8_t* stage_ptr = base + OFF_EPI + (warp - 2) * EPI_BYTES;
+            uint32_t pk[BN / 2];
+#pragma unroll
+            for (int ch = 0; ch < BN / 32; ++ch) {
+                uint32_t v[32];
+                tmem_ld_32x32b_x32(lane_addr + ch * 32, v);
+                tmem_ld_wait();
+#pragma unroll
+                for (int jj = 0; jj < 16; ++jj)
+                    pk[ch * 16 + jj] = pack_bf16x2(__uint_as_float(v[2 * jj]) * c,
+                                                   __uint_as_float(v[2 * jj + 1]) * c);
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(empty_even);
+            const int row0 = (mb2 * 2 + static_cast<int>(rank)) * BM + 32 * q;
+#pragma unroll
+            for (int ch = 0; ch < BN / 32; ++ch) {
+                if (lane == 0) bulk_wait_group_read0();
+                __syncwarp();
+#pragma unroll
+                for (int c4 = 0; c4 < 4; ++c4) {
+                    const int phys = c4 ^ ((lane >> 1) & 3);
+                    *reinterpret_cast<uint4*>(stage_ptr + lane * 64 + phys * 16) =
+                        make_uint4(pk[ch * 16 + 4 * c4], pk[ch * 16 + 4 * c4 + 1], pk[ch * 16 + 4 * c4 + 2],
+                                   pk[ch * 16 + 4 * c4 + 3]);
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    tma_store_2d(&tmOut, stage_u32, nb * BN + ch * 32, row0);
+                    bulk_commit_group();
+                }
+            }
+        }
+        if (lane == 0) bulk_wait_group0();
+        __syncwarp();
+    }
+
+    // Both CTAs are done issuing (remote arrives, loads, MMAs retired) before the pair's
+    // tensor memory is released and either CTA exits.
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc_pair(tmem, TMEM_COLS);
+}
+
+}  // namespace gemm2
+
+cudaError_t launch_gemm_fp4_lowrank_pair(const CUtensorMap& tmA, const CUtensorMap& tmB,
+                                         const CUtensorMap& tmLA, const CUtensorMap& tmLB,
+                                         const CUtensorMap& tmOut, const GemmFp4Args& args, int num_sms,
+                                         cudaStream_t stream) {
+    using namespace gemm2;
+    static const cudaError_t attr = cudaFuncSetAttribute(
+        gemm_fp4_lowrank_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+    if (attr != cudaSuccess) return attr;
+    const int tiles = (args.M / (2 * BM)) * (args.N / BN);
+    int pairs = num_sms / 2;
+    if (pairs > tiles) pairs = tiles;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(2 * pairs));
+    cfg.blockDim = dim3(THREADS);
+    cfg.dynamicSmemBytes = SMEM_BYTES;
+    cfg.stream = stream;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeClusterDimension;
+    at[0].val.clusterDim.x = 2;
+    at[0].val.clusterDim.y = 1;
+    at[0].val.clusterDim.z = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    before_launch(K_GEMM, stream);
+    cudaError_t e =
+        cudaLaunchKernelEx(&cfg, gemm_fp4_lowrank_pair_kernel, tmA, tmB, tmLA, tmLB, tmOut, args);
+    after_launch(K_GEMM, stream);
+    if (e != cudaSuccess) return e;
+    return cudaGetLastError();
+}
+
+}  // namespace ft

@@ -33,6 +33,13 @@ cudaError_t launch_gemm_fp4_lowrank(const CUtensorMap& tmA, const CUtensorMap& t
                                     const CUtensorMap& tmOut, const GemmFp4Args& args, int num_sms,
                                     cudaStream_t stream);
 
+// The same GEMM computed by CTA pairs (cta_group::2), 256 x 256 tiles; needs M % 256 == 0.
+// tmB / tmLB boxes are 128 rows: each CTA of a pair loads half of the tile's N.
+cudaError_t launch_gemm_fp4_lowrank_pair(const CUtensorMap& tmA, const CUtensorMap& tmB,
+                                         const CUtensorMap& tmLA, const CUtensorMap& tmLB,
+                                         const CUtensorMap& tmOut, const GemmFp4Args& args, int num_sms,
+                                         cudaStream_t stream);
+
 // quantizer and helpers (ft_quant.cu)
 cudaError_t launch_amax(const void* x, bool is_f32, int64_t rows, int64_t cols, int64_t ld,
                         float* amax_out, int num_sms, cudaStream_t stream);
