@@ -123,6 +123,10 @@ __global__ void __launch_bounds__(THREADS, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    // TMEM is allocated before dependents may be scheduled on this SM (a waiting
+    // dependent never holds tensor memory this CTA still needs).
+    pdl_trigger();
+    pdl_wait();
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer
@@ -342,7 +346,9 @@ cudaError_t launch_gemm_fp4_lowrank(const CUtensorMap& tmA, const CUtensorMap& t
     const int tiles = (args.M / BM) * (args.N / BN);
     const int grid = tiles < num_sms ? tiles : num_sms;
     before_launch(K_GEMM, stream);
-    gemm_fp4_lowrank_kernel<<<grid, THREADS, SMEM_BYTES, stream>>>(tmA, tmB, tmLA, tmLB, tmOut, args);
+    const cudaError_t le = launch_k(gemm_fp4_lowrank_kernel, dim3(grid), dim3(THREADS), SMEM_BYTES,
+                                    stream, tmA, tmB, tmLA, tmLB, tmOut, args);
+    if (le != cudaSuccess) return le;
     after_launch(K_GEMM, stream);
     return cudaGetLastError();
 }

@@ -123,6 +123,10 @@ __global__ void __launch_bounds__(THREADS, 1)
     cluster_sync();  // barriers initialised and TMEM allocated in both CTAs
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    // TMEM is allocated before dependents may be scheduled on this SM (a waiting
+    // dependent never holds tensor memory this CTA still needs).
+    pdl_trigger();
+    pdl_wait();
 
     if (warp == 0) {
         // ---------------------------------------------------------------- producer
@@ -327,13 +331,15 @@ cudaError_t launch_gemm_fp4_lowrank_pair(const CUtensorMap& tmA, const CUtensorM
     cfg.blockDim = dim3(THREADS);
     cfg.dynamicSmemBytes = SMEM_BYTES;
     cfg.stream = stream;
-    cudaLaunchAttribute at[1];
+    cudaLaunchAttribute at[2];
     at[0].id = cudaLaunchAttributeClusterDimension;
     at[0].val.clusterDim.x = 2;
     at[0].val.clusterDim.y = 1;
     at[0].val.clusterDim.z = 1;
+    at[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // see launch_k
+    at[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = at;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     before_launch(K_GEMM, stream);
     cudaError_t e =
         cudaLaunchKernelEx(&cfg, gemm_fp4_lowrank_pair_kernel, tmA, tmB, tmLA, tmLB, tmOut, args);

@@ -15,6 +15,27 @@ enum KernelKind { K_GEMM = 0, K_QUANT = 1, K_AMAX = 2, K_LOWRANK = 3, K_LORA_DB 
 void before_launch(int kind, cudaStream_t stream);
 void after_launch(int kind, cudaStream_t stream);
 
+// Every kernel of the library is launched through launch_k with programmatic stream
+// serialization: the next kernel on the stream may be scheduled while this one still
+// runs (hiding launch latency and its prologue), and every kernel executes
+// griddepcontrol.wait before its first global-memory access, so results are as if the
+// kernels ran one after another.  Kernels call griddepcontrol.launch_dependents early.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_k(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                     Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, static_cast<Args&&>(args)...);
+}
+
 struct GemmFp4Args {
     const uint8_t* sfa;     // tensor-core scale layout of A (rows M, cols K)
     const uint8_t* sfb;     // tensor-core scale layout of B (rows N, cols K)

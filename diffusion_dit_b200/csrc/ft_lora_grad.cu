@@ -87,6 +87,10 @@ __global__ void __launch_bounds__(THREADS, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    // TMEM is allocated before dependents may be scheduled on this SM (a waiting
+    // dependent never holds tensor memory this CTA still needs).
+    pdl_trigger();
+    pdl_wait();
 
     if (warp == 0) {
         if (lane == 0) {
@@ -158,6 +162,8 @@ __global__ void __launch_bounds__(THREADS, 1)
 // out = s * sum_split (D[f][j] + D[f][r + j]); transposed (out[j][f]) for dA.
 __global__ void lora_grad_finalize_kernel(const float* __restrict__ partial, int splits, int F, int NBW, int r,
                                           float s, bool transpose_out, float* __restrict__ out) {
+    pdl_trigger();
+    pdl_wait();
     const int total = F * r;
     for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < total; i += gridDim.x * blockDim.x) {
         int f, j;
@@ -184,6 +190,8 @@ __global__ void lora_grad_finalize_kernel(const float* __restrict__ partial, int
 // V' [M, NBW] bf16 = [hi(V), lo(V), 0] from fp32 V = src[:, c0 : c0 + r] (row stride ld).
 __global__ void build_hilo_kernel(const float* __restrict__ src, int ld, int c0, int r, int M, int NBW,
                                   __nv_bfloat16* __restrict__ dst) {
+    pdl_trigger();
+    pdl_wait();
     const int total = M * NBW;
     for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < total; i += gridDim.x * blockDim.x) {
         const int m = i / NBW;
@@ -221,7 +229,9 @@ cudaError_t launch_lora_grad(const CUtensorMap& tmP, const CUtensorMap& tmV, con
     if (attr != cudaSuccess) return attr;
     dim3 grid(static_cast<unsigned>(a.F / lg::BF), static_cast<unsigned>(splits));
     before_launch(kind, stream);
-    lg::lora_grad_kernel<<<grid, lg::THREADS, L.smem_bytes, stream>>>(tmP, tmV, a);
+    const cudaError_t le = launch_k(lg::lora_grad_kernel, dim3(grid), dim3(lg::THREADS),
+                                    L.smem_bytes, stream, tmP, tmV, a);
+    if (le != cudaSuccess) return le;
     after_launch(kind, stream);
     return cudaGetLastError();
 }
@@ -231,8 +241,10 @@ cudaError_t launch_lora_grad_finalize(const float* partial, int splits, int64_t 
     int64_t g = (F * r + 255) / 256;
     if (g > 148 * 8) g = 148 * 8;
     before_launch(K_OTHER, stream);
-    lg::lora_grad_finalize_kernel<<<static_cast<unsigned>(g), 256, 0, stream>>>(
-        partial, splits, static_cast<int>(F), NBW, r, s, transpose_out, out);
+    const cudaError_t le = launch_k(lg::lora_grad_finalize_kernel, dim3(static_cast<unsigned>(g)),
+                                    dim3(256), 0, stream, partial, splits, static_cast<int>(F), NBW,
+                                    r, s, transpose_out, out);
+    if (le != cudaSuccess) return le;
     after_launch(K_OTHER, stream);
     return cudaGetLastError();
 }
@@ -242,8 +254,10 @@ cudaError_t launch_build_hilo(const float* src, int64_t ld, int c0, int r, int64
     int64_t g = (M * NBW + 255) / 256;
     if (g > 148 * 8) g = 148 * 8;
     before_launch(K_OTHER, stream);
-    lg::build_hilo_kernel<<<static_cast<unsigned>(g), 256, 0, stream>>>(src, static_cast<int>(ld), c0, r,
-                                                                        static_cast<int>(M), NBW, dst);
+    const cudaError_t le = launch_k(lg::build_hilo_kernel, dim3(static_cast<unsigned>(g)),
+                                    dim3(256), 0, stream, src, static_cast<int>(ld), c0, r,
+                                    static_cast<int>(M), NBW, dst);
+    if (le != cudaSuccess) return le;
     after_launch(K_OTHER, stream);
     return cudaGetLastError();
 }

@@ -22,6 +22,8 @@ namespace {
 
 // One thread per (row, j < R): fixed-order sum over the splits, then the hi/lo operands.
 __global__ void lowrank_finalize_kernel(const LowRankFinalizeArgs a) {
+    pdl_trigger();
+    pdl_wait();
     const int rows = static_cast<int>(a.rows);
     const int total = rows * a.R;
     const float g = (a.cat != nullptr) ? __fmul_rn(*a.ga, *a.gb) : 1.0f;
@@ -68,6 +70,8 @@ __global__ void build_factors_kernel(const __nv_bfloat16* __restrict__ ls_down,
                                      int r, int Rp, int KL, __nv_bfloat16* __restrict__ dn,
                                      __nv_bfloat16* __restrict__ upcat, __nv_bfloat16* __restrict__ upt,
                                      __nv_bfloat16* __restrict__ dntcat) {
+    pdl_trigger();
+    pdl_wait();
     const int R = r_s + r;
     const __nv_bfloat16 zero = __float2bfloat16_rn(0.0f);
     const int stride = gridDim.x * blockDim.x;
@@ -125,7 +129,10 @@ static int grid_cap(int64_t work, int threads, int cap) {
 
 cudaError_t launch_lowrank_finalize(const LowRankFinalizeArgs& a, cudaStream_t stream) {
     before_launch(K_LOWRANK, stream);
-    lowrank_finalize_kernel<<<grid_cap(a.rows * a.R, 256, 148 * 8), 256, 0, stream>>>(a);
+    const cudaError_t le = launch_k(lowrank_finalize_kernel,
+                                    dim3(grid_cap(a.rows * a.R, 256, 148 * 8)), dim3(256), 0,
+                                    stream, a);
+    if (le != cudaSuccess) return le;
     after_launch(K_LOWRANK, stream);
     return cudaGetLastError();
 }
@@ -136,9 +143,10 @@ cudaError_t launch_build_factors(const __nv_bfloat16* ls_down, const __nv_bfloat
                                  __nv_bfloat16* upcat, __nv_bfloat16* upt, __nv_bfloat16* dntcat,
                                  cudaStream_t stream) {
     before_launch(K_OTHER, stream);
-    build_factors_kernel<<<148 * 4, 256, 0, stream>>>(ls_down, lora_a, ls_up, lora_b, static_cast<int>(N),
-                                                      static_cast<int>(K), r_s, r, Rp, KL, dn, upcat, upt,
-                                                      dntcat);
+    const cudaError_t le = launch_k(build_factors_kernel, dim3(148 * 4), dim3(256), 0, stream,
+                                    ls_down, lora_a, ls_up, lora_b, static_cast<int>(N),
+                                    static_cast<int>(K), r_s, r, Rp, KL, dn, upcat, upt, dntcat);
+    if (le != cudaSuccess) return le;
     after_launch(K_OTHER, stream);
     return cudaGetLastError();
 }

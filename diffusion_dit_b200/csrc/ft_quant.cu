@@ -57,6 +57,8 @@ __device__ __forceinline__ void load8(const float* p, float (&v)[8]) {
 template <typename T>
 __global__ void __launch_bounds__(256) amax_kernel(const T* __restrict__ x, int64_t rows, int64_t cols,
                                                    int64_t ld, unsigned* __restrict__ out) {
+    pdl_trigger();
+    pdl_wait();
     const int64_t vec_per_row = cols / 8;
     const int64_t nvec = rows * vec_per_row;
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
@@ -101,6 +103,8 @@ __global__ void __launch_bounds__(256) quant_block16_kernel(const T* __restrict_
                                                             uint8_t* __restrict__ codes,
                                                             uint8_t* __restrict__ scales,
                                                             float* __restrict__ g_out) {
+    pdl_trigger();
+    pdl_wait();
     const int lane = threadIdx.x & 31;
     const int64_t nbc = cols / 16;
     const int64_t nblocks = (rows / 16) * nbc;
@@ -141,6 +145,8 @@ __global__ void __launch_bounds__(256) quant_block16_kernel(const T* __restrict_
 // atom, (row m, column block b) sits at 16 (m % 32) + 4 ((m % 128) / 32) + b % 4.
 __global__ void expand_scales_kernel(const uint8_t* __restrict__ scales, int64_t rows, int64_t cols,
                                      uint8_t* __restrict__ sf) {
+    pdl_trigger();
+    pdl_wait();
     const int64_t total = rows * (cols / 16);
     const int64_t atoms_per_band = cols / 64;
     for (int64_t o = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; o < total;
@@ -159,6 +165,8 @@ __global__ void expand_scales_kernel(const uint8_t* __restrict__ scales, int64_t
 __global__ void transpose_q_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ scales,
                                    int64_t rows, int64_t cols, uint8_t* __restrict__ codes_t,
                                    uint8_t* __restrict__ scales_t) {
+    pdl_trigger();
+    pdl_wait();
     // output codes_t [cols, rows/2]
     const int64_t total = cols * (rows / 2);
     for (int64_t o = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; o < total;
@@ -178,15 +186,23 @@ __global__ void transpose_q_kernel(const uint8_t* __restrict__ codes, const uint
     }
 }
 
-__global__ void copy_scalar_kernel(const float* src, float* dst) { *dst = *src; }
+__global__ void copy_scalar_kernel(const float* src, float* dst) {
+    pdl_trigger();
+    pdl_wait();
+    *dst = *src;
+}
 
 __global__ void encode_e2m1_kernel(const float* __restrict__ v, int64_t n, uint8_t* __restrict__ out) {
+    pdl_trigger();
+    pdl_wait();
     for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n;
          i += (int64_t)gridDim.x * blockDim.x)
         out[i] = static_cast<uint8_t>(cvt_e2m1x2(v[i], 0.0f) & 15u);
 }
 
 __global__ void encode_ue4m3_kernel(const float* __restrict__ v, int64_t n, uint8_t* __restrict__ out) {
+    pdl_trigger();
+    pdl_wait();
     for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n;
          i += (int64_t)gridDim.x * blockDim.x)
         out[i] = static_cast<uint8_t>(cvt_ue4m3(v[i]));
@@ -214,6 +230,8 @@ __device__ __forceinline__ float gelu_tanh_grad_f(float p) {
 
 __global__ void gelu_fwd_kernel(const __nv_bfloat16* __restrict__ p, __nv_bfloat16* __restrict__ h,
                                 int64_t n) {
+    pdl_trigger();
+    pdl_wait();
     for (int64_t i = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) * 8; i < n;
          i += (int64_t)gridDim.x * blockDim.x * 8) {
         float v[8];
@@ -229,6 +247,8 @@ __global__ void gelu_fwd_kernel(const __nv_bfloat16* __restrict__ p, __nv_bfloat
 
 __global__ void gelu_bwd_kernel(const __nv_bfloat16* __restrict__ p, const __nv_bfloat16* __restrict__ dh,
                                 __nv_bfloat16* __restrict__ dp, int64_t n) {
+    pdl_trigger();
+    pdl_wait();
     for (int64_t i = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) * 8; i < n;
          i += (int64_t)gridDim.x * blockDim.x * 8) {
         float v[8], d[8];
@@ -258,12 +278,13 @@ cudaError_t launch_amax(const void* x, bool is_f32, int64_t rows, int64_t cols, 
     if (e != cudaSuccess) return e;
     const int grid = grid_for(rows * cols / 32, 256, num_sms * 4);
     before_launch(K_AMAX, stream);
-    if (is_f32)
-        amax_kernel<float><<<grid, 256, 0, stream>>>(static_cast<const float*>(x), rows, cols, ld,
-                                                      reinterpret_cast<unsigned*>(amax_out));
-    else
-        amax_kernel<__nv_bfloat16><<<grid, 256, 0, stream>>>(
-            static_cast<const __nv_bfloat16*>(x), rows, cols, ld, reinterpret_cast<unsigned*>(amax_out));
+    unsigned* out = reinterpret_cast<unsigned*>(amax_out);
+    const cudaError_t le =
+        is_f32 ? launch_k(amax_kernel<float>, dim3(grid), dim3(256), 0, stream, static_cast<const float*>(x),
+                          rows, cols, ld, out)
+               : launch_k(amax_kernel<__nv_bfloat16>, dim3(grid), dim3(256), 0, stream,
+                          static_cast<const __nv_bfloat16*>(x), rows, cols, ld, out);
+    if (le != cudaSuccess) return le;
     after_launch(K_AMAX, stream);
     return cudaGetLastError();
 }
@@ -274,12 +295,12 @@ cudaError_t launch_quant_block16(const void* x, bool is_f32, int64_t rows, int64
     const int64_t nblocks = (rows / 16) * (cols / 16);
     const int grid = grid_for(nblocks * 32, 256, num_sms * 8);
     before_launch(K_QUANT, stream);
-    if (is_f32)
-        quant_block16_kernel<float><<<grid, 256, 0, stream>>>(static_cast<const float*>(x), rows, cols,
-                                                               ld, amax, codes, scales, g_out);
-    else
-        quant_block16_kernel<__nv_bfloat16><<<grid, 256, 0, stream>>>(
-            static_cast<const __nv_bfloat16*>(x), rows, cols, ld, amax, codes, scales, g_out);
+    const cudaError_t le =
+        is_f32 ? launch_k(quant_block16_kernel<float>, dim3(grid), dim3(256), 0, stream,
+                          static_cast<const float*>(x), rows, cols, ld, amax, codes, scales, g_out)
+               : launch_k(quant_block16_kernel<__nv_bfloat16>, dim3(grid), dim3(256), 0, stream,
+                          static_cast<const __nv_bfloat16*>(x), rows, cols, ld, amax, codes, scales, g_out);
+    if (le != cudaSuccess) return le;
     after_launch(K_QUANT, stream);
     return cudaGetLastError();
 }
@@ -288,7 +309,9 @@ cudaError_t launch_expand_scales(const uint8_t* scales, int64_t rows, int64_t co
                                  cudaStream_t stream) {
     const int grid = grid_for(rows * cols / 16, 256, 148 * 8);
     before_launch(K_OTHER, stream);
-    expand_scales_kernel<<<grid, 256, 0, stream>>>(scales, rows, cols, sf_mma);
+    const cudaError_t le = launch_k(expand_scales_kernel, dim3(grid), dim3(256), 0, stream, scales,
+                                    rows, cols, sf_mma);
+    if (le != cudaSuccess) return le;
     after_launch(K_OTHER, stream);
     return cudaGetLastError();
 }
@@ -297,35 +320,44 @@ cudaError_t launch_transpose_q(const uint8_t* codes, const uint8_t* scales, int6
                                uint8_t* codes_t, uint8_t* scales_t, cudaStream_t stream) {
     const int grid = grid_for(rows * cols / 2, 256, 148 * 8);
     before_launch(K_OTHER, stream);
-    transpose_q_kernel<<<grid, 256, 0, stream>>>(codes, scales, rows, cols, codes_t, scales_t);
+    const cudaError_t le = launch_k(transpose_q_kernel, dim3(grid), dim3(256), 0, stream, codes,
+                                    scales, rows, cols, codes_t, scales_t);
+    if (le != cudaSuccess) return le;
     after_launch(K_OTHER, stream);
     return cudaGetLastError();
 }
 
 cudaError_t launch_copy_scalar(const float* src, float* dst, cudaStream_t stream) {
     before_launch(K_OTHER, stream);
-    copy_scalar_kernel<<<1, 1, 0, stream>>>(src, dst);
+    const cudaError_t le = launch_k(copy_scalar_kernel, dim3(1), dim3(1), 0, stream, src, dst);
+    if (le != cudaSuccess) return le;
     after_launch(K_OTHER, stream);
     return cudaGetLastError();
 }
 
 cudaError_t launch_encode_e2m1(const float* v, int64_t n, uint8_t* out, cudaStream_t stream) {
     before_launch(K_OTHER, stream);
-    encode_e2m1_kernel<<<grid_for(n, 256, 148 * 16), 256, 0, stream>>>(v, n, out);
+    const cudaError_t le = launch_k(encode_e2m1_kernel, dim3(grid_for(n, 256, 148 * 16)), dim3(256),
+                                    0, stream, v, n, out);
+    if (le != cudaSuccess) return le;
     after_launch(K_OTHER, stream);
     return cudaGetLastError();
 }
 
 cudaError_t launch_encode_ue4m3(const float* v, int64_t n, uint8_t* out, cudaStream_t stream) {
     before_launch(K_OTHER, stream);
-    encode_ue4m3_kernel<<<grid_for(n, 256, 148 * 16), 256, 0, stream>>>(v, n, out);
+    const cudaError_t le = launch_k(encode_ue4m3_kernel, dim3(grid_for(n, 256, 148 * 16)),
+                                    dim3(256), 0, stream, v, n, out);
+    if (le != cudaSuccess) return le;
     after_launch(K_OTHER, stream);
     return cudaGetLastError();
 }
 
 cudaError_t launch_gelu_fwd(const __nv_bfloat16* p, __nv_bfloat16* h, int64_t n, cudaStream_t stream) {
     before_launch(K_OTHER, stream);
-    gelu_fwd_kernel<<<grid_for(n / 8, 256, 148 * 8), 256, 0, stream>>>(p, h, n);
+    const cudaError_t le = launch_k(gelu_fwd_kernel, dim3(grid_for(n / 8, 256, 148 * 8)), dim3(256),
+                                    0, stream, p, h, n);
+    if (le != cudaSuccess) return le;
     after_launch(K_OTHER, stream);
     return cudaGetLastError();
 }
@@ -333,7 +365,9 @@ cudaError_t launch_gelu_fwd(const __nv_bfloat16* p, __nv_bfloat16* h, int64_t n,
 cudaError_t launch_gelu_bwd(const __nv_bfloat16* p, const __nv_bfloat16* dh, __nv_bfloat16* dp,
                             int64_t n, cudaStream_t stream) {
     before_launch(K_OTHER, stream);
-    gelu_bwd_kernel<<<grid_for(n / 8, 256, 148 * 8), 256, 0, stream>>>(p, dh, dp, n);
+    const cudaError_t le = launch_k(gelu_bwd_kernel, dim3(grid_for(n / 8, 256, 148 * 8)), dim3(256),
+                                    0, stream, p, dh, dp, n);
+    if (le != cudaSuccess) return le;
     after_launch(K_OTHER, stream);
     return cudaGetLastError();
 }
@@ -346,6 +380,8 @@ namespace {
 // Self-test of the bounded wait every pipelined kernel uses: wait on an mbarrier that
 // nothing will ever complete, give up after limit_ns, report FT_ERR_TIMEOUT.
 __global__ void bounded_wait_selftest_kernel(uint64_t limit_ns, int* status) {
+    pdl_trigger();
+    pdl_wait();
     __shared__ __align__(8) uint64_t bar;
     __shared__ int abort_flag;
     if (threadIdx.x == 0) {
@@ -362,7 +398,9 @@ __global__ void bounded_wait_selftest_kernel(uint64_t limit_ns, int* status) {
 
 cudaError_t launch_bounded_wait_selftest(uint64_t limit_ns, int* status, cudaStream_t stream) {
     before_launch(K_OTHER, stream);
-    bounded_wait_selftest_kernel<<<1, 32, 0, stream>>>(limit_ns, status);
+    const cudaError_t le = launch_k(bounded_wait_selftest_kernel, dim3(1), dim3(32), 0, stream,
+                                    limit_ns, status);
+    if (le != cudaSuccess) return le;
     after_launch(K_OTHER, stream);
     return cudaGetLastError();
 }

@@ -100,6 +100,10 @@ __global__ void __launch_bounds__(THREADS, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = has_mma ? *tmem_slot : 0;
+    // TMEM is allocated before dependents may be scheduled on this SM (a waiting
+    // dependent never holds tensor memory this CTA still needs).
+    pdl_trigger();
+    pdl_wait();
 
     if (warp == 0) {
         if (lane == 0) {
@@ -281,7 +285,9 @@ cudaError_t launch_quant_down(const CUtensorMap& tmX, const CUtensorMap& tmW, co
     if (attr != cudaSuccess) return attr;
     dim3 grid(static_cast<unsigned>(a.rows / 128), static_cast<unsigned>(splits));
     before_launch(K_QUANT, stream);
-    qf::quant_down_kernel<<<grid, qf::THREADS, L.smem_bytes, stream>>>(tmX, tmW, a);
+    const cudaError_t le = launch_k(qf::quant_down_kernel, dim3(grid), dim3(qf::THREADS),
+                                    L.smem_bytes, stream, tmX, tmW, a);
+    if (le != cudaSuccess) return le;
     after_launch(K_QUANT, stream);
     return cudaGetLastError();
 }
