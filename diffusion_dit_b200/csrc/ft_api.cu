@@ -185,12 +185,12 @@ __nv_bfloat16* bfm(void* p) { return static_cast<__nv_bfloat16*>(p); }
 // Rp > 0, its down-projection partials x w^T (w: bf16 [Rp, cols]) in one fused kernel.
 // Returns the number of column slices (partials) through *splits.
 ft_status quantize_operand(const void* x, int64_t rows, int64_t cols, int64_t ld, const float* amax_or_null,
-                           float* amax_slot, uint8_t* codes, uint8_t* scales, uint8_t* sf, float* g,
+                           float* amax_slot, bool amax_slot_cleared, uint8_t* codes, uint8_t* scales, uint8_t* sf, float* g,
                            const void* w, int Rp, float* partial, int* splits, int* status,
                            const DeviceInfo& dev, cudaStream_t st) {
     const float* amax = amax_or_null;
     if (!amax) {
-        FT_CUDA(ft::launch_amax(x, false, rows, cols, ld, amax_slot, dev.num_sms, st));
+        FT_CUDA(ft::launch_amax(x, false, rows, cols, ld, amax_slot, amax_slot_cleared, dev.num_sms, st));
         amax = amax_slot;
     }
     CUtensorMap tX, tW;
@@ -379,12 +379,14 @@ ft_status fourtune_quantize_block16(const void* x_dev, int32_t x_dtype, int64_t 
     const bool f32 = x_dtype == FT_DTYPE_F32;
     if (fused_ok) {
         const int Rp = padded_rank(r_down);
+        ft::PrologueExtras ex;
+        if (!amax_or_null) ex.zero_slot = amax_slot;
         if (Rp > 0)
             FT_CUDA(ft::launch_build_factors(bf(down_dev), nullptr, nullptr, nullptr, 0, cols, r_down, 0, Rp, 0,
-                                             bfm(W + qw.down), nullptr, nullptr, nullptr, st));
+                                             bfm(W + qw.down), nullptr, nullptr, nullptr, &ex, st));
         int splits = 1;
         float* partial = reinterpret_cast<float*>(W + qw.partial);
-        FT_TRY(quantize_operand(x_dev, rows, cols, ld, amax_or_null, amax_slot, out->codes, out->scales,
+        FT_TRY(quantize_operand(x_dev, rows, cols, ld, amax_or_null, amax_slot, Rp > 0, out->codes, out->scales,
                                 out->sf_mma, out->g, W + qw.down, Rp, partial, &splits, status, dev, st));
         if (Rp > 0) {
             ft::LowRankFinalizeArgs f{};
@@ -401,7 +403,7 @@ ft_status fourtune_quantize_block16(const void* x_dev, int32_t x_dtype, int64_t 
     } else {
         const float* amax = amax_or_null;
         if (!amax) {
-            FT_CUDA(ft::launch_amax(x_dev, f32, rows, cols, ld, amax_slot, dev.num_sms, st));
+            FT_CUDA(ft::launch_amax(x_dev, f32, rows, cols, ld, amax_slot, false, dev.num_sms, st));
             amax = amax_slot;
         }
         FT_CUDA(ft::launch_quant_block16(x_dev, f32, rows, cols, ld, amax, out->codes, out->scales, out->g,
@@ -445,12 +447,15 @@ ft_status fourtune_linear_fwd(const ft_linear* L, const void* x_dev, int64_t M, 
     // Eq. (2): the factors of this step ([Ls_down; A] and [Ls_up, B]; A, B train),
     // then Q(X) fused with T = X [Ls_down; A]^T, then the 4-bit GEMM with the
     // up-projections in its accumulator.
+    // The factor kernel also clears the tensor-max slot (no memset node between kernels).
+    ft::PrologueExtras ex;
+    if (!amax_or_null) ex.zero_slot = scal + SC_AMAX_X;
     if (R > 0)
         FT_CUDA(ft::launch_build_factors(bf(L->ls_down), bf(L->lora_a), bf(L->ls_up), bf(L->lora_b), N, K,
                                          L->r_s, L->r, Rp, KL, bfm(W + w.dn), bfm(W + w.upcat), nullptr,
-                                         nullptr, st));
+                                         nullptr, &ex, st));
     int splits = 1;
-    FT_TRY(quantize_operand(x_dev, M, K, K, amax_or_null, scal + SC_AMAX_X, W + w.qx_codes, W + w.qx_scales,
+    FT_TRY(quantize_operand(x_dev, M, K, K, amax_or_null, scal + SC_AMAX_X, R > 0, W + w.qx_codes, W + w.qx_scales,
                             W + w.qx_sf, scal + SC_G_X, W + w.dn, Rp, partial, &splits, status, dev, st));
     if (R > 0) {
         ft::LowRankFinalizeArgs f{};
@@ -500,12 +505,25 @@ ft_status fourtune_linear_bwd(const ft_linear* L, const void* x_dev, const float
 
     // Eq. (3): Q(G) fused with U = G [Ls_up, B], the dX GEMM through Q(R)^T with
     // U [Ls_down; A] in its accumulator, then the adapter gradients.
+    // The factor kernel also builds dB's operand V' = [hi, lo, 0] of T_lora (an input of
+    // this call) and clears the tensor-max slot.
+    ft::PrologueExtras ex;
+    if (!amax_or_null) ex.zero_slot = scal + SC_AMAX_G;
+    if (L->r > 0) {
+        ex.hilo_src = t_saved_dev;
+        ex.hilo_ld = R;
+        ex.hilo_c0 = L->r_s;
+        ex.hilo_r = L->r;
+        ex.hilo_M = static_cast<int>(M);
+        ex.hilo_NBW = lora_width(L->r);
+        ex.hilo_dst = bfm(W + w.vcat);
+    }
     if (R > 0)
         FT_CUDA(ft::launch_build_factors(bf(L->ls_down), bf(L->lora_a), bf(L->ls_up), bf(L->lora_b), N, K,
                                          L->r_s, L->r, Rp, KL, nullptr, nullptr, bfm(W + w.upt),
-                                         bfm(W + w.dntcat), st));
+                                         bfm(W + w.dntcat), &ex, st));
     int splits = 1;
-    FT_TRY(quantize_operand(dy_dev, M, N, N, amax_or_null, scal + SC_AMAX_G, W + w.qg_codes, W + w.qg_scales,
+    FT_TRY(quantize_operand(dy_dev, M, N, N, amax_or_null, scal + SC_AMAX_G, R > 0, W + w.qg_codes, W + w.qg_scales,
                             W + w.qg_sf, scal + SC_G_G, W + w.upt, Rp, partial, &splits, status, dev, st));
     if (R > 0) {
         ft::LowRankFinalizeArgs f{};
@@ -543,7 +561,6 @@ ft_status fourtune_linear_bwd(const ft_linear* L, const void* x_dev, const float
         g.partial = gpart;
         g.status = status;
         // dB over the output features n
-        FT_CUDA(ft::launch_build_hilo(t_saved_dev, R, L->r_s, L->r, M, NBW, vcat, st));
         FT_TRY(make_tmap(&tP, dy_dev, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, N, M, N * 2, 64, 64));
         int sp = ft::lora_grad_splits(M, N, dev.num_sms);
         g.F = N;

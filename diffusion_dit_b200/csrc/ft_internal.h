@@ -62,8 +62,10 @@ cudaError_t launch_gemm_fp4_lowrank_pair(const CUtensorMap& tmA, const CUtensorM
                                          cudaStream_t stream);
 
 // quantizer and helpers (ft_quant.cu)
+// amax_out accumulates with atomicMax: it is cleared here unless slot_cleared (an earlier
+// kernel of the same call cleared it).
 cudaError_t launch_amax(const void* x, bool is_f32, int64_t rows, int64_t cols, int64_t ld,
-                        float* amax_out, int num_sms, cudaStream_t stream);
+                        float* amax_out, bool slot_cleared, int num_sms, cudaStream_t stream);
 cudaError_t launch_quant_block16(const void* x, bool is_f32, int64_t rows, int64_t cols, int64_t ld,
                                  const float* amax, uint8_t* codes, uint8_t* scales, float* g_out,
                                  int num_sms, cudaStream_t stream);
@@ -117,13 +119,25 @@ struct LowRankFinalizeArgs {
 };
 cudaError_t launch_lowrank_finalize(const LowRankFinalizeArgs& a, cudaStream_t stream);
 
-// Build the concatenated low-rank factors used by the forward and backward GEMMs.
-// dn and upt get Rp rows (rows R..Rp-1 zero) so they can feed an MMA of width Rp.
+// Side jobs of the first kernel of a layer call (they depend only on the call's inputs):
+// V' = [hi(V), lo(V), 0] (bf16 [M, NBW]) of the fp32 columns V = src[:, c0 : c0 + r]
+// (row stride ld) for the adapter gradient dB, and clearing the tensor-max slot that the
+// call's max kernel accumulates into.
+struct PrologueExtras {
+    const float* hilo_src = nullptr;
+    int hilo_ld = 0, hilo_c0 = 0, hilo_r = 0, hilo_M = 0, hilo_NBW = 0;
+    __nv_bfloat16* hilo_dst = nullptr;
+    float* zero_slot = nullptr;
+};
+
+// Build the concatenated low-rank factors used by the forward and backward GEMMs (and
+// run the side jobs in `extra`, which may be null).  dn and upt get Rp rows (rows
+// R..Rp-1 zero) so they can feed an MMA of width Rp.
 cudaError_t launch_build_factors(const __nv_bfloat16* ls_down, const __nv_bfloat16* lora_a,
                                  const __nv_bfloat16* ls_up, const __nv_bfloat16* lora_b, int64_t N,
                                  int64_t K, int r_s, int r, int Rp, int KL, __nv_bfloat16* dn,
                                  __nv_bfloat16* upcat, __nv_bfloat16* upt, __nv_bfloat16* dntcat,
-                                 cudaStream_t stream);
+                                 const PrologueExtras* extra, cudaStream_t stream);
 
 // adapter gradients on the tensor cores (ft_lora_grad.cu):
 //   partial[split][f][c] = sum over the split's tokens m of P[m, f] V'[m, c]
@@ -140,7 +154,5 @@ cudaError_t launch_lora_grad(const CUtensorMap& tmP, const CUtensorMap& tmV, con
                              int kind, cudaStream_t stream);
 cudaError_t launch_lora_grad_finalize(const float* partial, int splits, int64_t F, int NBW, int r, float s,
                                       bool transpose_out, float* out, cudaStream_t stream);
-cudaError_t launch_build_hilo(const float* src, int64_t ld, int c0, int r, int64_t M, int NBW,
-                              __nv_bfloat16* dst, cudaStream_t stream);
 
 }  // namespace ft

@@ -187,25 +187,6 @@ __global__ void lora_grad_finalize_kernel(const float* __restrict__ partial, int
     }
 }
 
-// V' [M, NBW] bf16 = [hi(V), lo(V), 0] from fp32 V = src[:, c0 : c0 + r] (row stride ld).
-__global__ void build_hilo_kernel(const float* __restrict__ src, int ld, int c0, int r, int M, int NBW,
-                                  __nv_bfloat16* __restrict__ dst) {
-    pdl_trigger();
-    pdl_wait();
-    const int total = M * NBW;
-    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < total; i += gridDim.x * blockDim.x) {
-        const int m = i / NBW;
-        const int c = i - m * NBW;
-        __nv_bfloat16 o = __float2bfloat16_rn(0.0f);
-        if (c < 2 * r) {
-            const float v = src[m * ld + c0 + (c < r ? c : c - r)];
-            const __nv_bfloat16 hi = __float2bfloat16_rn(v);
-            o = c < r ? hi : __float2bfloat16_rn(v - __bfloat162float(hi));
-        }
-        dst[i] = o;
-    }
-}
-
 }  // namespace lg
 
 int lora_grad_splits(int64_t M, int64_t F, int num_sms) {
@@ -244,19 +225,6 @@ cudaError_t launch_lora_grad_finalize(const float* partial, int splits, int64_t 
     const cudaError_t le = launch_k(lg::lora_grad_finalize_kernel, dim3(static_cast<unsigned>(g)),
                                     dim3(256), 0, stream, partial, splits, static_cast<int>(F), NBW,
                                     r, s, transpose_out, out);
-    if (le != cudaSuccess) return le;
-    after_launch(K_OTHER, stream);
-    return cudaGetLastError();
-}
-
-cudaError_t launch_build_hilo(const float* src, int64_t ld, int c0, int r, int64_t M, int NBW,
-                              __nv_bfloat16* dst, cudaStream_t stream) {
-    int64_t g = (M * NBW + 255) / 256;
-    if (g > 148 * 8) g = 148 * 8;
-    before_launch(K_OTHER, stream);
-    const cudaError_t le = launch_k(lg::build_hilo_kernel, dim3(static_cast<unsigned>(g)),
-                                    dim3(256), 0, stream, src, static_cast<int>(ld), c0, r,
-                                    static_cast<int>(M), NBW, dst);
     if (le != cudaSuccess) return le;
     after_launch(K_OTHER, stream);
     return cudaGetLastError();

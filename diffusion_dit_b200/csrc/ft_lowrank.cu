@@ -69,7 +69,7 @@ __global__ void build_factors_kernel(const __nv_bfloat16* __restrict__ ls_down,
                                      const __nv_bfloat16* __restrict__ lora_b, int N, int K, int r_s,
                                      int r, int Rp, int KL, __nv_bfloat16* __restrict__ dn,
                                      __nv_bfloat16* __restrict__ upcat, __nv_bfloat16* __restrict__ upt,
-                                     __nv_bfloat16* __restrict__ dntcat) {
+                                     __nv_bfloat16* __restrict__ dntcat, const PrologueExtras x) {
     pdl_trigger();
     pdl_wait();
     const int R = r_s + r;
@@ -116,6 +116,21 @@ __global__ void build_factors_kernel(const __nv_bfloat16* __restrict__ ls_down,
             const int k = i / KL, c = i % KL;
             dntcat[i] = c < R ? dn_at(c, k) : (c < 2 * R ? dn_at(c - R, k) : zero);
         }
+    // side jobs: V' = [hi(V), lo(V), 0] for dB, and the cleared tensor-max slot
+    if (x.hilo_dst) {
+        const int w = x.hilo_NBW, rr = x.hilo_r;
+        for (int i = t0; i < x.hilo_M * w; i += stride) {
+            const int m = i / w, c = i - m * w;
+            __nv_bfloat16 o = zero;
+            if (c < 2 * rr) {
+                const float v = x.hilo_src[m * x.hilo_ld + x.hilo_c0 + (c < rr ? c : c - rr)];
+                const __nv_bfloat16 hi = __float2bfloat16_rn(v);
+                o = c < rr ? hi : __float2bfloat16_rn(v - __bfloat162float(hi));
+            }
+            x.hilo_dst[i] = o;
+        }
+    }
+    if (x.zero_slot && t0 == 0) *x.zero_slot = 0.0f;
 }
 
 }  // namespace
@@ -141,11 +156,12 @@ cudaError_t launch_build_factors(const __nv_bfloat16* ls_down, const __nv_bfloat
                                  const __nv_bfloat16* ls_up, const __nv_bfloat16* lora_b, int64_t N,
                                  int64_t K, int r_s, int r, int Rp, int KL, __nv_bfloat16* dn,
                                  __nv_bfloat16* upcat, __nv_bfloat16* upt, __nv_bfloat16* dntcat,
-                                 cudaStream_t stream) {
+                                 const PrologueExtras* extra, cudaStream_t stream) {
+    const PrologueExtras x = extra ? *extra : PrologueExtras{};
     before_launch(K_OTHER, stream);
     const cudaError_t le = launch_k(build_factors_kernel, dim3(148 * 4), dim3(256), 0, stream,
                                     ls_down, lora_a, ls_up, lora_b, static_cast<int>(N),
-                                    static_cast<int>(K), r_s, r, Rp, KL, dn, upcat, upt, dntcat);
+                                    static_cast<int>(K), r_s, r, Rp, KL, dn, upcat, upt, dntcat, x);
     if (le != cudaSuccess) return le;
     after_launch(K_OTHER, stream);
     return cudaGetLastError();

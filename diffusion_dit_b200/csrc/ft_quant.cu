@@ -273,9 +273,11 @@ int grid_for(int64_t work, int threads, int cap) {
 }  // namespace
 
 cudaError_t launch_amax(const void* x, bool is_f32, int64_t rows, int64_t cols, int64_t ld,
-                        float* amax_out, int num_sms, cudaStream_t stream) {
-    cudaError_t e = cudaMemsetAsync(amax_out, 0, sizeof(float), stream);
-    if (e != cudaSuccess) return e;
+                        float* amax_out, bool slot_cleared, int num_sms, cudaStream_t stream) {
+    if (!slot_cleared) {
+        const cudaError_t e = cudaMemsetAsync(amax_out, 0, sizeof(float), stream);
+        if (e != cudaSuccess) return e;
+    }
     const int grid = grid_for(rows * cols / 32, 256, num_sms * 4);
     before_launch(K_AMAX, stream);
     unsigned* out = reinterpret_cast<unsigned*>(amax_out);

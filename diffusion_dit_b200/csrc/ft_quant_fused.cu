@@ -9,11 +9,14 @@
 //   * the MMA warp multiplies it with the matching W tile on the tensor cores
 //     (tcgen05.mma kind::f16, accumulator [128 x Rp] fp32 in TMEM), giving this CTA's
 //     partial of T = X W^T;
-//   * eight quantizer warps read the same tile from shared memory and emit the E2M1
-//     codes, the compact block scales and the tensor-core scale layout (same
-//     arithmetic, bit for bit, as quant_block16_kernel in ft_quant.cu).
-// A stage is released when the MMA has finished reading it (tcgen05.commit) and all
-// eight quantizer warps have arrived.  At the end four warps drain the accumulator
+//   * a set of eight quantizer warps (one per 16-row block-row) reads the same tile
+//     from shared memory and emits the E2M1 codes, the compact block scales and the
+//     tensor-core scale layout (same arithmetic, bit for bit, as quant_block16_kernel
+//     in ft_quant.cu).  Two such sets take the stages in turn: a warp's work on one
+//     stage is a chain of dependent steps (loads, shuffles, scale, convert, stores), so
+//     two stages in flight double the quantizer's throughput per SM.
+// A stage is released when the MMA has finished reading it (tcgen05.commit) and the
+// eight warps of its set have arrived.  At the end four warps drain the accumulator
 // into partials[split][row][Rp]; ft_lowrank.cu sums the splits in a fixed order.
 #include "ft_internal.h"
 #include "ft_ptx.cuh"
@@ -24,8 +27,13 @@ namespace qf {
 constexpr int BM = 128;
 constexpr int BKE = 64;                 // bf16 columns per stage (one 128-byte row)
 constexpr int X_BYTES = BM * 128;       // 16 KB
-constexpr int NQ = 8;                   // quantizer warps
-constexpr int THREADS = 32 * (2 + NQ);  // producer, MMA, quantizers
+#ifndef FT_QUANT_SETS
+#define FT_QUANT_SETS 2
+#endif
+constexpr int NQ_SET = 8;                  // quantizer warps per set: one per 16-row block-row
+constexpr int NSETS = FT_QUANT_SETS;       // sets take the stages in turn (k % NSETS)
+constexpr int NQ = NQ_SET * NSETS;         // quantizer warps
+constexpr int THREADS = 32 * (2 + NQ);     // producer, MMA, quantizers
 constexpr int MAX_STAGES = 8;
 constexpr int BAR_BYTES = 768;           // barriers, TMEM slot, abort flag, inv table at +160
 
@@ -80,7 +88,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     if (threadIdx.x == 0) {
         for (int i = 0; i < S; ++i) {
             mbar_init(bar(i), 1);
-            mbar_init(bar(S + i), NQ + (has_mma ? 1 : 0));
+            mbar_init(bar(S + i), NQ_SET + (has_mma ? 1 : 0));  // one set of quantizer warps + MMA
         }
         mbar_init(bar(2 * S), 1);
         mbar_init(bar(2 * S + 1), 1);
@@ -150,7 +158,8 @@ __global__ void __launch_bounds__(THREADS, 1)
         // shuffle steps inside the 8-lane group, and each lane derives its block's scale
         // once.  The per-tensor table inv[sb] = fl32(g / val(sb)) replaces the division
         // per block; the block max / 6 uses div6_bf16 (exact for bf16 inputs).
-        const int qw = warp - 2;
+        const int qw = (warp - 2) % NQ_SET;  // block-row of the band
+        const int set = (warp - 2) / NQ_SET;  // this warp takes stages k with k % NSETS == set
         float g = 1.0f;
         bool degenerate = true;
         {
@@ -176,7 +185,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         const int rB = rA + 8;
         const int64_t cbs = p.cols / 16;
         const int64_t atoms_per_band = p.cols / 64;
-        for (int k = 0; k < nk; ++k) {
+        for (int k = set; k < nk; k += NSETS) {
             const int s = k % S;
             if (!mbar_wait(bar(s), (k / S) & 1, abort_flag, p.status)) break;
             const uint8_t* tile = base + s * L.stage_bytes;
@@ -227,7 +236,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             if (lane == 0) mbar_arrive(bar(S + s));
         }
         // ------------------------------------------------------------ T partial epilogue
-        if (has_mma && qw < 4) {
+        if (has_mma && warp < 6) {
             const int q = warp & 3;
             if (mbar_wait(bar(2 * S), 0, abort_flag, p.status)) {
                 tc_fence_after();
