@@ -138,6 +138,24 @@ def run_reference(args, spec):
     print(json.dumps(line), flush=True)
 
 
+def gemm_traffic():
+    """DRAM bytes per launch of the 4-bit GEMM from the committed ncu summary, or None
+    when the kernel's sources have changed since those counters were taken."""
+    import hashlib
+    import re
+    here = os.path.dirname(os.path.abspath(__file__))
+    try:
+        text = open(os.path.join(here, "profiles", "gemm_fp4_lowrank_pair_kernel.md")).read()
+        m = re.search(r"traffic_bytes_per_launch: (\d+) sources_sha256_16: ([0-9a-f]{16})", text)
+        src = b"".join(open(os.path.join(here, "diffusion_dit_b200", "csrc", f), "rb").read()
+                       for f in ("ft_gemm2.cu", "ft_ptx.cuh"))
+    except OSError:
+        return None
+    if not m or hashlib.sha256(src).hexdigest()[:16] != m.group(2):
+        return None
+    return int(m.group(1))
+
+
 def blas_threads():
     try:
         from threadpoolctl import threadpool_info
@@ -370,7 +388,7 @@ def main():
         fp4_peak = bf16_peak * NOMINAL_FP4_OVER_BF16
         gemm_avg = statistics.mean(gemm_ms)
         achieved = 2.0 * M * N * K / (gemm_avg * 1e-3) / 1e12
-        traffic = None
+        traffic = gemm_traffic()  # ncu dram read + write per launch (mean of fwd and dX)
         # quantizer: X [M, K] and G [M, N] alternate; algorithmic bytes per element:
         # 2 (read bf16) + 0.5 (codes) + 1/256 (block scales); the tensor max is one more read.
         elems = [M * K, M * N] * Kst
