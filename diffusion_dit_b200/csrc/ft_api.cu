@@ -503,8 +503,8 @@ ft_status fourtune_linear_bwd(const ft_linear* L, const void* x_dev, const float
     const int Rp = padded_rank(R);
     float* partial = reinterpret_cast<float*>(W + w.partial);
 
-    // Eq. (3): Q(G) fused with U = G [Ls_up, B], the dX GEMM through Q(R)^T with
-    // U [Ls_down; A] in its accumulator, then the adapter gradients.
+    // Eq. (3): Q(G) fused with U = G [Ls_up, B], the adapter gradients, then the dX
+    // GEMM through Q(R)^T with U [Ls_down; A] in its accumulator.
     // The factor kernel also builds dB's operand V' = [hi, lo, 0] of T_lora (an input of
     // this call) and clears the tensor-max slot.
     ft::PrologueExtras ex;
@@ -545,8 +545,6 @@ ft_status fourtune_linear_bwd(const ft_linear* L, const void* x_dev, const float
         }
         FT_CUDA(ft::launch_lowrank_finalize(f, st));
     }
-    FT_TRY(run_gemm(W + w.qg_codes, W + w.qg_sf, scal + SC_G_G, L->qr_t, bf(W + w.ucat), bf(W + w.dntcat), KL,
-                    M, K, N, dx_dev, status, dev, st));
     if (L->r > 0) {
         // Section 3.2 adapter gradients: dB = s G^T T_lora, dA = s U_lora^T X, on the
         // tensor cores, reading G and X straight (MN-major operands).
@@ -576,6 +574,10 @@ ft_status fourtune_linear_bwd(const ft_linear* L, const void* x_dev, const float
         FT_CUDA(ft::launch_lora_grad(tP, tV, g, sp, ft::K_LORA_DA, st));
         FT_CUDA(ft::launch_lora_grad_finalize(gpart, sp, K, NBW, L->r, L->lora_scale, true, da_dev, st));
     }
+    // The dX GEMM goes last: the adapter gradients read G again, and right after Q(G)
+    // most of G is still in L2, which the GEMM's operand and output traffic would evict.
+    FT_TRY(run_gemm(W + w.qg_codes, W + w.qg_sf, scal + SC_G_G, L->qr_t, bf(W + w.ucat), bf(W + w.dntcat), KL,
+                    M, K, N, dx_dev, status, dev, st));
     return FT_OK;
 }
 
