@@ -503,8 +503,8 @@ ft_status fourtune_linear_bwd(const ft_linear* L, const void* x_dev, const float
     const int Rp = padded_rank(R);
     float* partial = reinterpret_cast<float*>(W + w.partial);
 
-    // Eq. (3): Q(G) fused with U = G [Ls_up, B], the adapter gradients, then the dX
-    // GEMM through Q(R)^T with U [Ls_down; A] in its accumulator.
+    // Eq. (3): dB (with max |G|), Q(G) fused with U = G [Ls_up, B], dA, then the dX GEMM
+    // through Q(R)^T with U [Ls_down; A] in its accumulator.
     // The factor kernel also builds dB's operand V' = [hi, lo, 0] of T_lora (an input of
     // this call) and clears the tensor-max slot.
     ft::PrologueExtras ex;
@@ -522,8 +522,35 @@ ft_status fourtune_linear_bwd(const ft_linear* L, const void* x_dev, const float
         FT_CUDA(ft::launch_build_factors(bf(L->ls_down), bf(L->lora_a), bf(L->ls_up), bf(L->lora_b), N, K,
                                          L->r_s, L->r, Rp, KL, nullptr, nullptr, bfm(W + w.upt),
                                          bfm(W + w.dntcat), &ex, st));
+    // Section 3.2 adapter gradients: dB = s G^T T_lora, dA = s U_lora^T X, on the tensor
+    // cores, reading G and X straight (MN-major operands).  dB goes first: its kernel
+    // reads every element of G once and also takes max |G| (into the slot the factor
+    // kernel cleared), so Q(G) needs no separate pass over G; G is then still in L2.
+    const int NBW = lora_width(L->r);
+    float* gpart = reinterpret_cast<float*>(W + w.gpartial);
+    ft::LoraGradArgs g{};
+    g.NBW = NBW;
+    g.tmem_cols = tmem_cols_for(NBW);
+    g.partial = gpart;
+    g.status = status;
+    const float* amax_g = amax_or_null;
+    if (L->r > 0) {
+        CUtensorMap tP, tV;
+        FT_TRY(make_tmap(&tV, W + w.vcat, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, NBW, M, NBW * 2, 64, 64));
+        FT_TRY(make_tmap(&tP, dy_dev, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, N, M, N * 2, 64, 64));
+        const int sp = ft::lora_grad_splits(M, N, dev.num_sms);
+        g.F = N;
+        g.tokens_per_split = static_cast<int>(M / sp);
+        if (!amax_or_null) {
+            g.amax_out = reinterpret_cast<unsigned*>(scal + SC_AMAX_G);
+            amax_g = scal + SC_AMAX_G;
+        }
+        FT_CUDA(ft::launch_lora_grad(tP, tV, g, sp, ft::K_LORA_DB, st));
+        g.amax_out = nullptr;
+        FT_CUDA(ft::launch_lora_grad_finalize(gpart, sp, N, NBW, L->r, L->lora_scale, false, db_dev, st));
+    }
     int splits = 1;
-    FT_TRY(quantize_operand(dy_dev, M, N, N, amax_or_null, scal + SC_AMAX_G, R > 0, W + w.qg_codes, W + w.qg_scales,
+    FT_TRY(quantize_operand(dy_dev, M, N, N, amax_g, scal + SC_AMAX_G, R > 0, W + w.qg_codes, W + w.qg_scales,
                             W + w.qg_sf, scal + SC_G_G, W + w.upt, Rp, partial, &splits, status, dev, st));
     if (R > 0) {
         ft::LowRankFinalizeArgs f{};
@@ -541,41 +568,22 @@ ft_status fourtune_linear_bwd(const ft_linear* L, const void* x_dev, const float
         f.KL = KL;
         if (L->r > 0) {  // U_lora's hi/lo operand for dA, written by the same pass
             f.lora_cat = bfm(W + w.ucat_lora);
-            f.NBW = lora_width(L->r);
+            f.NBW = NBW;
         }
         FT_CUDA(ft::launch_lowrank_finalize(f, st));
     }
     if (L->r > 0) {
-        // Section 3.2 adapter gradients: dB = s G^T T_lora, dA = s U_lora^T X, on the
-        // tensor cores, reading G and X straight (MN-major operands).
-        const int NBW = lora_width(L->r);
-        __nv_bfloat16* vcat = bfm(W + w.vcat);
-        float* gpart = reinterpret_cast<float*>(W + w.gpartial);
-        CUtensorMap tP, tV;
-        FT_TRY(make_tmap(&tV, vcat, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, NBW, M, NBW * 2, 64, 64));
-        ft::LoraGradArgs g{};
-        g.NBW = NBW;
-        g.tmem_cols = tmem_cols_for(NBW);
-        g.partial = gpart;
-        g.status = status;
-        // dB over the output features n
-        FT_TRY(make_tmap(&tP, dy_dev, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, N, M, N * 2, 64, 64));
-        int sp = ft::lora_grad_splits(M, N, dev.num_sms);
-        g.F = N;
-        g.tokens_per_split = static_cast<int>(M / sp);
-        FT_CUDA(ft::launch_lora_grad(tP, tV, g, sp, ft::K_LORA_DB, st));
-        FT_CUDA(ft::launch_lora_grad_finalize(gpart, sp, N, NBW, L->r, L->lora_scale, false, db_dev, st));
         // dA over the input features k (V' = U_lora's hi/lo, written by the split sum)
+        CUtensorMap tP, tV;
         FT_TRY(make_tmap(&tV, W + w.ucat_lora, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, NBW, M, NBW * 2, 64, 64));
         FT_TRY(make_tmap(&tP, x_dev, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, K, M, K * 2, 64, 64));
-        sp = ft::lora_grad_splits(M, K, dev.num_sms);
+        const int sp = ft::lora_grad_splits(M, K, dev.num_sms);
         g.F = K;
         g.tokens_per_split = static_cast<int>(M / sp);
         FT_CUDA(ft::launch_lora_grad(tP, tV, g, sp, ft::K_LORA_DA, st));
         FT_CUDA(ft::launch_lora_grad_finalize(gpart, sp, K, NBW, L->r, L->lora_scale, true, da_dev, st));
     }
-    // The dX GEMM goes last: the adapter gradients read G again, and right after Q(G)
-    // most of G is still in L2, which the GEMM's operand and output traffic would evict.
+    // The dX GEMM goes last: the GEMM's operand and output traffic would evict G from L2.
     FT_TRY(run_gemm(W + w.qg_codes, W + w.qg_sf, scal + SC_G_G, L->qr_t, bf(W + w.ucat), bf(W + w.dntcat), KL,
                     M, K, N, dx_dev, status, dev, st));
     return FT_OK;

@@ -148,6 +148,9 @@ struct LoraGradArgs {
     uint32_t tmem_cols;      // power of two >= max(32, NBW)
     float* partial;          // [splits, F, NBW]
     int* status;
+    // optional: max |P| over every element of P (each is read by exactly one CTA),
+    // accumulated with atomicMax on the float's bits into a slot cleared beforehand
+    unsigned* amax_out;
 };
 int lora_grad_splits(int64_t M, int64_t F, int num_sms);
 cudaError_t launch_lora_grad(const CUtensorMap& tmP, const CUtensorMap& tmV, const LoraGradArgs& a, int splits,

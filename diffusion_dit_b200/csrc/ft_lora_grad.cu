@@ -13,6 +13,10 @@
 //
 // One CTA = 128 features x a slice of the tokens; partials[split][f][NBW] fp32 are
 // summed in a fixed order by lora_grad_finalize_kernel (deterministic).
+//
+// When asked (amax_out), the four epilogue warps, idle until the final drain, also take
+// max |P| over every tile that lands: with dB computed first in the backward pass this
+// gives the tensor max of G for Q(G) without a separate pass over G.
 #include "ft_internal.h"
 #include "ft_ptx.cuh"
 
@@ -67,7 +71,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     if (threadIdx.x == 0) {
         for (int i = 0; i < S; ++i) {
             mbar_init(bar(i), 1);
-            mbar_init(bar(S + i), 1);
+            mbar_init(bar(S + i), 1 + (p.amax_out ? 4 : 0));  // MMA commit (+ 4 max warps)
         }
         mbar_init(bar(2 * S), 1);
         mbar_init(bar(2 * S + 1), 1);
@@ -136,6 +140,30 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
     } else {
         const int q = warp & 3;
+        if (p.amax_out) {
+            // max |x| of each landed P tile (16 KB: 8 x 16 bytes per thread), fp32 fmaxf
+            // as in amax_kernel (a NaN never wins); the stage is released after the read
+            float m = 0.0f;
+            const int t = threadIdx.x - 64;  // 0..127
+            for (int k = 0; k < nk; ++k) {
+                const int s = k % S;
+                if (!mbar_wait(bar(s), (k / S) & 1, abort_flag, p.status)) break;
+                const uint8_t* tile = base + s * L.stage_bytes;
+#pragma unroll
+                for (int i = 0; i < A_BYTES / (128 * 16); ++i) {
+                    const uint4 w = *reinterpret_cast<const uint4*>(tile + (i * 128 + t) * 16);
+                    const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        m = fmaxf(m, fmaxf(fabsf(bf16lo_to_f32(ws[e])), fabsf(bf16hi_to_f32(ws[e]))));
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar(S + s));
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+            if (lane == 0) atomicMax(p.amax_out, __float_as_uint(m));
+        }
         if (mbar_wait(bar(2 * S), 0, abort_flag, p.status)) {
             tc_fence_after();
             const int f = f0 + 32 * q + lane;
