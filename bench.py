@@ -30,6 +30,12 @@ sys.path.insert(0, ROOT)
 
 METRIC = "W4A4G4 linear fwd+bwd TFLOPS & % FP4 roofline; quantizer GB/s vs HBM"
 NOMINAL_FP4_OVER_BF16 = 4.0   # 9 / 2.25 PFLOP/s dense (B200 spec ratio)
+NOMINAL_FP4_TFLOPS = 9000.0   # B200 dense FP4 spec
+
+# single-layer workloads (one FourTune linear, forward + backward); the default is the
+# attention QKV projection, the others are the MLP and single-stream layers
+WORKLOADS = {"qkv": "FLUX_QKV", "mlp_up": "FLUX_MLP_UP", "mlp_down": "FLUX_MLP_DOWN",
+             "single_l1": "FLUX_SS_L1", "single_l2": "FLUX_SS_L2"}
 
 
 def layer_flops(M, K, N, r_s, r):
@@ -37,6 +43,15 @@ def layer_flops(M, K, N, r_s, r):
     fp4 = 4.0 * M * N * K                              # forward GEMM + dX GEMM
     bf16 = 2.0 * R * (2 * M * K + 2 * M * N) + 2.0 * r * (M * N + M * K)
     return fp4, bf16
+
+
+def pass_flops(M, K, N, r_s, r):
+    """(forward, backward) algorithmic FLOPs: FP4 GEMM + low-rank down / up projections,
+    plus dB and dA in the backward."""
+    R = r_s + r
+    fwd = 2.0 * M * N * K + 2.0 * R * (M * K + M * N)
+    bwd = 2.0 * M * N * K + 2.0 * R * (M * N + M * K) + 2.0 * r * (M * N + M * K)
+    return fwd, bwd
 
 
 def peaks():
@@ -156,6 +171,37 @@ def gemm_traffic():
     return int(m.group(1))
 
 
+def cublaslt_nvfp4_tflops(M, N, K, iters=20):
+    """cuBLASLt's block-scaled NVFP4 GEMM (torch._scaled_mm, bf16 out) at one shape: the
+    attainable rate of a library 4-bit GEMM on this GPU, for context.  None if the
+    installed torch cannot run it."""
+    import torch
+    try:
+        dev = torch.device("cuda")
+        g = torch.Generator(device=dev).manual_seed(0)
+        a = torch.randint(0, 256, (M, K // 2), dtype=torch.uint8, device=dev, generator=g)
+        b = torch.randint(0, 256, (N, K // 2), dtype=torch.uint8, device=dev, generator=g)
+        a, b = a.view(torch.float4_e2m1fn_x2), b.view(torch.float4_e2m1fn_x2)
+        rup = lambda x, m: (x + m - 1) // m * m  # noqa: E731
+        sa = torch.ones(rup(M, 128) * rup(K // 16, 4), device=dev).to(torch.float8_e4m3fn)
+        sb = torch.ones(rup(N, 128) * rup(K // 16, 4), device=dev).to(torch.float8_e4m3fn)
+        mm = lambda: torch._scaled_mm(a, b.t(), scale_a=sa, scale_b=sb, out_dtype=torch.bfloat16)  # noqa: E731
+        mm()
+        flush = torch.empty(128 * 1024 * 1024, dtype=torch.float32, device=dev)
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ts = []
+        for _ in range(iters):
+            flush.zero_()
+            s.record()
+            mm()
+            e.record()
+            torch.cuda.synchronize()
+            ts.append(s.elapsed_time(e))
+        return 2.0 * M * N * K / (statistics.median(ts) * 1e-3) / 1e12
+    except Exception:
+        return None
+
+
 def blas_threads():
     try:
         from threadpoolctl import threadpool_info
@@ -205,11 +251,13 @@ def main():
     ap.add_argument("--graph", dest="graph", action="store_true", default=True,
                     help="replay each step as a captured CUDA graph (default)")
     ap.add_argument("--no-graph", dest="graph", action="store_false")
+    ap.add_argument("--workload", default="qkv", choices=sorted(WORKLOADS),
+                    help="single-layer workload (default: the attention QKV projection)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
     from diffusion_dit_b200 import workloads as wl
-    spec = wl.FLUX_QKV
+    spec = getattr(wl, WORKLOADS[args.workload])
     if args.impl == "reference":
         run_reference(args, spec)
         return
@@ -275,11 +323,19 @@ def main():
         for k, (b_, a_) in kev.items():
             ft.time_next_launch(k, b_[0], a_[0])
         ft.linear_fwd(w, x, ws, y=y, t_saved=t)
-        for k, (b_, a_) in kev.items():
-            ft.time_next_launch(k, b_[1], a_[1])
+        # the backward has no separate tensor-max launch: its adapter-gradient kernel
+        # takes max |G| on the way
+        for k in (ft.FT_KERNEL_GEMM, ft.FT_KERNEL_QUANT):
+            ft.time_next_launch(k, kev[k][0][1], kev[k][1][1])
         ft.linear_bwd(w, x, t, dy, ws, dx=dx, da=da, db=db)
 
-    graph = graph_k = None
+    def fwd_kernels():
+        ft.linear_fwd(w, x, ws, y=y, t_saved=t)
+
+    def bwd_kernels():
+        ft.linear_bwd(w, x, t, dy, ws, dx=dx, da=da, db=db)
+
+    graph = graph_k = graph_f = graph_b = None
     launches_per_step = None
     if args.graph:
         # One step (forward + backward: all of the library's kernels) captured once as a
@@ -296,11 +352,16 @@ def main():
         graph_k = torch.cuda.CUDAGraph()
         with torch.cuda.graph(graph_k):
             one_step_with_events()
+        # forward alone and backward alone, for the per-pass figures
+        graph_f, graph_b = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph_f):
+            fwd_kernels()
+        with torch.cuda.graph(graph_b):
+            bwd_kernels()
         for _ in range(args.warmup):
-            flush.zero_()
-            graph.replay()
-            flush.zero_()
-            graph_k.replay()
+            for g_ in (graph, graph_k, graph_f, graph_b):
+                flush.zero_()
+                g_.replay()
         torch.cuda.synchronize()
 
     gemm_ms, quant_ms, amax_ms = [], [], []
@@ -336,13 +397,27 @@ def main():
             ev_ke[i].record()
             # the per-launch events are reused by every step: read them before the next one
             torch.cuda.synchronize()
-            for k, dst in ((ft.FT_KERNEL_GEMM, gemm_ms), (ft.FT_KERNEL_QUANT, quant_ms), (ft.FT_KERNEL_AMAX, amax_ms)):
+            for k, dst in ((ft.FT_KERNEL_GEMM, gemm_ms), (ft.FT_KERNEL_QUANT, quant_ms)):
                 b_, a_ = kev[k]
                 dst.extend([b_[0].elapsed_time(a_[0]), b_[1].elapsed_time(a_[1])])
+            amax_ms.append(kev[ft.FT_KERNEL_AMAX][0][0].elapsed_time(kev[ft.FT_KERNEL_AMAX][1][0]))
         torch.cuda.synchronize()
+        ms_per_step_events = sum(ev_ks[i].elapsed_time(ev_ke[i]) for i in range(Kst)) / Kst
+        # per-pass pass: the forward alone, then the backward alone, as many steps each
+        pass_ms = {"fwd": [], "bwd": []}
+        for name, g_, fn in (("fwd", graph_f, fwd_kernels), ("bwd", graph_b, bwd_kernels)):
+            for i in range(Kst):
+                flush.zero_()
+                ev_ks[i].record()
+                if g_ is not None:
+                    g_.replay()
+                else:
+                    fn()
+                ev_ke[i].record()
+            torch.cuda.synchronize()
+            pass_ms[name] = [ev_ks[i].elapsed_time(ev_ke[i]) for i in range(Kst)]
     if ws.device_status() != 0:
         raise RuntimeError("device status reports a timeout in the timed region")
-    ms_per_step_events = sum(ev_ks[i].elapsed_time(ev_ke[i]) for i in range(Kst)) / Kst
 
     total_ms = sum(ev_s[i].elapsed_time(ev_e[i]) for i in range(Kst))
     tm = torch.tensor([total_ms], dtype=torch.float64, device=dev)
@@ -388,13 +463,20 @@ def main():
         fp4_peak = bf16_peak * NOMINAL_FP4_OVER_BF16
         gemm_avg = statistics.mean(gemm_ms)
         achieved = 2.0 * M * N * K / (gemm_avg * 1e-3) / 1e12
-        traffic = gemm_traffic()  # ncu dram read + write per launch (mean of fwd and dX)
+        # ncu dram read + write per launch (mean of fwd and dX), captured on this workload
+        traffic = gemm_traffic() if args.workload == "qkv" else None
         # quantizer: X [M, K] and G [M, N] alternate; algorithmic bytes per element:
-        # 2 (read bf16) + 0.5 (codes) + 1/256 (block scales); the tensor max is one more read.
+        # 2 (read bf16) + 0.5 (codes) + 1/256 (block scales).  The tensor max of X is one
+        # more read of X by its own kernel; max |G| is taken by the dB kernel.
         elems = [M * K, M * N] * Kst
         qbytes = sum(e * (2.0 + 0.5 + 1.0 / 256) for e in elems)
         q_gbs = qbytes / (sum(quant_ms) * 1e-3) / 1e9
-        qa_gbs = (qbytes + sum(2.0 * e for e in elems)) / ((sum(quant_ms) + sum(amax_ms)) * 1e-3) / 1e9
+        qa_gbs = (qbytes + 2.0 * M * K * Kst) / ((sum(quant_ms) + sum(amax_ms)) * 1e-3) / 1e9
+        fl_f, fl_b = pass_flops(M, K, N, spec.r_s, spec.r)
+        fwd_ms, bwd_ms = statistics.median(pass_ms["fwd"]), statistics.median(pass_ms["bwd"])
+        lt_fwd = cublaslt_nvfp4_tflops(M, N, K)
+        lt_dx = cublaslt_nvfp4_tflops(M, K, N)
+        lt_mean = (lt_fwd + lt_dx) / 2 if lt_fwd and lt_dx else None
         line = {
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": Kst,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
@@ -407,11 +489,17 @@ def main():
                          "peak_source": f"{src} bf16 {bf16_peak} TFLOP/s x {NOMINAL_FP4_OVER_BF16} "
                                         f"(nominal fp4/bf16 ratio)",
                          "avg_launch_ms": gemm_avg,
+                         "frac_of_nominal_9pf": achieved / NOMINAL_FP4_TFLOPS,
+                         "cublaslt_nvfp4_tflops": {"fwd_shape": lt_fwd, "dx_shape": lt_dx},
+                         "frac_of_cublaslt": achieved / lt_mean if lt_mean else None,
                          "timing": "CUDA events around each launch, recorded in a second pass of "
                                    f"{Kst} steps (that pass: {ms_per_step_events:.4f} ms per step)"},
             "quantizer": {"kernel": "quant_down_kernel (quantizer fused with the down-projection)", "achieved_gbs": q_gbs,
                           "with_amax_pass_gbs": qa_gbs, "peak_gbs": hbm, "frac": q_gbs / hbm,
                           "frac_with_amax": qa_gbs / hbm, "avg_launch_ms": statistics.mean(quant_ms)},
+            "per_pass": {"fwd_ms": fwd_ms, "fwd_tflops": fl_f / (fwd_ms * 1e-3) / 1e12,
+                         "bwd_ms": bwd_ms, "bwd_tflops": fl_b / (bwd_ms * 1e-3) / 1e12,
+                         "timing": f"median of {Kst} replays of a forward-only / backward-only graph"},
             "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
             "gpu_launches": launches,
             "launch_mode": "cuda_graph_replay" if graph is not None else "stream",
