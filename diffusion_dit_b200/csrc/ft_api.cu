@@ -218,10 +218,12 @@ ft_status quantize_operand(const void* x, int64_t rows, int64_t cols, int64_t ld
     return FT_OK;
 }
 
-// One 4-bit GEMM with its low-rank tail: out[M, N] from A (M x K) and B (N x K).
+// One 4-bit GEMM with its low-rank tail: out[M, N] from A (M x K) and B (N x K); with
+// act_out, also act_out = bf16(gelu_tanh(out)) and max |act_out| into *act_amax.
 ft_status run_gemm(const uint8_t* a_codes, const uint8_t* a_sf, const float* ga, const ft_fp4& b,
                    const __nv_bfloat16* la, const __nv_bfloat16* lb, int KL, int64_t M, int64_t N,
-                   int64_t K, void* out, int* status, const DeviceInfo& dev, cudaStream_t st) {
+                   int64_t K, void* out, int* status, const DeviceInfo& dev, cudaStream_t st,
+                   void* act_out = nullptr, float* act_amax = nullptr) {
     // CTA pairs (256 x 256 tiles) when M allows, single CTAs (128 x 256) otherwise.
     const bool pair = (M % 256) == 0 && dev.num_sms >= 2;
     const uint32_t b_rows = pair ? 128 : 256;
@@ -235,8 +237,13 @@ ft_status run_gemm(const uint8_t* a_codes, const uint8_t* a_sf, const float* ga,
         tLA = tA;
         tLB = tB;
     }
-    CUtensorMap tOut;
+    CUtensorMap tOut, tAct;
     FT_TRY(make_tmap(&tOut, out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, N, M, N * 2, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B));
+    if (act_out)
+        FT_TRY(make_tmap(&tAct, act_out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, N, M, N * 2, 32, 32,
+                         CU_TENSOR_MAP_SWIZZLE_64B));
+    else
+        tAct = tOut;
     GemmFp4Args g{};
     g.sfa = a_sf;
     g.sfb = b.sf_mma;
@@ -249,10 +256,12 @@ ft_status run_gemm(const uint8_t* a_codes, const uint8_t* a_sf, const float* ga,
     g.K = static_cast<int>(K);
     g.KL = KL;
     g.status = status;
+    g.act_out = bfm(act_out);
+    g.act_amax = reinterpret_cast<unsigned*>(act_amax);
     if (pair)
-        FT_CUDA(ft::launch_gemm_fp4_lowrank_pair(tA, tB, tLA, tLB, tOut, g, dev.num_sms, st));
+        FT_CUDA(ft::launch_gemm_fp4_lowrank_pair(tA, tB, tLA, tLB, tOut, tAct, g, dev.num_sms, st));
     else
-        FT_CUDA(ft::launch_gemm_fp4_lowrank(tA, tB, tLA, tLB, tOut, g, dev.num_sms, st));
+        FT_CUDA(ft::launch_gemm_fp4_lowrank(tA, tB, tLA, tLB, tOut, tAct, g, dev.num_sms, st));
     return FT_OK;
 }
 
@@ -423,8 +432,13 @@ size_t fourtune_linear_workspace_bytes(const ft_linear* L, int64_t M) {
     return linear_ws(M, L->N, L->K, L->r_s + L->r, L->r).total;
 }
 
-ft_status fourtune_linear_fwd(const ft_linear* L, const void* x_dev, int64_t M, const float* amax_or_null,
-                              void* y_dev, float* t_saved_dev, void* ws, size_t ws_bytes, void* stream) {
+namespace {
+
+// The forward of fourtune_linear_fwd; with h_dev also the GELU epilogue (h = bf16(gelu(y)),
+// max |h| into *h_amax_dev).
+ft_status linear_fwd_impl(const ft_linear* L, const void* x_dev, int64_t M, const float* amax_or_null,
+                          void* y_dev, float* t_saved_dev, void* h_dev, float* h_amax_dev, void* ws,
+                          size_t ws_bytes, void* stream) {
     FT_TRY(check_layer(L));
     const int R = L->r_s + L->r;
     if (!x_dev || !y_dev || (R > 0 && !t_saved_dev) || M <= 0) return FT_ERR_INVALID_ARG;
@@ -450,10 +464,13 @@ ft_status fourtune_linear_fwd(const ft_linear* L, const void* x_dev, int64_t M, 
     // The factor kernel also clears the tensor-max slot (no memset node between kernels).
     ft::PrologueExtras ex;
     if (!amax_or_null) ex.zero_slot = scal + SC_AMAX_X;
+    if (h_dev) ex.zero_slot2 = h_amax_dev;
     if (R > 0)
         FT_CUDA(ft::launch_build_factors(bf(L->ls_down), bf(L->lora_a), bf(L->ls_up), bf(L->lora_b), N, K,
                                          L->r_s, L->r, Rp, KL, bfm(W + w.dn), bfm(W + w.upcat), nullptr,
                                          nullptr, &ex, st));
+    else if (h_dev)
+        FT_CUDA(cudaMemsetAsync(h_amax_dev, 0, sizeof(float), st));
     int splits = 1;
     FT_TRY(quantize_operand(x_dev, M, K, K, amax_or_null, scal + SC_AMAX_X, R > 0, W + w.qx_codes, W + w.qx_scales,
                             W + w.qx_sf, scal + SC_G_X, W + w.dn, Rp, partial, &splits, status, dev, st));
@@ -474,7 +491,23 @@ ft_status fourtune_linear_fwd(const ft_linear* L, const void* x_dev, int64_t M, 
         FT_CUDA(ft::launch_lowrank_finalize(f, st));
     }
     return run_gemm(W + w.qx_codes, W + w.qx_sf, scal + SC_G_X, L->qr, bf(W + w.tcat), bf(W + w.upcat), KL, M,
-                    N, K, y_dev, status, dev, st);
+                    N, K, y_dev, status, dev, st, h_dev, h_amax_dev);
+}
+
+}  // namespace
+
+ft_status fourtune_linear_fwd(const ft_linear* L, const void* x_dev, int64_t M, const float* amax_or_null,
+                              void* y_dev, float* t_saved_dev, void* ws, size_t ws_bytes, void* stream) {
+    return linear_fwd_impl(L, x_dev, M, amax_or_null, y_dev, t_saved_dev, nullptr, nullptr, ws, ws_bytes, stream);
+}
+
+ft_status fourtune_linear_fwd_gelu(const ft_linear* L, const void* x_dev, int64_t M, const float* amax_or_null,
+                                   void* p_dev, void* h_dev, float* h_amax_dev, float* t_saved_dev, void* ws,
+                                   size_t ws_bytes, void* stream) {
+    if (!h_dev || !h_amax_dev) return FT_ERR_INVALID_ARG;
+    if (!aligned16(h_dev) || (reinterpret_cast<uintptr_t>(h_amax_dev) & 3u)) return FT_ERR_ALIGN;
+    return linear_fwd_impl(L, x_dev, M, amax_or_null, p_dev, t_saved_dev, h_dev, h_amax_dev, ws, ws_bytes,
+                           stream);
 }
 
 ft_status fourtune_linear_bwd(const ft_linear* L, const void* x_dev, const float* t_saved_dev,

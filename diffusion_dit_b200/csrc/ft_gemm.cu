@@ -76,7 +76,8 @@ __global__ void __launch_bounds__(THREADS, 1)
                             const __grid_constant__ CUtensorMap tmB,
                             const __grid_constant__ CUtensorMap tmLA,
                             const __grid_constant__ CUtensorMap tmLB,
-                            const __grid_constant__ CUtensorMap tmOut, const GemmFp4Args p) {
+                            const __grid_constant__ CUtensorMap tmOut,
+                            const __grid_constant__ CUtensorMap tmAct, const GemmFp4Args p) {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_u32 = smem_u32(smem_raw);
     const uint32_t pad = (1024 - (raw_u32 & 1023)) & 1023;
@@ -274,6 +275,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         const int q = warp & 3;  // TMEM lane quarter this warp may access
         const float ga = *p.ga, gb = *p.gb;
         const float c = 1.0f / (ga * gb);
+        float hmax = 0.0f;  // max |gelu output| of this thread's elements (GELU epilogue)
         int ti = 0;
         for (int t = blockIdx.x; t < num_tiles && !*abort_flag; t += gridDim.x, ++ti) {
             const int mb = t % MB, nb = t / MB;
@@ -317,7 +319,32 @@ __global__ void __launch_bounds__(THREADS, 1)
                     tma_store_2d(&tmOut, stage_u32, nb * BN + ch * 32, mb * BM + 32 * q);
                     bulk_commit_group();
                 }
+                if (p.act_out) {
+                    // the same chunk through GELU, once the store above has read the buffer
+                    if (lane == 0) bulk_wait_group_read0();
+                    __syncwarp();
+#pragma unroll
+                    for (int c4 = 0; c4 < 4; ++c4) {
+                        const int phys = c4 ^ ((lane >> 1) & 3);
+                        *reinterpret_cast<uint4*>(stage_ptr + lane * 64 + phys * 16) =
+                            make_uint4(gelu_bf16x2(pk[ch * 16 + 4 * c4], hmax),
+                                       gelu_bf16x2(pk[ch * 16 + 4 * c4 + 1], hmax),
+                                       gelu_bf16x2(pk[ch * 16 + 4 * c4 + 2], hmax),
+                                       gelu_bf16x2(pk[ch * 16 + 4 * c4 + 3], hmax));
+                    }
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) {
+                        tma_store_2d(&tmAct, stage_u32, nb * BN + ch * 32, mb * BM + 32 * q);
+                        bulk_commit_group();
+                    }
+                }
             }
+        }
+        if (p.act_amax) {
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) hmax = fmaxf(hmax, __shfl_xor_sync(0xffffffffu, hmax, o));
+            if (lane == 0) atomicMax(p.act_amax, __float_as_uint(hmax));
         }
         if (lane == 0) bulk_wait_group0();
         __syncwarp();
@@ -333,8 +360,8 @@ __global__ void __launch_bounds__(THREADS, 1)
 
 cudaError_t launch_gemm_fp4_lowrank(const CUtensorMap& tmA, const CUtensorMap& tmB,
                                     const CUtensorMap& tmLA, const CUtensorMap& tmLB,
-                                    const CUtensorMap& tmOut, const GemmFp4Args& args, int num_sms,
-                                    cudaStream_t stream) {
+                                    const CUtensorMap& tmOut, const CUtensorMap& tmAct,
+                                    const GemmFp4Args& args, int num_sms, cudaStream_t stream) {
     using namespace gemm;
     static bool attr_set = false;
     if (!attr_set) {
@@ -347,7 +374,7 @@ cudaError_t launch_gemm_fp4_lowrank(const CUtensorMap& tmA, const CUtensorMap& t
     const int grid = tiles < num_sms ? tiles : num_sms;
     before_launch(K_GEMM, stream);
     const cudaError_t le = launch_k(gemm_fp4_lowrank_kernel, dim3(grid), dim3(THREADS), SMEM_BYTES,
-                                    stream, tmA, tmB, tmLA, tmLB, tmOut, args);
+                                    stream, tmA, tmB, tmLA, tmLB, tmOut, tmAct, args);
     if (le != cudaSuccess) return le;
     after_launch(K_GEMM, stream);
     return cudaGetLastError();

@@ -70,7 +70,8 @@ __global__ void __launch_bounds__(THREADS, 1)
                                  const __grid_constant__ CUtensorMap tmB,
                                  const __grid_constant__ CUtensorMap tmLA,
                                  const __grid_constant__ CUtensorMap tmLB,
-                                 const __grid_constant__ CUtensorMap tmOut, const GemmFp4Args p) {
+                                 const __grid_constant__ CUtensorMap tmOut,
+                                 const __grid_constant__ CUtensorMap tmAct, const GemmFp4Args p) {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_u32 = smem_u32(smem_raw);
     const uint32_t pad = (1024 - (raw_u32 & 1023)) & 1023;
@@ -258,6 +259,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         const float ga = *p.ga, gb = *p.gb;
         const float c = 1.0f / (ga * gb);
         const uint32_t empty_even = mapa_shared(bar(BAR_TMEM_EMPTY), 0);
+        float hmax = 0.0f;  // max |gelu output| of this thread's elements (GELU epilogue)
         int ti = 0;
         for (int t = pair; t < num_tiles && !*abort_flag; t += num_pairs, ++ti) {
             const int mb2 = t % MB2, nb = t / MB2;
@@ -298,7 +300,32 @@ __global__ void __launch_bounds__(THREADS, 1)
                     tma_store_2d(&tmOut, stage_u32, nb * BN + ch * 32, row0);
                     bulk_commit_group();
                 }
+                if (p.act_out) {
+                    // the same chunk through GELU, once the store above has read the buffer
+                    if (lane == 0) bulk_wait_group_read0();
+                    __syncwarp();
+#pragma unroll
+                    for (int c4 = 0; c4 < 4; ++c4) {
+                        const int phys = c4 ^ ((lane >> 1) & 3);
+                        *reinterpret_cast<uint4*>(stage_ptr + lane * 64 + phys * 16) =
+                            make_uint4(gelu_bf16x2(pk[ch * 16 + 4 * c4], hmax),
+                                       gelu_bf16x2(pk[ch * 16 + 4 * c4 + 1], hmax),
+                                       gelu_bf16x2(pk[ch * 16 + 4 * c4 + 2], hmax),
+                                       gelu_bf16x2(pk[ch * 16 + 4 * c4 + 3], hmax));
+                    }
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) {
+                        tma_store_2d(&tmAct, stage_u32, nb * BN + ch * 32, row0);
+                        bulk_commit_group();
+                    }
+                }
             }
+        }
+        if (p.act_amax) {
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) hmax = fmaxf(hmax, __shfl_xor_sync(0xffffffffu, hmax, o));
+            if (lane == 0) atomicMax(p.act_amax, __float_as_uint(hmax));
         }
         if (lane == 0) bulk_wait_group0();
         __syncwarp();
@@ -317,8 +344,8 @@ __global__ void __launch_bounds__(THREADS, 1)
 
 cudaError_t launch_gemm_fp4_lowrank_pair(const CUtensorMap& tmA, const CUtensorMap& tmB,
                                          const CUtensorMap& tmLA, const CUtensorMap& tmLB,
-                                         const CUtensorMap& tmOut, const GemmFp4Args& args, int num_sms,
-                                         cudaStream_t stream) {
+                                         const CUtensorMap& tmOut, const CUtensorMap& tmAct,
+                                         const GemmFp4Args& args, int num_sms, cudaStream_t stream) {
     using namespace gemm2;
     static const cudaError_t attr = cudaFuncSetAttribute(
         gemm_fp4_lowrank_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
@@ -342,7 +369,7 @@ cudaError_t launch_gemm_fp4_lowrank_pair(const CUtensorMap& tmA, const CUtensorM
     cfg.numAttrs = 2;
     before_launch(K_GEMM, stream);
     cudaError_t e =
-        cudaLaunchKernelEx(&cfg, gemm_fp4_lowrank_pair_kernel, tmA, tmB, tmLA, tmLB, tmOut, args);
+        cudaLaunchKernelEx(&cfg, gemm_fp4_lowrank_pair_kernel, tmA, tmB, tmLA, tmLB, tmOut, tmAct, args);
     after_launch(K_GEMM, stream);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();

@@ -46,20 +46,24 @@ struct GemmFp4Args {
     int M, N, K;            // K: reduction length in elements (multiple of 256)
     int KL;                 // low-rank reduction length in bf16 elements (multiple of 64), 0 = none
     int* status;            // device status word
+    // optional GELU epilogue: also store act = bf16(gelu_tanh(out)) (same layout as out,
+    // through tmAct) and take max |act| into *act_amax (float bits, cleared beforehand)
+    __nv_bfloat16* act_out;
+    unsigned* act_amax;
 };
 
-// tmOut: bf16 [M, N] output, box 32 x 32, 64-byte swizzle.
+// tmOut (and tmAct): bf16 [M, N] output, box 32 x 32, 64-byte swizzle.
 cudaError_t launch_gemm_fp4_lowrank(const CUtensorMap& tmA, const CUtensorMap& tmB,
                                     const CUtensorMap& tmLA, const CUtensorMap& tmLB,
-                                    const CUtensorMap& tmOut, const GemmFp4Args& args, int num_sms,
-                                    cudaStream_t stream);
+                                    const CUtensorMap& tmOut, const CUtensorMap& tmAct,
+                                    const GemmFp4Args& args, int num_sms, cudaStream_t stream);
 
 // The same GEMM computed by CTA pairs (cta_group::2), 256 x 256 tiles; needs M % 256 == 0.
 // tmB / tmLB boxes are 128 rows: each CTA of a pair loads half of the tile's N.
 cudaError_t launch_gemm_fp4_lowrank_pair(const CUtensorMap& tmA, const CUtensorMap& tmB,
                                          const CUtensorMap& tmLA, const CUtensorMap& tmLB,
-                                         const CUtensorMap& tmOut, const GemmFp4Args& args, int num_sms,
-                                         cudaStream_t stream);
+                                         const CUtensorMap& tmOut, const CUtensorMap& tmAct,
+                                         const GemmFp4Args& args, int num_sms, cudaStream_t stream);
 
 // quantizer and helpers (ft_quant.cu)
 // amax_out accumulates with atomicMax: it is cleared here unless slot_cleared (an earlier
@@ -128,6 +132,7 @@ struct PrologueExtras {
     int hilo_ld = 0, hilo_c0 = 0, hilo_r = 0, hilo_M = 0, hilo_NBW = 0;
     __nv_bfloat16* hilo_dst = nullptr;
     float* zero_slot = nullptr;
+    float* zero_slot2 = nullptr;  // a second cleared max slot (the GELU epilogue's)
 };
 
 // Build the concatenated low-rank factors used by the forward and backward GEMMs (and

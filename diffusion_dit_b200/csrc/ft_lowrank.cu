@@ -131,6 +131,7 @@ __global__ void build_factors_kernel(const __nv_bfloat16* __restrict__ ls_down,
         }
     }
     if (x.zero_slot && t0 == 0) *x.zero_slot = 0.0f;
+    if (x.zero_slot2 && t0 == 0) *x.zero_slot2 = 0.0f;
 }
 
 }  // namespace

@@ -417,6 +417,33 @@ __device__ __forceinline__ float ue4m3_to_f32(uint32_t code) {
     return __half2float(__ushort_as_half(static_cast<unsigned short>(h2 & 0xFFFF)));
 }
 
+// GELU, tanh form: 0.5 p (1 + tanh(u)), u = sqrt(2/pi) (p + 0.044715 p^3), evaluated as
+// p * sigmoid(2u), the same function (0.5 (1 + tanh u) = 1 / (1 + exp(-2u))), which keeps
+// full relative accuracy for large negative p where 1 + tanh(u) cancels.  Every step is
+// an explicitly rounded fp32 operation (no contraction), so the stand-alone kernel and
+// the GEMM epilogue produce the same bits; exp is the library expf.
+__device__ __forceinline__ float gelu_tanh_u(float p) {
+    const float k = 0.7978845608028654f;  // sqrt(2 / pi)
+    const float p3 = __fmul_rn(__fmul_rn(p, p), p);
+    return __fmul_rn(k, __fadd_rn(p, __fmul_rn(0.044715f, p3)));
+}
+
+__device__ __forceinline__ float gelu_tanh_f(float p) {
+    return __fdiv_rn(p, __fadd_rn(1.0f, expf(__fmul_rn(-2.0f, gelu_tanh_u(p)))));
+}
+
+// dP = dH * gelu'(P); with s = sigmoid(2u): gelu' = s + 2 p s (1 - s) u', and
+// 1 - s = sigmoid(-2u) taken directly (no inf / inf for large |u|).
+__device__ __forceinline__ float gelu_tanh_bwd_f(float p, float dh) {
+    const float k = 0.7978845608028654f;
+    const float u = gelu_tanh_u(p);
+    const float sg = __fdiv_rn(1.0f, __fadd_rn(1.0f, expf(__fmul_rn(-2.0f, u))));
+    const float one_minus = __fdiv_rn(1.0f, __fadd_rn(1.0f, expf(__fmul_rn(2.0f, u))));
+    const float du = __fmul_rn(k, __fadd_rn(1.0f, __fmul_rn(3.0f * 0.044715f, __fmul_rn(p, p))));
+    const float g = __fadd_rn(sg, __fmul_rn(__fmul_rn(__fmul_rn(__fmul_rn(2.0f, p), sg), one_minus), du));
+    return __fmul_rn(dh, g);
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     uint32_t out;
     asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(out) : "f"(hi), "f"(lo));
@@ -425,5 +452,13 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 
 __device__ __forceinline__ float bf16lo_to_f32(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16hi_to_f32(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+// Two packed bf16 -> bf16(gelu_tanh(.)) each, packed the same way; hmax takes the larger
+// of itself and the two results' magnitudes (fmaxf: a NaN never wins).
+__device__ __forceinline__ uint32_t gelu_bf16x2(uint32_t w, float& hmax) {
+    const uint32_t r = pack_bf16x2(gelu_tanh_f(bf16lo_to_f32(w)), gelu_tanh_f(bf16hi_to_f32(w)));
+    hmax = fmaxf(hmax, fmaxf(fabsf(bf16lo_to_f32(r)), fabsf(bf16hi_to_f32(r))));
+    return r;
+}
 
 }  // namespace ft

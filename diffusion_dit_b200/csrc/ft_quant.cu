@@ -208,26 +208,6 @@ __global__ void encode_ue4m3_kernel(const float* __restrict__ v, int64_t n, uint
         out[i] = static_cast<uint8_t>(cvt_ue4m3(v[i]));
 }
 
-// GELU, tanh form: 0.5 p (1 + tanh(u)), u = sqrt(2/pi) (p + 0.044715 p^3).  Evaluated
-// as p * sigmoid(2u), the same function (0.5 (1 + tanh u) = 1 / (1 + exp(-2u))), which
-// keeps full relative accuracy for large negative p where 1 + tanh(u) cancels; fp32
-// with the library expf, result rounded to bf16 (nearest even).
-__device__ __forceinline__ float gelu_tanh_f(float p) {
-    const float k = 0.7978845608028654f;  // sqrt(2 / pi)
-    const float u = k * (p + 0.044715f * p * p * p);
-    return p / (1.0f + expf(-2.0f * u));
-}
-
-// d/dp: with s = sigmoid(2u), gelu' = s + 2 p s (1 - s) u'.
-__device__ __forceinline__ float gelu_tanh_grad_f(float p) {
-    const float k = 0.7978845608028654f;
-    const float u = k * (p + 0.044715f * p * p * p);
-    const float sg = 1.0f / (1.0f + expf(-2.0f * u));
-    const float one_minus = 1.0f / (1.0f + expf(2.0f * u));  // sigmoid(-2u), no inf / inf
-    const float du = k * (1.0f + 3.0f * 0.044715f * p * p);
-    return sg + 2.0f * p * sg * one_minus * du;
-}
-
 __global__ void gelu_fwd_kernel(const __nv_bfloat16* __restrict__ p, __nv_bfloat16* __restrict__ h,
                                 int64_t n) {
     pdl_trigger();
@@ -255,10 +235,10 @@ __global__ void gelu_bwd_kernel(const __nv_bfloat16* __restrict__ p, const __nv_
         load8(p + i, v);
         load8(dh + i, d);
         uint4 o;
-        o.x = pack_bf16x2(d[0] * gelu_tanh_grad_f(v[0]), d[1] * gelu_tanh_grad_f(v[1]));
-        o.y = pack_bf16x2(d[2] * gelu_tanh_grad_f(v[2]), d[3] * gelu_tanh_grad_f(v[3]));
-        o.z = pack_bf16x2(d[4] * gelu_tanh_grad_f(v[4]), d[5] * gelu_tanh_grad_f(v[5]));
-        o.w = pack_bf16x2(d[6] * gelu_tanh_grad_f(v[6]), d[7] * gelu_tanh_grad_f(v[7]));
+        o.x = pack_bf16x2(gelu_tanh_bwd_f(v[0], d[0]), gelu_tanh_bwd_f(v[1], d[1]));
+        o.y = pack_bf16x2(gelu_tanh_bwd_f(v[2], d[2]), gelu_tanh_bwd_f(v[3], d[3]));
+        o.z = pack_bf16x2(gelu_tanh_bwd_f(v[4], d[4]), gelu_tanh_bwd_f(v[5], d[5]));
+        o.w = pack_bf16x2(gelu_tanh_bwd_f(v[6], d[6]), gelu_tanh_bwd_f(v[7], d[7]));
         *reinterpret_cast<uint4*>(dp + i) = o;
     }
 }

@@ -56,6 +56,9 @@ EXPORTS = {
     "fourtune_linear_fwd": ([ctypes.POINTER(FtLinear), ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p,
                              ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t,
                              ctypes.c_void_p], ctypes.c_int),
+    "fourtune_linear_fwd_gelu": ([ctypes.POINTER(FtLinear), ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p,
+                                  ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                  ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p], ctypes.c_int),
     "fourtune_linear_bwd": ([ctypes.POINTER(FtLinear), ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
                              ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
                              ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p],
@@ -242,6 +245,29 @@ def linear_fwd(w: LinearWeights, x: torch.Tensor, ws: Workspace, y: Optional[tor
                                    ws.nbytes, _stream(stream))
     _check("fourtune_linear_fwd", st)
     return y, t_saved
+
+
+def linear_fwd_gelu(w: LinearWeights, x: torch.Tensor, ws: Workspace, p: Optional[torch.Tensor] = None,
+                    h: Optional[torch.Tensor] = None, h_amax: Optional[torch.Tensor] = None,
+                    t_saved: Optional[torch.Tensor] = None, amax: Optional[torch.Tensor] = None, stream=None):
+    """Eq. (2) with GELU fused into the GEMM epilogue (an MLP's first linear).
+    Returns (P bf16 [M, N], H = bf16(gelu_tanh(P)) [M, N], max|H| fp32 [1], T fp32 [M, r_s + r])."""
+    _require_cuda(x)
+    M = x.shape[0]
+    if p is None:
+        p = torch.empty(M, w.N, dtype=torch.bfloat16, device=x.device)
+    if h is None:
+        h = torch.empty(M, w.N, dtype=torch.bfloat16, device=x.device)
+    if h_amax is None:
+        h_amax = torch.empty(1, dtype=torch.float32, device=x.device)
+    R = w.r_s + w.r
+    if t_saved is None:
+        t_saved = torch.empty(M, max(R, 1), dtype=torch.float32, device=x.device)
+    s = w.c_struct()
+    st = lib().fourtune_linear_fwd_gelu(ctypes.byref(s), _p(x), M, _p(amax), _p(p), _p(h), _p(h_amax),
+                                        _p(t_saved), _p(ws.buf), ws.nbytes, _stream(stream))
+    _check("fourtune_linear_fwd_gelu", st)
+    return p, h, h_amax, t_saved
 
 
 def linear_bwd(w: LinearWeights, x: torch.Tensor, t_saved: torch.Tensor, dy: torch.Tensor, ws: Workspace,

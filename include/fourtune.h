@@ -191,6 +191,24 @@ ft_status fourtune_linear_fwd(const ft_linear* layer, const void* x_dev, int64_t
                               void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * Forward pass with GELU (tanh form) fused into the 4-bit GEMM's epilogue, for the first
+ * linear of an MLP (section 3.3 "MLP Fusion": the FC1 GEMM is fused with what FC2's
+ * quantization needs, so the activation is not read back and re-written by a separate
+ * pass).
+ *   p_dev      : bf16 [M, N], written: the layer output P (exactly fourtune_linear_fwd's y).
+ *   h_dev      : bf16 [M, N], written: H = bf16(gelu_tanh(P)) evaluated in fp32 from the bf16
+ *                P (the same bits as fourtune_gelu_tanh_fwd on p_dev).
+ *   h_amax_dev : device float[1], written: max |H|.  Pass it as amax_or_null to the next
+ *                layer's fourtune_linear_fwd, which then needs no pass of its own over H.
+ *   The other arguments, shapes and the workspace are those of fourtune_linear_fwd.  P is
+ *   what the backward's gelu' needs; H is the next layer's input (its forward and its dA).
+ */
+ft_status fourtune_linear_fwd_gelu(const ft_linear* layer, const void* x_dev, int64_t M,
+                                   const float* amax_or_null, void* p_dev, void* h_dev,
+                                   float* h_amax_dev, float* t_saved_dev, void* ws, size_t ws_bytes,
+                                   void* stream);
+
+/*
  * Backward pass, Eq. (3) and the adapter gradients of section 3.2.
  *   x_dev       : bf16 [M, K], the forward input.
  *   t_saved_dev : fp32 [M, r_s + r] from fourtune_linear_fwd.
