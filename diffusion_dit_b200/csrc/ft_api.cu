@@ -223,7 +223,7 @@ ft_status quantize_operand(const void* x, int64_t rows, int64_t cols, int64_t ld
 ft_status run_gemm(const uint8_t* a_codes, const uint8_t* a_sf, const float* ga, const ft_fp4& b,
                    const __nv_bfloat16* la, const __nv_bfloat16* lb, int KL, int64_t M, int64_t N,
                    int64_t K, void* out, int* status, const DeviceInfo& dev, cudaStream_t st,
-                   void* act_out = nullptr, float* act_amax = nullptr) {
+                   void* act_out = nullptr, float* act_amax = nullptr, const void* gelu_in = nullptr) {
     // CTA pairs (256 x 256 tiles) when M allows, single CTAs (128 x 256) otherwise.
     const bool pair = (M % 256) == 0 && dev.num_sms >= 2;
     const uint32_t b_rows = pair ? 128 : 256;
@@ -258,6 +258,7 @@ ft_status run_gemm(const uint8_t* a_codes, const uint8_t* a_sf, const float* ga,
     g.status = status;
     g.act_out = bfm(act_out);
     g.act_amax = reinterpret_cast<unsigned*>(act_amax);
+    g.gelu_in = bf(gelu_in);
     if (pair)
         FT_CUDA(ft::launch_gemm_fp4_lowrank_pair(tA, tB, tLA, tLB, tOut, tAct, g, dev.num_sms, st));
     else
@@ -510,9 +511,12 @@ ft_status fourtune_linear_fwd_gelu(const ft_linear* L, const void* x_dev, int64_
                            stream);
 }
 
-ft_status fourtune_linear_bwd(const ft_linear* L, const void* x_dev, const float* t_saved_dev,
-                              const void* dy_dev, int64_t M, const float* amax_or_null, void* dx_dev,
-                              float* da_dev, float* db_dev, void* ws, size_t ws_bytes, void* stream) {
+namespace {
+
+// The backward of fourtune_linear_bwd; with gelu_in, dx_dev receives bf16(dX * gelu'(gelu_in)).
+ft_status linear_bwd_impl(const ft_linear* L, const void* x_dev, const float* t_saved_dev, const void* dy_dev,
+                          int64_t M, const float* amax_or_null, void* dx_dev, float* da_dev, float* db_dev,
+                          const void* gelu_in, void* ws, size_t ws_bytes, void* stream) {
     FT_TRY(check_layer(L));
     const int R = L->r_s + L->r;
     if (!x_dev || !dy_dev || !dx_dev || M <= 0) return FT_ERR_INVALID_ARG;
@@ -618,8 +622,27 @@ ft_status fourtune_linear_bwd(const ft_linear* L, const void* x_dev, const float
     }
     // The dX GEMM goes last: the GEMM's operand and output traffic would evict G from L2.
     FT_TRY(run_gemm(W + w.qg_codes, W + w.qg_sf, scal + SC_G_G, L->qr_t, bf(W + w.ucat), bf(W + w.dntcat), KL,
-                    M, K, N, dx_dev, status, dev, st));
+                    M, K, N, dx_dev, status, dev, st, nullptr, nullptr, gelu_in));
     return FT_OK;
+}
+
+}  // namespace
+
+ft_status fourtune_linear_bwd(const ft_linear* L, const void* x_dev, const float* t_saved_dev,
+                              const void* dy_dev, int64_t M, const float* amax_or_null, void* dx_dev,
+                              float* da_dev, float* db_dev, void* ws, size_t ws_bytes, void* stream) {
+    return linear_bwd_impl(L, x_dev, t_saved_dev, dy_dev, M, amax_or_null, dx_dev, da_dev, db_dev, nullptr, ws,
+                           ws_bytes, stream);
+}
+
+ft_status fourtune_linear_bwd_gelu(const ft_linear* L, const void* x_dev, const float* t_saved_dev,
+                                   const void* dy_dev, int64_t M, const float* amax_or_null, const void* p_dev,
+                                   void* dp_dev, float* da_dev, float* db_dev, void* ws, size_t ws_bytes,
+                                   void* stream) {
+    if (!p_dev) return FT_ERR_INVALID_ARG;
+    if (!aligned16(p_dev)) return FT_ERR_ALIGN;
+    return linear_bwd_impl(L, x_dev, t_saved_dev, dy_dev, M, amax_or_null, dp_dev, da_dev, db_dev, p_dev, ws,
+                           ws_bytes, stream);
 }
 
 ft_status fourtune_selftest_bounded_wait(int64_t limit_ns, void* ws, void* stream) {

@@ -71,6 +71,7 @@ constexpr int NUM_BARS = 3 * STAGES + 3;
 constexpr int OFF_TMEM_SLOT = 8 * 16;   // inside the barrier area
 constexpr int OFF_ABORT = 8 * 16 + 4;
 
+template <int EPI>
 __global__ void __launch_bounds__(THREADS, 1)
     gemm_fp4_lowrank_kernel(const __grid_constant__ CUtensorMap tmA,
                             const __grid_constant__ CUtensorMap tmB,
@@ -302,10 +303,35 @@ __global__ void __launch_bounds__(THREADS, 1)
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(sm.bar(BAR_TMEM_EMPTY));
+            // GELU-backward epilogue: this thread's row of gelu_in, one 32-column chunk ahead
+            const __nv_bfloat16* prow =
+                EPI == kEpiGeluBwd ? p.gelu_in + static_cast<size_t>(mb * BM + 32 * q + lane) * p.ldo + nb * BN : nullptr;
+            uint4 pin[4];
+            if constexpr (EPI == kEpiGeluBwd) {
+#pragma unroll
+                for (int c4 = 0; c4 < 4; ++c4) pin[c4] = *reinterpret_cast<const uint4*>(prow + 8 * c4);
+            }
 #pragma unroll
             for (int ch = 0; ch < BN / 32; ++ch) {
                 if (lane == 0) bulk_wait_group_read0();  // previous store has read the buffer
                 __syncwarp();
+                if constexpr (EPI == kEpiGeluBwd) {
+                    uint4 cur[4];
+#pragma unroll
+                    for (int c4 = 0; c4 < 4; ++c4) cur[c4] = pin[c4];
+                    if (ch + 1 < BN / 32) {
+#pragma unroll
+                        for (int c4 = 0; c4 < 4; ++c4)
+                            pin[c4] = *reinterpret_cast<const uint4*>(prow + 32 * (ch + 1) + 8 * c4);
+                    }
+#pragma unroll
+                    for (int c4 = 0; c4 < 4; ++c4) {
+                        pk[ch * 16 + 4 * c4] = gelu_bwd_bf16x2(pk[ch * 16 + 4 * c4], cur[c4].x);
+                        pk[ch * 16 + 4 * c4 + 1] = gelu_bwd_bf16x2(pk[ch * 16 + 4 * c4 + 1], cur[c4].y);
+                        pk[ch * 16 + 4 * c4 + 2] = gelu_bwd_bf16x2(pk[ch * 16 + 4 * c4 + 2], cur[c4].z);
+                        pk[ch * 16 + 4 * c4 + 3] = gelu_bwd_bf16x2(pk[ch * 16 + 4 * c4 + 3], cur[c4].w);
+                    }
+                }
 #pragma unroll
                 for (int c4 = 0; c4 < 4; ++c4) {
                     const int phys = c4 ^ ((lane >> 1) & 3);
@@ -319,7 +345,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                     tma_store_2d(&tmOut, stage_u32, nb * BN + ch * 32, mb * BM + 32 * q);
                     bulk_commit_group();
                 }
-                if (p.act_out) {
+                if constexpr (EPI == kEpiGelu) {
                     // the same chunk through GELU, once the store above has read the buffer
                     if (lane == 0) bulk_wait_group_read0();
                     __syncwarp();
@@ -341,7 +367,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                 }
             }
         }
-        if (p.act_amax) {
+        if (EPI == kEpiGelu && p.act_amax) {
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) hmax = fmaxf(hmax, __shfl_xor_sync(0xffffffffu, hmax, o));
             if (lane == 0) atomicMax(p.act_amax, __float_as_uint(hmax));
@@ -358,23 +384,35 @@ __global__ void __launch_bounds__(THREADS, 1)
 
 }  // namespace gemm
 
+namespace {
+
+// One epilogue variant: its own instantiation, its shared-memory opt-in set once.
+template <int EPI>
+cudaError_t launch_variant(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmLA,
+                           const CUtensorMap& tmLB, const CUtensorMap& tmOut, const CUtensorMap& tmAct,
+                           const GemmFp4Args& args, int grid, cudaStream_t stream) {
+    using namespace gemm;
+    static const cudaError_t attr = cudaFuncSetAttribute(
+        gemm_fp4_lowrank_kernel<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+    if (attr != cudaSuccess) return attr;
+    return launch_k(gemm_fp4_lowrank_kernel<EPI>, dim3(grid), dim3(THREADS), SMEM_BYTES, stream, tmA, tmB, tmLA,
+                    tmLB, tmOut, tmAct, args);
+}
+
+}  // namespace
+
 cudaError_t launch_gemm_fp4_lowrank(const CUtensorMap& tmA, const CUtensorMap& tmB,
                                     const CUtensorMap& tmLA, const CUtensorMap& tmLB,
                                     const CUtensorMap& tmOut, const CUtensorMap& tmAct,
                                     const GemmFp4Args& args, int num_sms, cudaStream_t stream) {
     using namespace gemm;
-    static bool attr_set = false;
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(gemm_fp4_lowrank_kernel,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
-        if (e != cudaSuccess) return e;
-        attr_set = true;
-    }
     const int tiles = (args.M / BM) * (args.N / BN);
     const int grid = tiles < num_sms ? tiles : num_sms;
     before_launch(K_GEMM, stream);
-    const cudaError_t le = launch_k(gemm_fp4_lowrank_kernel, dim3(grid), dim3(THREADS), SMEM_BYTES,
-                                    stream, tmA, tmB, tmLA, tmLB, tmOut, tmAct, args);
+    const cudaError_t le =
+        args.gelu_in  ? launch_variant<kEpiGeluBwd>(tmA, tmB, tmLA, tmLB, tmOut, tmAct, args, grid, stream)
+        : args.act_out ? launch_variant<kEpiGelu>(tmA, tmB, tmLA, tmLB, tmOut, tmAct, args, grid, stream)
+                       : launch_variant<kEpiPlain>(tmA, tmB, tmLA, tmLB, tmOut, tmAct, args, grid, stream);
     if (le != cudaSuccess) return le;
     after_launch(K_GEMM, stream);
     return cudaGetLastError();

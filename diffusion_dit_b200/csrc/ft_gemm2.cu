@@ -65,6 +65,7 @@ constexpr int OFF_TMEM_SLOT = 8 * NUM_BARS;
 constexpr int OFF_ABORT = OFF_TMEM_SLOT + 4;
 static_assert(OFF_ABORT + 4 <= BAR_BYTES, "barrier area overflow");
 
+template <int EPI>
 __global__ void __launch_bounds__(THREADS, 1)
     gemm_fp4_lowrank_pair_kernel(const __grid_constant__ CUtensorMap tmA,
                                  const __grid_constant__ CUtensorMap tmB,
@@ -283,10 +284,35 @@ __global__ void __launch_bounds__(THREADS, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(empty_even);
             const int row0 = (mb2 * 2 + static_cast<int>(rank)) * BM + 32 * q;
+            // GELU-backward epilogue: this thread's row of gelu_in, one 32-column chunk ahead
+            const __nv_bfloat16* prow =
+                EPI == kEpiGeluBwd ? p.gelu_in + static_cast<size_t>(row0 + lane) * p.ldo + nb * BN : nullptr;
+            uint4 pin[4];
+            if constexpr (EPI == kEpiGeluBwd) {
+#pragma unroll
+                for (int c4 = 0; c4 < 4; ++c4) pin[c4] = *reinterpret_cast<const uint4*>(prow + 8 * c4);
+            }
 #pragma unroll
             for (int ch = 0; ch < BN / 32; ++ch) {
                 if (lane == 0) bulk_wait_group_read0();
                 __syncwarp();
+                if constexpr (EPI == kEpiGeluBwd) {
+                    uint4 cur[4];
+#pragma unroll
+                    for (int c4 = 0; c4 < 4; ++c4) cur[c4] = pin[c4];
+                    if (ch + 1 < BN / 32) {
+#pragma unroll
+                        for (int c4 = 0; c4 < 4; ++c4)
+                            pin[c4] = *reinterpret_cast<const uint4*>(prow + 32 * (ch + 1) + 8 * c4);
+                    }
+#pragma unroll
+                    for (int c4 = 0; c4 < 4; ++c4) {
+                        pk[ch * 16 + 4 * c4] = gelu_bwd_bf16x2(pk[ch * 16 + 4 * c4], cur[c4].x);
+                        pk[ch * 16 + 4 * c4 + 1] = gelu_bwd_bf16x2(pk[ch * 16 + 4 * c4 + 1], cur[c4].y);
+                        pk[ch * 16 + 4 * c4 + 2] = gelu_bwd_bf16x2(pk[ch * 16 + 4 * c4 + 2], cur[c4].z);
+                        pk[ch * 16 + 4 * c4 + 3] = gelu_bwd_bf16x2(pk[ch * 16 + 4 * c4 + 3], cur[c4].w);
+                    }
+                }
 #pragma unroll
                 for (int c4 = 0; c4 < 4; ++c4) {
                     const int phys = c4 ^ ((lane >> 1) & 3);
@@ -300,7 +326,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                     tma_store_2d(&tmOut, stage_u32, nb * BN + ch * 32, row0);
                     bulk_commit_group();
                 }
-                if (p.act_out) {
+                if constexpr (EPI == kEpiGelu) {
                     // the same chunk through GELU, once the store above has read the buffer
                     if (lane == 0) bulk_wait_group_read0();
                     __syncwarp();
@@ -322,7 +348,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                 }
             }
         }
-        if (p.act_amax) {
+        if (EPI == kEpiGelu && p.act_amax) {
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) hmax = fmaxf(hmax, __shfl_xor_sync(0xffffffffu, hmax, o));
             if (lane == 0) atomicMax(p.act_amax, __float_as_uint(hmax));
@@ -342,14 +368,27 @@ __global__ void __launch_bounds__(THREADS, 1)
 
 }  // namespace gemm2
 
+namespace {
+
+// One epilogue variant: its own instantiation, its shared-memory opt-in set once.
+template <int EPI>
+cudaError_t launch_variant(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmLA,
+                           const CUtensorMap& tmLB, const CUtensorMap& tmOut, const CUtensorMap& tmAct,
+                           const GemmFp4Args& args, cudaLaunchConfig_t cfg) {
+    using namespace gemm2;
+    static const cudaError_t attr = cudaFuncSetAttribute(
+        gemm_fp4_lowrank_pair_kernel<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+    if (attr != cudaSuccess) return attr;
+    return cudaLaunchKernelEx(&cfg, gemm_fp4_lowrank_pair_kernel<EPI>, tmA, tmB, tmLA, tmLB, tmOut, tmAct, args);
+}
+
+}  // namespace
+
 cudaError_t launch_gemm_fp4_lowrank_pair(const CUtensorMap& tmA, const CUtensorMap& tmB,
                                          const CUtensorMap& tmLA, const CUtensorMap& tmLB,
                                          const CUtensorMap& tmOut, const CUtensorMap& tmAct,
                                          const GemmFp4Args& args, int num_sms, cudaStream_t stream) {
     using namespace gemm2;
-    static const cudaError_t attr = cudaFuncSetAttribute(
-        gemm_fp4_lowrank_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
-    if (attr != cudaSuccess) return attr;
     const int tiles = (args.M / (2 * BM)) * (args.N / BN);
     int pairs = num_sms / 2;
     if (pairs > tiles) pairs = tiles;
@@ -368,8 +407,10 @@ cudaError_t launch_gemm_fp4_lowrank_pair(const CUtensorMap& tmA, const CUtensorM
     cfg.attrs = at;
     cfg.numAttrs = 2;
     before_launch(K_GEMM, stream);
-    cudaError_t e =
-        cudaLaunchKernelEx(&cfg, gemm_fp4_lowrank_pair_kernel, tmA, tmB, tmLA, tmLB, tmOut, tmAct, args);
+    const cudaError_t e =
+        args.gelu_in  ? launch_variant<kEpiGeluBwd>(tmA, tmB, tmLA, tmLB, tmOut, tmAct, args, cfg)
+        : args.act_out ? launch_variant<kEpiGelu>(tmA, tmB, tmLA, tmLB, tmOut, tmAct, args, cfg)
+                       : launch_variant<kEpiPlain>(tmA, tmB, tmLA, tmLB, tmOut, tmAct, args, cfg);
     after_launch(K_GEMM, stream);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();

@@ -36,6 +36,9 @@ cudaError_t launch_k(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t sme
     return cudaLaunchKernelEx(&cfg, kernel, static_cast<Args&&>(args)...);
 }
 
+// GEMM epilogue variants, one kernel instantiation each (the plain one carries no GELU code)
+enum EpilogueKind { kEpiPlain = 0, kEpiGelu = 1, kEpiGeluBwd = 2 };
+
 struct GemmFp4Args {
     const uint8_t* sfa;     // tensor-core scale layout of A (rows M, cols K)
     const uint8_t* sfb;     // tensor-core scale layout of B (rows N, cols K)
@@ -50,6 +53,9 @@ struct GemmFp4Args {
     // through tmAct) and take max |act| into *act_amax (float bits, cleared beforehand)
     __nv_bfloat16* act_out;
     unsigned* act_amax;
+    // optional GELU-backward epilogue: store bf16(bf16(out) * gelu_tanh'(gelu_in)) instead
+    // of out, gelu_in bf16 with out's layout (the MLP's pre-activation P)
+    const __nv_bfloat16* gelu_in;
 };
 
 // tmOut (and tmAct): bf16 [M, N] output, box 32 x 32, 64-byte swizzle.

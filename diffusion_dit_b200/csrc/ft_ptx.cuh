@@ -453,6 +453,12 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 __device__ __forceinline__ float bf16lo_to_f32(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16hi_to_f32(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
+// Two packed bf16 gradients dh -> bf16(dh * gelu_tanh'(p)) each (p: two packed bf16).
+__device__ __forceinline__ uint32_t gelu_bwd_bf16x2(uint32_t dh, uint32_t p) {
+    return pack_bf16x2(gelu_tanh_bwd_f(bf16lo_to_f32(p), bf16lo_to_f32(dh)),
+                       gelu_tanh_bwd_f(bf16hi_to_f32(p), bf16hi_to_f32(dh)));
+}
+
 // Two packed bf16 -> bf16(gelu_tanh(.)) each, packed the same way; hmax takes the larger
 // of itself and the two results' magnitudes (fmaxf: a NaN never wins).
 __device__ __forceinline__ uint32_t gelu_bf16x2(uint32_t w, float& hmax) {

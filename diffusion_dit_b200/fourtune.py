@@ -63,6 +63,10 @@ EXPORTS = {
                              ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
                              ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p],
                             ctypes.c_int),
+    "fourtune_linear_bwd_gelu": ([ctypes.POINTER(FtLinear), ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                  ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                  ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t,
+                                  ctypes.c_void_p], ctypes.c_int),
     "fourtune_device_status": ([ctypes.c_void_p, ctypes.POINTER(ctypes.c_int32), ctypes.c_void_p], ctypes.c_int),
     "fourtune_gelu_tanh_fwd": ([ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p], ctypes.c_int),
     "fourtune_gelu_tanh_bwd": ([ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64,
@@ -287,6 +291,26 @@ def linear_bwd(w: LinearWeights, x: torch.Tensor, t_saved: torch.Tensor, dy: tor
                                    _p(db), _p(ws.buf), ws.nbytes, _stream(stream))
     _check("fourtune_linear_bwd", st)
     return dx, da, db
+
+
+def linear_bwd_gelu(w: LinearWeights, x: torch.Tensor, t_saved: torch.Tensor, dy: torch.Tensor, p: torch.Tensor,
+                    ws: Workspace, dp: Optional[torch.Tensor] = None, da: Optional[torch.Tensor] = None,
+                    db: Optional[torch.Tensor] = None, amax: Optional[torch.Tensor] = None, stream=None):
+    """Backward of an MLP's second linear with gelu' fused into the dX GEMM's epilogue.
+    Returns (dP = bf16(dX * gelu'(p)) bf16 [M, K], dA fp32 [r, K], dB fp32 [N, r])."""
+    _require_cuda(x, t_saved, dy, p)
+    M = x.shape[0]
+    if dp is None:
+        dp = torch.empty(M, w.K, dtype=torch.bfloat16, device=x.device)
+    if da is None:
+        da = torch.empty(max(w.r, 1), w.K, dtype=torch.float32, device=x.device)
+    if db is None:
+        db = torch.empty(w.N, max(w.r, 1), dtype=torch.float32, device=x.device)
+    s = w.c_struct()
+    st = lib().fourtune_linear_bwd_gelu(ctypes.byref(s), _p(x), _p(t_saved), _p(dy), M, _p(amax), _p(p), _p(dp),
+                                        _p(da), _p(db), _p(ws.buf), ws.nbytes, _stream(stream))
+    _check("fourtune_linear_bwd_gelu", st)
+    return dp, da, db
 
 
 def gelu_tanh_fwd(p: torch.Tensor, h: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:

@@ -225,6 +225,21 @@ ft_status fourtune_linear_bwd(const ft_linear* layer, const void* x_dev, const f
                               size_t ws_bytes, void* stream);
 
 /*
+ * Backward pass of an MLP's second linear with the GELU derivative fused into the dX
+ * GEMM's epilogue (section 3.3 "MLP Fusion", backward side): instead of dX (= dH, the
+ * gradient at the GELU output) it writes dP = bf16(bf16(dH) * gelu_tanh'(P)), the same bits
+ * as fourtune_linear_bwd followed by fourtune_gelu_tanh_bwd, so dH is never stored.
+ *   p_dev  : bf16 [M, K], the pre-activation P (p_dev of fourtune_linear_fwd_gelu).
+ *   dp_dev : bf16 [M, K], written (in place of dx_dev).
+ *   The other arguments (x_dev is this layer's input H), shapes and the workspace are those
+ *   of fourtune_linear_bwd.
+ */
+ft_status fourtune_linear_bwd_gelu(const ft_linear* layer, const void* x_dev, const float* t_saved_dev,
+                                   const void* dy_dev, int64_t M, const float* amax_or_null,
+                                   const void* p_dev, void* dp_dev, float* da_dev, float* db_dev, void* ws,
+                                   size_t ws_bytes, void* stream);
+
+/*
  * Reads (synchronously, on `stream`) the device status word that the kernels of the
  * last call using workspace `ws` left behind: FT_OK or FT_ERR_TIMEOUT.  *status_out is
  * a HOST pointer.  Clears the word.

@@ -1,9 +1,10 @@
-"""GELU fused into the 4-bit GEMM's epilogue (FourTune section 3.3, "MLP Fusion"):
-fourtune_linear_fwd_gelu must give exactly what the unfused path gives -- the layer output
-P of fourtune_linear_fwd, H = the stand-alone GELU kernel applied to P, and max |H| as the
-max kernel would take it -- on both GEMM kernels (CTA pairs when M % 256 == 0, single CTAs
-otherwise), and a next layer fed that max must produce the same bits as one that takes
-its own."""
+"""GELU fused into the 4-bit GEMM's epilogues (FourTune section 3.3, "MLP Fusion").
+Forward: fourtune_linear_fwd_gelu must give exactly what the unfused path gives -- the
+layer output P of fourtune_linear_fwd, H = the stand-alone GELU kernel applied to P, and
+max |H| as the max kernel would take it -- and a next layer fed that max must produce the
+same bits as one that takes its own.  Backward: fourtune_linear_bwd_gelu must write the
+same bits as fourtune_linear_bwd followed by the stand-alone GELU-backward kernel.  Both
+GEMM kernels are covered (CTA pairs when M % 256 == 0, single CTAs otherwise)."""
 import functools
 
 import numpy as np
@@ -80,3 +81,28 @@ def test_fused_gelu_full_size_mlp_up_then_down():
     assert ws.device_status() == 0
     assert torch.equal(y_fed, y_own)
     assert torch.equal(t_fed, t_own)
+
+
+@pytest.mark.parametrize("spec", [wl.PARITY_SMALL, MID], ids=lambda s: s.name)
+def test_fused_gelu_backward_equals_unfused(spec):
+    ft = _ft()
+    inp, w = _setup(spec)
+    ws = ft.Workspace(w, spec.M, "cuda")
+    x, dy = inp.x.cuda(), inp.dy.cuda()
+    # a pre-activation P of the layer's input shape [M, K]: bf16 values around the GELU's
+    # curved region, with zeros, negatives and a few large magnitudes
+    g = torch.Generator().manual_seed(7)
+    p = (torch.randn(spec.M, spec.K, generator=g) * 2.0).to(torch.bfloat16)
+    p[0, :8] = 0.0
+    p[1, :8] = torch.tensor([-12.0, -6.0, -0.75, 0.5, 3.0, 9.0, -1e-3, 1e-3]).to(torch.bfloat16)
+    p = p.cuda()
+    _, t = ft.linear_fwd(w, x, ws)
+    t = t.clone()
+    dx, da, db = ft.linear_bwd(w, x, t, dy, ws)
+    dx, da, db = dx.clone(), da.clone(), db.clone()
+    dp_ref = ft.gelu_tanh_bwd(p, dx)
+    dp, da2, db2 = ft.linear_bwd_gelu(w, x, t, dy, p, ws)
+    torch.cuda.synchronize()
+    assert ws.device_status() == 0
+    assert torch.equal(dp, dp_ref), "dP differs from dX followed by the GELU-backward kernel"
+    assert torch.equal(da2, da) and torch.equal(db2, db)
