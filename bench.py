@@ -240,6 +240,181 @@ def cpu_baseline(spec, budget_s=12.0, rows=512):
                       f"(quantize + fwd + bwd, fp64 products) in {time.perf_counter() - t0:.1f} s"}
 
 
+def run_mlp_pair(args):
+    """The MLP pair of a FLUX block (C3): FC1 4608 x 3072 -> 12288, GELU-tanh, FC2 12288 ->
+    3072, forward and backward, with GELU and its derivative fused into the 4-bit GEMMs'
+    epilogues (FC1's also takes max|H| for FC2's quantizer).  The unfused sequence (separate
+    GELU kernels, FC2 taking its own max) is timed in the same run for comparison."""
+    import torch
+
+    from diffusion_dit_b200 import fourtune as ft
+    from diffusion_dit_b200 import prep, workloads as wl
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    up, down = wl.FLUX_MLP_UP, wl.FLUX_MLP_DOWN
+    M = up.M
+
+    def weights(spec):
+        inp = wl.make_layer_inputs(spec, seed=0)
+        split = prep.svd_split(inp.w, spec.r_s)
+        w = ft.prepare_weights(split.residual.to(dev), split.ls_up.to(dev), split.ls_down.to(dev),
+                               inp.lora_a.to(dev), inp.lora_b.to(dev), spec.lora_scale)
+        return inp, w
+
+    inp_u, wu = weights(up)
+    inp_d, wd = weights(down)
+    wsu, wsd = ft.Workspace(wu, M, dev), ft.Workspace(wd, M, dev)
+    x, dy = inp_u.x.to(dev), inp_d.dy.to(dev)
+    bf, f32 = torch.bfloat16, torch.float32
+    P = torch.empty(M, up.N, dtype=bf, device=dev)
+    H = torch.empty(M, up.N, dtype=bf, device=dev)
+    hmax = torch.empty(1, dtype=f32, device=dev)
+    tu = torch.empty(M, up.r_s + up.r, dtype=f32, device=dev)
+    td = torch.empty(M, down.r_s + down.r, dtype=f32, device=dev)
+    Y = torch.empty(M, down.N, dtype=bf, device=dev)
+    dP = torch.empty(M, up.N, dtype=bf, device=dev)
+    dH = torch.empty(M, up.N, dtype=bf, device=dev)
+    dX = torch.empty(M, up.K, dtype=bf, device=dev)
+    dAu = torch.empty(up.r, up.K, dtype=f32, device=dev)
+    dBu = torch.empty(up.N, up.r, dtype=f32, device=dev)
+    dAd = torch.empty(down.r, down.K, dtype=f32, device=dev)
+    dBd = torch.empty(down.N, down.r, dtype=f32, device=dev)
+    flush = torch.empty(512 * 1024 * 1024 // 4, dtype=f32, device=dev)
+
+    def fwd_fused():
+        ft.linear_fwd_gelu(wu, x, wsu, p=P, h=H, h_amax=hmax, t_saved=tu)
+        ft.linear_fwd(wd, H, wsd, y=Y, t_saved=td, amax=hmax)
+
+    def bwd_fused():
+        ft.linear_bwd_gelu(wd, H, td, dy, P, wsd, dp=dP, da=dAd, db=dBd)
+        ft.linear_bwd(wu, x, tu, dP, wsu, dx=dX, da=dAu, db=dBu)
+
+    def step_fused():
+        fwd_fused()
+        bwd_fused()
+
+    def step_unfused():
+        ft.linear_fwd(wu, x, wsu, y=P, t_saved=tu)
+        ft.gelu_tanh_fwd(P, h=H)
+        ft.linear_fwd(wd, H, wsd, y=Y, t_saved=td)
+        ft.linear_bwd(wd, H, td, dy, wsd, dx=dH, da=dAd, db=dBd)
+        ft.gelu_tanh_bwd(P, dH, dp=dP)
+        ft.linear_bwd(wu, x, tu, dP, wsu, dx=dX, da=dAu, db=dBu)
+
+    E = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+    gev = [(E(), E()) for _ in range(4)]
+    for b_, a_ in gev:
+        b_.record()
+        a_.record()
+    torch.cuda.synchronize()
+
+    def step_events():  # the four GEMM launches timed by the library, on the launch stream
+        ft.time_next_launch(ft.FT_KERNEL_GEMM, *gev[0])
+        ft.linear_fwd_gelu(wu, x, wsu, p=P, h=H, h_amax=hmax, t_saved=tu)
+        ft.time_next_launch(ft.FT_KERNEL_GEMM, *gev[1])
+        ft.linear_fwd(wd, H, wsd, y=Y, t_saved=td, amax=hmax)
+        ft.time_next_launch(ft.FT_KERNEL_GEMM, *gev[2])
+        ft.linear_bwd_gelu(wd, H, td, dy, P, wsd, dp=dP, da=dAd, db=dBd)
+        ft.time_next_launch(ft.FT_KERNEL_GEMM, *gev[3])
+        ft.linear_bwd(wu, x, tu, dP, wsu, dx=dX, da=dAu, db=dBu)
+
+    graphs = {}
+    for name, fn in (("fused", step_fused), ("unfused", step_unfused), ("fwd", fwd_fused), ("bwd", bwd_fused),
+                     ("events", step_events)):
+        for _ in range(args.warmup):
+            fn()
+        torch.cuda.synchronize()
+        c0 = ft.launch_count()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            fn()
+        graphs[name] = (g, ft.launch_count() - c0)
+        for _ in range(args.warmup):
+            flush.zero_()
+            g.replay()
+    torch.cuda.synchronize()
+    if wsu.device_status() or wsd.device_status():
+        raise RuntimeError("device status reports a timeout during warm-up")
+    Kst = args.steps
+    s_, e_ = E(), E()
+
+    def timed(name):
+        out = []
+        for _ in range(Kst):
+            flush.zero_()
+            s_.record()
+            graphs[name][0].replay()
+            e_.record()
+            torch.cuda.synchronize()
+            out.append(s_.elapsed_time(e_))
+        return out
+
+    gemm_ms = []
+    with ClockSampler(0) as clocks:
+        fused = timed("fused")
+        unfused = timed("unfused")
+        fwd, bwd = timed("fwd"), timed("bwd")
+        for _ in range(Kst):
+            flush.zero_()
+            graphs["events"][0].replay()
+            torch.cuda.synchronize()
+            gemm_ms.extend(b_.elapsed_time(a_) for b_, a_ in gev)
+    if wsu.device_status() or wsd.device_status():
+        raise RuntimeError("device status reports a timeout in the timed region")
+    # end to end through the API: pinned host X and dY in, the four adapter gradients out
+    x_h, dy_h = inp_u.x.pin_memory(), inp_d.dy.pin_memory()
+    outs = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in (dAu, dBu, dAd, dBd)]
+    e2e = []
+    for _ in range(Kst):
+        flush.zero_()
+        s_.record()
+        x.copy_(x_h, non_blocking=True)
+        dy.copy_(dy_h, non_blocking=True)
+        step_fused()
+        for o, t in zip(outs, (dAu, dBu, dAd, dBd)):
+            o.copy_(t, non_blocking=True)
+        e_.record()
+        torch.cuda.synchronize()
+        e2e.append(s_.elapsed_time(e_))
+
+    fu4, fub = layer_flops(M, up.K, up.N, up.r_s, up.r)
+    fd4, fdb = layer_flops(M, down.K, down.N, down.r_s, down.r)
+    flops = fu4 + fub + fd4 + fdb
+    ms = statistics.mean(fused)
+    ms_un = statistics.mean(unfused)
+    f_u, b_u = pass_flops(M, up.K, up.N, up.r_s, up.r)
+    f_d, b_d = pass_flops(M, down.K, down.N, down.r_s, down.r)
+    hbm, bf16_peak, src = peaks()
+    fp4_peak = bf16_peak * NOMINAL_FP4_OVER_BF16
+    gemm_avg = statistics.mean(gemm_ms)
+    achieved = (fu4 + fd4) / 4 / (gemm_avg * 1e-3) / 1e12
+    line = {
+        "metric": METRIC, "value": flops / (ms * 1e-3) / 1e12, "unit": "TFLOP/s", "n_gpus": 1, "steps": Kst,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "nvfp4(e2m1,ue4m3)+bf16", "data": "synthetic",
+        "config": {"workload": f"flux_mlp_pair {M}x{up.K}->{up.N}->{down.N} gelu_tanh fwd+bwd",
+                   "M_tokens_per_gpu": M, "stabilizer_rank": up.r_s, "lora_rank": up.r,
+                   "l2": "flushed between steps (512 MiB write, outside the step events)",
+                   "parallelism": "dp1", "flops_per_step": {"fp4": fu4 + fd4, "bf16": fub + fdb}},
+        "roofline": {"bound": "tensor", "kernel": "gemm_fp4_lowrank_pair_kernel (4 launches per step)",
+                     "achieved": achieved, "peak": fp4_peak, "unit": "TFLOP/s", "frac": achieved / fp4_peak,
+                     "traffic": None, "frac_of_nominal_9pf": achieved / NOMINAL_FP4_TFLOPS,
+                     "peak_source": f"{src} bf16 {bf16_peak} TFLOP/s x {NOMINAL_FP4_OVER_BF16}",
+                     "avg_launch_ms": gemm_avg},
+        "per_pass": {"fwd_ms": statistics.mean(fwd), "fwd_tflops": (f_u + f_d) / (statistics.mean(fwd) * 1e-3) / 1e12,
+                     "bwd_ms": statistics.mean(bwd), "bwd_tflops": (b_u + b_d) / (statistics.mean(bwd) * 1e-3) / 1e12},
+        "unfused": {"ms_per_step": ms_un, "value": flops / (ms_un * 1e-3) / 1e12,
+                    "speedup_of_fusion": ms_un / ms,
+                    "what": "separate GELU and GELU-backward kernels, FC2 takes its own max|H|"},
+        "e2e": {"value": flops / (statistics.mean(e2e) * 1e-3) / 1e12, "unit": "TFLOP/s",
+                "h2d_bytes_per_step": x.numel() * 2 + dy.numel() * 2,
+                "d2h_bytes_per_step": sum(t.numel() * 4 for t in (dAu, dBu, dAd, dBd))},
+        "gpu_launches": graphs["fused"][1] * Kst, "launch_mode": "cuda_graph_replay",
+        "clocks": clocks.summary(),
+    }
+    print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -251,13 +426,19 @@ def main():
     ap.add_argument("--graph", dest="graph", action="store_true", default=True,
                     help="replay each step as a captured CUDA graph (default)")
     ap.add_argument("--no-graph", dest="graph", action="store_false")
-    ap.add_argument("--workload", default="qkv", choices=sorted(WORKLOADS),
-                    help="single-layer workload (default: the attention QKV projection)")
+    ap.add_argument("--workload", default="qkv", choices=sorted(WORKLOADS) + ["mlp"],
+                    help="single-layer workload (default: the attention QKV projection), or mlp: "
+                         "the MLP pair with GELU, fused")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
+    if args.workload == "mlp" and args.impl == "ours":
+        if int(os.environ.get("WORLD_SIZE", "1")) > 1:
+            raise SystemExit("--workload mlp runs on one GPU")
+        run_mlp_pair(args)
+        return
 
     from diffusion_dit_b200 import workloads as wl
-    spec = getattr(wl, WORKLOADS[args.workload])
+    spec = getattr(wl, WORKLOADS.get(args.workload, "FLUX_MLP_UP"))
     if args.impl == "reference":
         run_reference(args, spec)
         return

@@ -18,8 +18,9 @@
 // on both TMEM_FULL barriers; each CTA drains its own 128 x 256 accumulator and releases
 // it on the even CTA's TMEM_EMPTY.  No load is multicast.
 //
-// Warp roles (320 threads per CTA): warp 0 = TMA producer, warp 1 = MMA issuer (even CTA)
-// and TMEM owner, warps 2..5 = epilogue, warps 6..9 = scale writers.
+// Warp roles: warp 0 = TMA producer, warp 1 = MMA issuer (even CTA) and TMEM owner, then
+// the epilogue warps (4, or 8 for the GELU epilogues: two per TMEM lane quarter, 128
+// columns each), then 4 scale writers.
 #include "ft_internal.h"
 #include "ft_ptx.cuh"
 
@@ -42,8 +43,14 @@ constexpr int OFF_SFB = OFF_SFA + SFA_BYTES;
 constexpr int EPI_BYTES = 32 * 64;
 constexpr int OFF_EPI = STAGES * STAGE_BYTES;
 constexpr int BAR_BYTES = 256;
-constexpr int SMEM_BYTES = OFF_EPI + 4 * EPI_BYTES + BAR_BYTES + 1024;
-constexpr int THREADS = 320;
+constexpr int EPI_BUFS = 2;              // staging buffers per epilogue warp (one store in flight)
+// Epilogue warps per variant: 4 (one per TMEM lane quarter, all 256 columns) for the plain
+// GEMM; 8 (two per quarter, 128 columns each) for the GELU epilogues, whose arithmetic
+// needs two warps per scheduler to hide its latency.
+__host__ __device__ constexpr int epi_warps(int epi) { return epi == kEpiPlain ? 4 : 8; }
+__host__ __device__ constexpr int epi_region(int epi) { return epi_warps(epi) * EPI_BUFS * EPI_BYTES; }
+__host__ __device__ constexpr int smem_bytes(int epi) { return OFF_EPI + epi_region(epi) + BAR_BYTES + 1024; }
+__host__ __device__ constexpr int threads(int epi) { return 32 * (2 + epi_warps(epi) + 4); }
 
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t COL_ACC = 0;
@@ -51,7 +58,7 @@ constexpr uint32_t COL_SFA = 256;                    // STAGES x 16 columns
 constexpr uint32_t COL_SFB = COL_SFA + STAGES * 16;  // STAGES x 32 columns
 
 static_assert(STAGE_BYTES % 1024 == 0, "stage must keep 1024-byte alignment");
-static_assert(SMEM_BYTES <= 232448, "exceeds 227 KB of dynamic shared memory");
+static_assert(smem_bytes(kEpiGelu) <= 232448, "exceeds 227 KB of dynamic shared memory");
 static_assert(COL_SFB + STAGES * 32 <= TMEM_COLS, "tensor memory overflow");
 
 __host__ __device__ constexpr int BAR_FULL(int s) { return s; }
@@ -66,7 +73,7 @@ constexpr int OFF_ABORT = OFF_TMEM_SLOT + 4;
 static_assert(OFF_ABORT + 4 <= BAR_BYTES, "barrier area overflow");
 
 template <int EPI>
-__global__ void __launch_bounds__(THREADS, 1)
+__global__ void __launch_bounds__(threads(EPI), 1)
     gemm_fp4_lowrank_pair_kernel(const __grid_constant__ CUtensorMap tmA,
                                  const __grid_constant__ CUtensorMap tmB,
                                  const __grid_constant__ CUtensorMap tmLA,
@@ -78,8 +85,10 @@ __global__ void __launch_bounds__(THREADS, 1)
     const uint32_t pad = (1024 - (raw_u32 & 1023)) & 1023;
     uint8_t* base = smem_raw + pad;
     const uint32_t base_u32 = raw_u32 + pad;
-    uint8_t* bar_area = base + OFF_EPI + 4 * EPI_BYTES;
-    auto bar = [&](int i) { return base_u32 + OFF_EPI + 4 * EPI_BYTES + 8 * i; };
+    constexpr int EPI_WARPS = epi_warps(EPI);
+    constexpr int EPI_COLS = BN / (EPI_WARPS / 4);  // tile columns per epilogue warp
+    uint8_t* bar_area = base + OFF_EPI + epi_region(EPI);
+    auto bar = [&](int i) { return base_u32 + OFF_EPI + epi_region(EPI) + 8 * i; };
     auto stage = [&](int s) { return base_u32 + s * STAGE_BYTES; };
     volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(bar_area + OFF_TMEM_SLOT);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(bar_area + OFF_ABORT);
@@ -103,7 +112,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             mbar_init(bar(BAR_SF_READY(i)), 8);   // 4 scale warps x 2 CTAs (even CTA's copy used)
         }
         mbar_init(bar(BAR_TMEM_FULL), 1);
-        mbar_init(bar(BAR_TMEM_EMPTY), 8);        // 4 epilogue warps x 2 CTAs (even CTA's copy used)
+        mbar_init(bar(BAR_TMEM_EMPTY), 2 * EPI_WARPS);  // epilogue warps x 2 CTAs (even CTA's copy used)
         mbar_init(bar(BAR_FINAL), 1);
         *abort_flag = 0;
         fence_mbar_init();
@@ -215,7 +224,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             volatile int no_abort = 0;
             mbar_wait(bar(BAR_FINAL), 0, &no_abort, p.status);
         }
-    } else if (warp >= 6) {
+    } else if (warp >= 2 + EPI_WARPS) {
         // ---------------------------------------------------------------- scale writers
         // Same tensor-memory layout as the single-CTA kernel: lane l of quarter q holds row
         // l of every 512-byte scale atom (4 columns per A k-block, 8 per B k-block).
@@ -257,21 +266,31 @@ __global__ void __launch_bounds__(THREADS, 1)
     } else {
         // ---------------------------------------------------------------- epilogue (both CTAs)
         const int q = warp & 3;
+        const int cbase = EPI_COLS * ((warp - 2) >> 2);  // this warp's first tile column
         const float ga = *p.ga, gb = *p.gb;
         const float c = 1.0f / (ga * gb);
         const uint32_t empty_even = mapa_shared(bar(BAR_TMEM_EMPTY), 0);
         float hmax = 0.0f;  // max |gelu output| of this thread's elements (GELU epilogue)
+        int sc = 0;         // stores staged by this warp (staging buffer sc % 2)
         int ti = 0;
         for (int t = pair; t < num_tiles && !*abort_flag; t += num_pairs, ++ti) {
             const int mb2 = t % MB2, nb = t / MB2;
             if (!mbar_wait(bar(BAR_TMEM_FULL), ti & 1, abort_flag, p.status)) break;
             tc_fence_after();
-            const uint32_t lane_addr = tmem + COL_ACC + (static_cast<uint32_t>(32 * q) << 16);
-            const uint32_t stage_u32 = base_u32 + OFF_EPI + (warp - 2) * EPI_BYTES;
-            uint8_t* stage_ptr = base + OFF_EPI + (warp - 2) * EPI_BYTES;
-            uint32_t pk[BN / 2];
+            if constexpr (EPI == kEpiGeluBwd) {
+                // this thread's 512 bytes of gelu_in for the tile, into L2 while the drain runs
+                const __nv_bfloat16* r = p.gelu_in +
+                    static_cast<size_t>((mb2 * 2 + static_cast<int>(rank)) * BM + 32 * q + lane) * p.ldo + nb * BN +
+                    cbase;
 #pragma unroll
-            for (int ch = 0; ch < BN / 32; ++ch) {
+                for (int i = 0; i < EPI_COLS / 64; ++i) prefetch_l2(r + 64 * i);
+            }
+            const uint32_t lane_addr = tmem + COL_ACC + cbase + (static_cast<uint32_t>(32 * q) << 16);
+            const uint32_t stage0_u32 = base_u32 + OFF_EPI + (warp - 2) * EPI_BUFS * EPI_BYTES;
+            uint8_t* stage0_ptr = base + OFF_EPI + (warp - 2) * EPI_BUFS * EPI_BYTES;
+            uint32_t pk[EPI_COLS / 2];
+#pragma unroll
+            for (int ch = 0; ch < EPI_COLS / 32; ++ch) {
                 uint32_t v[32];
                 tmem_ld_32x32b_x32(lane_addr + ch * 32, v);
                 tmem_ld_wait();
@@ -286,21 +305,24 @@ __global__ void __launch_bounds__(THREADS, 1)
             const int row0 = (mb2 * 2 + static_cast<int>(rank)) * BM + 32 * q;
             // GELU-backward epilogue: this thread's row of gelu_in, one 32-column chunk ahead
             const __nv_bfloat16* prow =
-                EPI == kEpiGeluBwd ? p.gelu_in + static_cast<size_t>(row0 + lane) * p.ldo + nb * BN : nullptr;
+                EPI == kEpiGeluBwd ? p.gelu_in + static_cast<size_t>(row0 + lane) * p.ldo + nb * BN + cbase : nullptr;
             uint4 pin[4];
             if constexpr (EPI == kEpiGeluBwd) {
 #pragma unroll
                 for (int c4 = 0; c4 < 4; ++c4) pin[c4] = *reinterpret_cast<const uint4*>(prow + 8 * c4);
             }
 #pragma unroll
-            for (int ch = 0; ch < BN / 32; ++ch) {
-                if (lane == 0) bulk_wait_group_read0();
+            for (int ch = 0; ch < EPI_COLS / 32; ++ch) {
+                uint32_t stage_u32 = stage0_u32 + (sc & 1) * EPI_BYTES;
+                uint8_t* stage_ptr = stage0_ptr + (sc & 1) * EPI_BYTES;
+                ++sc;
+                if (lane == 0) bulk_wait_group_read1();  // this buffer's last store has read it
                 __syncwarp();
                 if constexpr (EPI == kEpiGeluBwd) {
                     uint4 cur[4];
 #pragma unroll
                     for (int c4 = 0; c4 < 4; ++c4) cur[c4] = pin[c4];
-                    if (ch + 1 < BN / 32) {
+                    if (ch + 1 < EPI_COLS / 32) {
 #pragma unroll
                         for (int c4 = 0; c4 < 4; ++c4)
                             pin[c4] = *reinterpret_cast<const uint4*>(prow + 32 * (ch + 1) + 8 * c4);
@@ -323,12 +345,15 @@ __global__ void __launch_bounds__(THREADS, 1)
                 fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0) {
-                    tma_store_2d(&tmOut, stage_u32, nb * BN + ch * 32, row0);
+                    tma_store_2d(&tmOut, stage_u32, nb * BN + cbase + ch * 32, row0);
                     bulk_commit_group();
                 }
                 if constexpr (EPI == kEpiGelu) {
-                    // the same chunk through GELU, once the store above has read the buffer
-                    if (lane == 0) bulk_wait_group_read0();
+                    // the same chunk through GELU, staged in the other buffer
+                    stage_u32 = stage0_u32 + (sc & 1) * EPI_BYTES;
+                    stage_ptr = stage0_ptr + (sc & 1) * EPI_BYTES;
+                    ++sc;
+                    if (lane == 0) bulk_wait_group_read1();
                     __syncwarp();
 #pragma unroll
                     for (int c4 = 0; c4 < 4; ++c4) {
@@ -342,7 +367,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                     fence_proxy_async_smem();
                     __syncwarp();
                     if (lane == 0) {
-                        tma_store_2d(&tmAct, stage_u32, nb * BN + ch * 32, row0);
+                        tma_store_2d(&tmAct, stage_u32, nb * BN + cbase + ch * 32, row0);
                         bulk_commit_group();
                     }
                 }
@@ -377,8 +402,10 @@ cudaError_t launch_variant(const CUtensorMap& tmA, const CUtensorMap& tmB, const
                            const GemmFp4Args& args, cudaLaunchConfig_t cfg) {
     using namespace gemm2;
     static const cudaError_t attr = cudaFuncSetAttribute(
-        gemm_fp4_lowrank_pair_kernel<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+        gemm_fp4_lowrank_pair_kernel<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes(EPI));
     if (attr != cudaSuccess) return attr;
+    cfg.blockDim = dim3(threads(EPI));
+    cfg.dynamicSmemBytes = smem_bytes(EPI);
     return cudaLaunchKernelEx(&cfg, gemm_fp4_lowrank_pair_kernel<EPI>, tmA, tmB, tmLA, tmLB, tmOut, tmAct, args);
 }
 
@@ -394,8 +421,6 @@ cudaError_t launch_gemm_fp4_lowrank_pair(const CUtensorMap& tmA, const CUtensorM
     if (pairs > tiles) pairs = tiles;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(2 * pairs));
-    cfg.blockDim = dim3(THREADS);
-    cfg.dynamicSmemBytes = SMEM_BYTES;
     cfg.stream = stream;
     cudaLaunchAttribute at[2];
     at[0].id = cudaLaunchAttributeClusterDimension;

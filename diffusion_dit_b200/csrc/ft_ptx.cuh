@@ -127,6 +127,16 @@ __device__ __forceinline__ void bulk_wait_group_read0() {
     asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
 }
 
+// The bulk groups this thread committed, except the most recent one, have finished
+// reading their shared-memory source (double-buffered staging).
+__device__ __forceinline__ void bulk_wait_group_read1() {
+    asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+}
+
+__device__ __forceinline__ void prefetch_l2(const void* p) {
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(reinterpret_cast<uint64_t>(p)));
+}
+
 __device__ __forceinline__ void bulk_wait_group0() {
     asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
 }
@@ -419,9 +429,13 @@ __device__ __forceinline__ float ue4m3_to_f32(uint32_t code) {
 
 // GELU, tanh form: 0.5 p (1 + tanh(u)), u = sqrt(2/pi) (p + 0.044715 p^3), evaluated as
 // p * sigmoid(2u), the same function (0.5 (1 + tanh u) = 1 / (1 + exp(-2u))), which keeps
-// full relative accuracy for large negative p where 1 + tanh(u) cancels.  Every step is
-// an explicitly rounded fp32 operation (no contraction), so the stand-alone kernel and
-// the GEMM epilogue produce the same bits; exp is the library expf.
+// full relative accuracy for large negative p where 1 + tanh(u) cancels.  The exponential
+// and the divisions are CUDA's fast intrinsics (__expf, __fdividef: a few ulp, ~1e-6
+// relative for the arguments that reach a bf16 result), so the GEMM epilogue that applies
+// it stays cheap next to the tile's MMAs; the polynomial steps are explicitly rounded.
+// The stand-alone kernels use these same functions, so they and the epilogue agree bit
+// for bit.  For |2u| beyond the fp32 exp range the sigmoid goes to 0 or 1 as it should
+// (__fdividef(x, inf) = 0).
 __device__ __forceinline__ float gelu_tanh_u(float p) {
     const float k = 0.7978845608028654f;  // sqrt(2 / pi)
     const float p3 = __fmul_rn(__fmul_rn(p, p), p);
@@ -429,7 +443,7 @@ __device__ __forceinline__ float gelu_tanh_u(float p) {
 }
 
 __device__ __forceinline__ float gelu_tanh_f(float p) {
-    return __fdiv_rn(p, __fadd_rn(1.0f, expf(__fmul_rn(-2.0f, gelu_tanh_u(p)))));
+    return __fdividef(p, __fadd_rn(1.0f, __expf(__fmul_rn(-2.0f, gelu_tanh_u(p)))));
 }
 
 // dP = dH * gelu'(P); with s = sigmoid(2u): gelu' = s + 2 p s (1 - s) u', and
@@ -437,8 +451,8 @@ __device__ __forceinline__ float gelu_tanh_f(float p) {
 __device__ __forceinline__ float gelu_tanh_bwd_f(float p, float dh) {
     const float k = 0.7978845608028654f;
     const float u = gelu_tanh_u(p);
-    const float sg = __fdiv_rn(1.0f, __fadd_rn(1.0f, expf(__fmul_rn(-2.0f, u))));
-    const float one_minus = __fdiv_rn(1.0f, __fadd_rn(1.0f, expf(__fmul_rn(2.0f, u))));
+    const float sg = __fdividef(1.0f, __fadd_rn(1.0f, __expf(__fmul_rn(-2.0f, u))));
+    const float one_minus = __fdividef(1.0f, __fadd_rn(1.0f, __expf(__fmul_rn(2.0f, u))));
     const float du = __fmul_rn(k, __fadd_rn(1.0f, __fmul_rn(3.0f * 0.044715f, __fmul_rn(p, p))));
     const float g = __fadd_rn(sg, __fmul_rn(__fmul_rn(__fmul_rn(__fmul_rn(2.0f, p), sg), one_minus), du));
     return __fmul_rn(dh, g);
