@@ -137,18 +137,20 @@ float ora_global_scale(float amax_t) {
 }
 
 /*
- * Quantize a matrix x[rows, cols] (bf16 or fp32, row stride ld elements) in 16x16
- * blocks.
+ * Quantize a matrix x[rows, cols] (bf16 or fp32, row stride ld elements) in blocks of
+ * bh rows x 16 columns: bh = 16 is FourTune's block-wise 16x16 (section 3.1), bh = 1 the
+ * group-wise 1x16 it is compared with (section 4.3, "Impact of Quantization Granularity",
+ * Table 5).  The same two-level scaling either way.
  * amax_t < 0 means "compute it here"; otherwise it is used as given.
  * Outputs (caller-allocated):
  *   codes  [rows, cols/2]  element (i, 2j) in the low nibble of byte (i, j)
- *   scales [rows/16, cols/16]  one UE4M3 byte per block
+ *   scales [rows/bh, cols/16]  one UE4M3 byte per block
  *   *g_out                 the tensor factor g
- * rows and cols must be multiples of 16.  Returns 0, or -1 on bad shape.
+ * rows must be a multiple of bh, cols of 16.  Returns 0, or -1 on bad shape.
  */
-static int quantize_any(const void* x, int is_f32, int64_t rows, int64_t cols, int64_t ld,
-                        float amax_t, uint8_t* codes, uint8_t* scales, float* g_out) {
-    if (rows % 16 || cols % 16 || rows < 0 || cols < 0) return -1;
+static int quantize_blocks(const void* x, int is_f32, int64_t rows, int64_t cols, int64_t ld, int bh,
+                           float amax_t, uint8_t* codes, uint8_t* scales, float* g_out) {
+    if (bh < 1 || rows % bh || cols % 16 || rows < 0 || cols < 0) return -1;
     if (amax_t < 0.0f) amax_t = amax_any(x, is_f32, rows, cols, ld);
     int degenerate = 1;
     float g = 1.0f;
@@ -162,14 +164,14 @@ static int quantize_any(const void* x, int is_f32, int64_t rows, int64_t cols, i
     }
     *g_out = g;
     memset(codes, 0, (size_t)(rows * (cols / 2)));
-    memset(scales, 0, (size_t)((rows / 16) * (cols / 16)));
+    memset(scales, 0, (size_t)((rows / bh) * (cols / 16)));
     if (degenerate) return 0;
-    for (int64_t bi = 0; bi < rows / 16; ++bi) {
+    for (int64_t bi = 0; bi < rows / bh; ++bi) {
         for (int64_t bj = 0; bj < cols / 16; ++bj) {
             float amax_b = 0.0f;
-            for (int r = 0; r < 16; ++r)
+            for (int r = 0; r < bh; ++r)
                 for (int c = 0; c < 16; ++c) {
-                    float a = fabsf(load_elem(x, is_f32, (bi * 16 + r) * ld + bj * 16 + c));
+                    float a = fabsf(load_elem(x, is_f32, (bi * bh + r) * ld + bj * 16 + c));
                     if (a > amax_b) amax_b = a;
                 }
             volatile float six = 6.0f;
@@ -179,9 +181,9 @@ static int quantize_any(const void* x, int is_f32, int64_t rows, int64_t cols, i
             scales[bi * (cols / 16) + bj] = (uint8_t)sb;
             if (sb == 0) continue; /* codes stay 0 */
             float inv = g / (float)ue4m3_value(sb);
-            for (int r = 0; r < 16; ++r) {
+            for (int r = 0; r < bh; ++r) {
                 for (int c = 0; c < 16; ++c) {
-                    int64_t i = bi * 16 + r, j = bj * 16 + c;
+                    int64_t i = bi * bh + r, j = bj * 16 + c;
                     float v = load_elem(x, is_f32, i * ld + j) * inv;
                     int code = ora_e2m1_encode(v);
                     uint8_t* byte = &codes[i * (cols / 2) + j / 2];
@@ -196,24 +198,35 @@ static int quantize_any(const void* x, int is_f32, int64_t rows, int64_t cols, i
 
 int ora_quantize_block16(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld,
                          float amax_t, uint8_t* codes, uint8_t* scales, float* g_out) {
-    return quantize_any(x, 0, rows, cols, ld, amax_t, codes, scales, g_out);
+    return quantize_blocks(x, 0, rows, cols, ld, 16, amax_t, codes, scales, g_out);
 }
 
 int ora_quantize_block16_f32(const float* x, int64_t rows, int64_t cols, int64_t ld,
                              float amax_t, uint8_t* codes, uint8_t* scales, float* g_out) {
-    return quantize_any(x, 1, rows, cols, ld, amax_t, codes, scales, g_out);
+    return quantize_blocks(x, 1, rows, cols, ld, 16, amax_t, codes, scales, g_out);
 }
 
-/* Dequantize: xhat = val(code) * val(sb) / g, evaluated in double. */
-void ora_dequantize_block16(const uint8_t* codes, const uint8_t* scales, float g,
-                            int64_t rows, int64_t cols, double* out) {
+/* Group-wise 1x16 (bf16 input): scales [rows, cols/16]. */
+int ora_quantize_1x16(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld,
+                      float amax_t, uint8_t* codes, uint8_t* scales, float* g_out) {
+    return quantize_blocks(x, 0, rows, cols, ld, 1, amax_t, codes, scales, g_out);
+}
+
+/* Dequantize blocks of bh rows x 16: xhat = val(code) * val(sb) / g, in double. */
+void ora_dequantize_blocks(const uint8_t* codes, const uint8_t* scales, float g, int64_t rows,
+                           int64_t cols, int bh, double* out) {
     for (int64_t i = 0; i < rows; ++i)
         for (int64_t j = 0; j < cols; ++j) {
             uint8_t byte = codes[i * (cols / 2) + j / 2];
             int code = (j & 1) ? (byte >> 4) : (byte & 15);
-            double sb = ue4m3_value(scales[(i / 16) * (cols / 16) + j / 16]);
+            double sb = ue4m3_value(scales[(i / bh) * (cols / 16) + j / 16]);
             out[i * cols + j] = ora_e2m1_value(code) * sb / (double)g;
         }
+}
+
+void ora_dequantize_block16(const uint8_t* codes, const uint8_t* scales, float g,
+                            int64_t rows, int64_t cols, double* out) {
+    ora_dequantize_blocks(codes, scales, g, rows, cols, 16, out);
 }
 
 /* Transpose of a quantized matrix without requantization (section 3.2): the codes

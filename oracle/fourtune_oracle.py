@@ -86,6 +86,9 @@ def lib():
         L.ora_amax_f32.argtypes = [vp, i64, i64, i64]
         L.ora_amax_f32.restype = f32
         L.ora_dequantize_block16.argtypes = [vp, vp, f32, i64, i64, vp]
+        L.ora_quantize_1x16.argtypes = [vp, i64, i64, i64, f32, vp, vp, vp]
+        L.ora_quantize_1x16.restype = ctypes.c_int
+        L.ora_dequantize_blocks.argtypes = [vp, vp, f32, i64, i64, ctypes.c_int, vp]
         L.ora_transpose_block16.argtypes = [vp, vp, i64, i64, vp, vp]
         L.ora_e2m1_encode_array.argtypes = [vp, i64, vp]
         L.ora_ue4m3_encode_array.argtypes = [vp, i64, vp]
@@ -148,22 +151,26 @@ def global_scale(amax_t: float) -> float:
 
 @dataclasses.dataclass
 class QTensor:
-    """A 16x16-block quantized matrix: codes [rows, cols/2] (element 2j in the low
-    nibble), scales [rows/16, cols/16] UE4M3 bytes, tensor factor g (fp32)."""
+    """A block-quantized matrix: codes [rows, cols/2] (element 2j in the low nibble),
+    scales [rows/block_rows, cols/16] UE4M3 bytes, tensor factor g (fp32).  block_rows is
+    16 for the 16x16 blocks of section 3.1, 1 for the group-wise 1x16 of Table 5."""
 
     codes: np.ndarray
     scales: np.ndarray
     g: float
     rows: int
     cols: int
+    block_rows: int = 16
 
     def dequantize(self) -> np.ndarray:
         out = np.empty((self.rows, self.cols), dtype=np.float64)
-        lib().ora_dequantize_block16(_ptr(self.codes), _ptr(self.scales), np.float32(self.g),
-                                     self.rows, self.cols, _ptr(out))
+        lib().ora_dequantize_blocks(_ptr(self.codes), _ptr(self.scales), np.float32(self.g),
+                                    self.rows, self.cols, self.block_rows, _ptr(out))
         return out
 
     def transpose(self) -> "QTensor":
+        if self.block_rows != 16:
+            raise ValueError("only 16x16 blocks transpose without requantization")
         ct = np.empty((self.cols, self.rows // 2), dtype=np.uint8)
         st = np.empty((self.cols // 16, self.rows // 16), dtype=np.uint8)
         lib().ora_transpose_block16(_ptr(self.codes), _ptr(self.scales), self.rows, self.cols,
@@ -189,6 +196,22 @@ def quantize_block16(x: torch.Tensor, amax_t: Optional[float] = None) -> QTensor
     if rc != 0:
         raise ValueError("rows and cols must be multiples of 16")
     return QTensor(codes, scales, float(g[0]), rows, cols)
+
+
+def quantize_1x16(x: torch.Tensor, amax_t: Optional[float] = None) -> QTensor:
+    """The group-wise 1x16 granularity FourTune compares its 16x16 blocks with (section
+    4.3, "Impact of Quantization Granularity", Table 5): each row's 16 consecutive
+    elements share one UE4M3 scale, with the same tensor factor g.  ``x`` is bf16."""
+    xb = bf16_bits(x)
+    rows, cols = xb.shape
+    codes = np.empty((rows, cols // 2), dtype=np.uint8)
+    scales = np.empty((rows, cols // 16), dtype=np.uint8)
+    g = np.zeros(1, dtype=np.float32)
+    rc = lib().ora_quantize_1x16(_ptr(xb), rows, cols, cols, -1.0 if amax_t is None else float(amax_t),
+                                 _ptr(codes), _ptr(scales), _ptr(g))
+    if rc != 0:
+        raise ValueError("cols must be a multiple of 16")
+    return QTensor(codes, scales, float(g[0]), rows, cols, block_rows=1)
 
 
 # ----------------------------------------------------------------------------
@@ -277,10 +300,11 @@ class FwdResult:
 
 
 def linear_fwd(x: torch.Tensor, layer: Layer, amax_x: Optional[float] = None,
-               rows: Optional[np.ndarray] = None) -> FwdResult:
+               rows: Optional[np.ndarray] = None, x_block_rows: int = 16) -> FwdResult:
     """Eq. (2): Y = Xhat Rhat^T + X Ls_down^T Ls_up^T + s X A^T B^T.
-    ``rows`` (optional) evaluates Y only for those token rows."""
-    qx = quantize_block16(x, amax_x)
+    ``rows`` (optional) evaluates Y only for those token rows.  ``x_block_rows`` = 1
+    quantizes X group-wise 1x16 (Table 5's comparison, forward only) instead of 16x16."""
+    qx = quantize_block16(x, amax_x) if x_block_rows == 16 else quantize_1x16(x, amax_x)
     Xd = bf16_f64(x)
     Xh = qx.dequantize()
     Rh = layer.qr.dequantize()
