@@ -130,7 +130,7 @@ LinearWs linear_ws(int64_t M, int64_t N, int64_t K, int R, int r) {
     w.status = take(16);
     w.scal = take(16 * sizeof(float));
     w.qx_codes = take(static_cast<size_t>(M) * K / 2);
-    w.qx_scales = take(static_cast<size_t>(M) * K / 256);
+    w.qx_scales = take(static_cast<size_t>(M) * K / 16);  // 16x16 blocks use 1/16 of it, 1x16 groups all
     w.qx_sf = take(static_cast<size_t>(M) * K / 16);
     w.dn = take(static_cast<size_t>(Rp) * K * 2);
     w.upcat = take(static_cast<size_t>(N) * KL * 2);
@@ -187,7 +187,7 @@ __nv_bfloat16* bfm(void* p) { return static_cast<__nv_bfloat16*>(p); }
 ft_status quantize_operand(const void* x, int64_t rows, int64_t cols, int64_t ld, const float* amax_or_null,
                            float* amax_slot, bool amax_slot_cleared, uint8_t* codes, uint8_t* scales, uint8_t* sf, float* g,
                            const void* w, int Rp, float* partial, int* splits, int* status,
-                           const DeviceInfo& dev, cudaStream_t st) {
+                           const DeviceInfo& dev, cudaStream_t st, int block_rows = 16) {
     const float* amax = amax_or_null;
     if (!amax) {
         FT_CUDA(ft::launch_amax(x, false, rows, cols, ld, amax_slot, amax_slot_cleared, dev.num_sms, st));
@@ -213,6 +213,7 @@ ft_status quantize_operand(const void* x, int64_t rows, int64_t cols, int64_t ld
     a.g_out = g;
     a.partial = partial;
     a.status = status;
+    a.block_rows = block_rows;
     FT_CUDA(ft::launch_quant_down(tX, tW, a, s, st));
     *splits = s;
     return FT_OK;
@@ -361,6 +362,28 @@ size_t fourtune_quantize_workspace_bytes(int64_t rows, int64_t cols, int32_t r_d
     return quant_ws(rows, cols, r_down).total;
 }
 
+ft_status fourtune_quantize_1x16(const void* x_dev, int64_t rows, int64_t cols, int64_t ld,
+                                 const float* amax_or_null, const ft_fp4* out, void* ws, size_t ws_bytes,
+                                 void* stream) {
+    if (!x_dev || !out) return FT_ERR_INVALID_ARG;
+    if (rows <= 0 || cols <= 0 || ld < cols) return FT_ERR_INVALID_ARG;
+    if (rows % 128 || cols % 64 || ld % 8) return FT_ERR_SHAPE;
+    FT_TRY(check_fp4(*out, rows, cols, false));
+    if (!aligned16(x_dev)) return FT_ERR_ALIGN;
+    const QuantWs qw = quant_ws(rows, cols, 0);
+    if (!ws || ws_bytes < qw.total) return FT_ERR_WORKSPACE;
+    if (reinterpret_cast<uintptr_t>(ws) % kAlign) return FT_ERR_ALIGN;
+    DeviceInfo dev;
+    FT_TRY(device_info(&dev));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    uint8_t* W = static_cast<uint8_t*>(ws);
+    int splits = 1;
+    return quantize_operand(x_dev, rows, cols, ld, amax_or_null, reinterpret_cast<float*>(W + qw.amax), false,
+                            out->codes, out->scales, out->sf_mma, out->g, nullptr, 0,
+                            reinterpret_cast<float*>(W + qw.partial), &splits,
+                            reinterpret_cast<int*>(W + qw.status), dev, st, 1);
+}
+
 ft_status fourtune_quantize_block16(const void* x_dev, int32_t x_dtype, int64_t rows, int64_t cols,
                                     int64_t ld, const float* amax_or_null, const void* down_dev,
                                     int32_t r_down, float* down_out_dev, const ft_fp4* out,
@@ -439,7 +462,7 @@ namespace {
 // max |h| into *h_amax_dev).
 ft_status linear_fwd_impl(const ft_linear* L, const void* x_dev, int64_t M, const float* amax_or_null,
                           void* y_dev, float* t_saved_dev, void* h_dev, float* h_amax_dev, void* ws,
-                          size_t ws_bytes, void* stream) {
+                          size_t ws_bytes, void* stream, int x_block_rows = 16) {
     FT_TRY(check_layer(L));
     const int R = L->r_s + L->r;
     if (!x_dev || !y_dev || (R > 0 && !t_saved_dev) || M <= 0) return FT_ERR_INVALID_ARG;
@@ -474,7 +497,8 @@ ft_status linear_fwd_impl(const ft_linear* L, const void* x_dev, int64_t M, cons
         FT_CUDA(cudaMemsetAsync(h_amax_dev, 0, sizeof(float), st));
     int splits = 1;
     FT_TRY(quantize_operand(x_dev, M, K, K, amax_or_null, scal + SC_AMAX_X, R > 0, W + w.qx_codes, W + w.qx_scales,
-                            W + w.qx_sf, scal + SC_G_X, W + w.dn, Rp, partial, &splits, status, dev, st));
+                            W + w.qx_sf, scal + SC_G_X, W + w.dn, Rp, partial, &splits, status, dev, st,
+                            x_block_rows));
     if (R > 0) {
         ft::LowRankFinalizeArgs f{};
         f.partial = partial;
@@ -500,6 +524,12 @@ ft_status linear_fwd_impl(const ft_linear* L, const void* x_dev, int64_t M, cons
 ft_status fourtune_linear_fwd(const ft_linear* L, const void* x_dev, int64_t M, const float* amax_or_null,
                               void* y_dev, float* t_saved_dev, void* ws, size_t ws_bytes, void* stream) {
     return linear_fwd_impl(L, x_dev, M, amax_or_null, y_dev, t_saved_dev, nullptr, nullptr, ws, ws_bytes, stream);
+}
+
+ft_status fourtune_linear_fwd_1x16(const ft_linear* L, const void* x_dev, int64_t M, const float* amax_or_null,
+                                   void* y_dev, float* t_saved_dev, void* ws, size_t ws_bytes, void* stream) {
+    return linear_fwd_impl(L, x_dev, M, amax_or_null, y_dev, t_saved_dev, nullptr, nullptr, ws, ws_bytes, stream,
+                           1);
 }
 
 ft_status fourtune_linear_fwd_gelu(const ft_linear* L, const void* x_dev, int64_t M, const float* amax_or_null,

@@ -105,6 +105,7 @@ struct QuantDownArgs {
     float* g_out;
     float* partial;          // [splits, rows, Rp] fp32
     int* status;
+    int block_rows;          // 16: 16x16 blocks, scales [rows/16, cols/16]; 1: 1x16 groups, [rows, cols/16]
 };
 int quant_down_splits(int64_t rows, int64_t cols, int num_sms);
 size_t quant_down_smem_bytes(int Rp);

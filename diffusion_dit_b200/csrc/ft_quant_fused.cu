@@ -60,6 +60,7 @@ __device__ __forceinline__ float warp_max(float v) {
     return v;
 }
 
+template <int GRAN>
 __global__ void __launch_bounds__(THREADS, 1)
     quant_down_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
                       const QuantDownArgs p) {
@@ -195,42 +196,71 @@ __global__ void __launch_bounds__(THREADS, 1)
             w[1] = *reinterpret_cast<const uint4*>(tile + rA * 128 + (((2 * j + 1) ^ (rA & 7)) << 4));
             w[2] = *reinterpret_cast<const uint4*>(tile + rB * 128 + (((2 * j) ^ (rB & 7)) << 4));
             w[3] = *reinterpret_cast<const uint4*>(tile + rB * 128 + (((2 * j + 1) ^ (rB & 7)) << 4));
-            // block max |x| on the bf16 bit patterns (sign cleared: integer order = numeric order)
-            uint32_t m2 = 0;
-#pragma unroll
-            for (int q2 = 0; q2 < 4; ++q2)
-                m2 = __vmaxu2(m2, __vmaxu2(__vmaxu2(w[q2].x & 0x7FFF7FFFu, w[q2].y & 0x7FFF7FFFu),
-                                           __vmaxu2(w[q2].z & 0x7FFF7FFFu, w[q2].w & 0x7FFF7FFFu)));
-            uint32_t amb = max(m2 & 0xFFFFu, m2 >> 16);
-            amb = max(amb, __shfl_xor_sync(0xffffffffu, amb, 1));
-            amb = max(amb, __shfl_xor_sync(0xffffffffu, amb, 2));
-            amb = max(amb, __shfl_xor_sync(0xffffffffu, amb, 4));
-            const uint32_t sb =
-                degenerate ? 0u : cvt_ue4m3(__fmul_rn(div6_bf16(__uint_as_float(amb << 16)), g));
-            const float inv = inv_lut[sb];
-            uint32_t code[4];  // row rA: words 0, 1; row rB: words 2, 3
-#pragma unroll
-            for (int q2 = 0; q2 < 4; ++q2) {
-                float v[8];
-                v[0] = __fmul_rn(bf16lo_to_f32(w[q2].x), inv); v[1] = __fmul_rn(bf16hi_to_f32(w[q2].x), inv);
-                v[2] = __fmul_rn(bf16lo_to_f32(w[q2].y), inv); v[3] = __fmul_rn(bf16hi_to_f32(w[q2].y), inv);
-                v[4] = __fmul_rn(bf16lo_to_f32(w[q2].z), inv); v[5] = __fmul_rn(bf16hi_to_f32(w[q2].z), inv);
-                v[6] = __fmul_rn(bf16lo_to_f32(w[q2].w), inv); v[7] = __fmul_rn(bf16hi_to_f32(w[q2].w), inv);
-                code[q2] = sb ? cvt_e2m1x8(v) : 0u;
-            }
             uint8_t* crow = p.codes + (row0 + rA) * (p.cols / 2) + c0 / 2 + 8 * j;
-            *reinterpret_cast<uint2*>(crow) = make_uint2(code[0], code[1]);
-            *reinterpret_cast<uint2*>(crow + 8 * (p.cols / 2)) = make_uint2(code[2], code[3]);
-            // the four blocks' scales, gathered from lanes l8, l8 + 8, l8 + 16, l8 + 24
-            const uint32_t sb4 = __shfl_sync(0xffffffffu, sb, l8) | (__shfl_sync(0xffffffffu, sb, l8 + 8) << 8) |
-                                 (__shfl_sync(0xffffffffu, sb, l8 + 16) << 16) |
-                                 (__shfl_sync(0xffffffffu, sb, l8 + 24) << 24);
-            if (lane == 0)
-                *reinterpret_cast<uint32_t*>(p.scales + (row0 / 16 + qw) * cbs + c0 / 16) = sb4;
-            if (p.sf_mma && j == 0) {
-                uint8_t* atom = p.sf_mma + (static_cast<int64_t>(band) * atoms_per_band + c0 / 64) * 512;
-                *reinterpret_cast<uint32_t*>(atom + 16 * (rA % 32) + 4 * (rA / 32)) = sb4;
-                *reinterpret_cast<uint32_t*>(atom + 16 * (rB % 32) + 4 * (rB / 32)) = sb4;
+            // max |x| on the bf16 bit patterns (sign cleared: integer order = numeric order)
+            auto wmax = [](const uint4& u) {
+                return __vmaxu2(__vmaxu2(u.x & 0x7FFF7FFFu, u.y & 0x7FFF7FFFu),
+                                __vmaxu2(u.z & 0x7FFF7FFFu, u.w & 0x7FFF7FFFu));
+            };
+            auto half_max = [](uint32_t m2) { return max(m2 & 0xFFFFu, m2 >> 16); };
+            auto scale_of = [&](uint32_t amb) -> uint32_t {  // amb: bf16 bits of the block max
+                return degenerate ? 0u : cvt_ue4m3(__fmul_rn(div6_bf16(__uint_as_float(amb << 16)), g));
+            };
+            auto encode8 = [&](const uint4& u, float inv) {
+                float v[8];
+                v[0] = __fmul_rn(bf16lo_to_f32(u.x), inv); v[1] = __fmul_rn(bf16hi_to_f32(u.x), inv);
+                v[2] = __fmul_rn(bf16lo_to_f32(u.y), inv); v[3] = __fmul_rn(bf16hi_to_f32(u.y), inv);
+                v[4] = __fmul_rn(bf16lo_to_f32(u.z), inv); v[5] = __fmul_rn(bf16hi_to_f32(u.z), inv);
+                v[6] = __fmul_rn(bf16lo_to_f32(u.w), inv); v[7] = __fmul_rn(bf16hi_to_f32(u.w), inv);
+                return cvt_e2m1x8(v);
+            };
+            // the four blocks' scale bytes of this lane's rows, gathered from the lanes with
+            // the same l8: l8, l8 + 8, l8 + 16, l8 + 24 hold blocks 0..3
+            auto gather4 = [&](uint32_t sbv) {
+                return __shfl_sync(0xffffffffu, sbv, l8) | (__shfl_sync(0xffffffffu, sbv, l8 + 8) << 8) |
+                       (__shfl_sync(0xffffffffu, sbv, l8 + 16) << 16) |
+                       (__shfl_sync(0xffffffffu, sbv, l8 + 24) << 24);
+            };
+            uint8_t* atom = p.sf_mma ? p.sf_mma + (static_cast<int64_t>(band) * atoms_per_band + c0 / 64) * 512
+                                     : nullptr;
+            if constexpr (GRAN == 16) {
+                // 16x16 block: the 8 lanes of block j hold its 16 rows
+                uint32_t amb = half_max(__vmaxu2(__vmaxu2(wmax(w[0]), wmax(w[1])), __vmaxu2(wmax(w[2]), wmax(w[3]))));
+                amb = max(amb, __shfl_xor_sync(0xffffffffu, amb, 1));
+                amb = max(amb, __shfl_xor_sync(0xffffffffu, amb, 2));
+                amb = max(amb, __shfl_xor_sync(0xffffffffu, amb, 4));
+                const uint32_t sb = scale_of(amb);
+                const float inv = inv_lut[sb];
+                uint32_t code[4];  // row rA: words 0, 1; row rB: words 2, 3
+#pragma unroll
+                for (int q2 = 0; q2 < 4; ++q2) code[q2] = sb ? encode8(w[q2], inv) : 0u;
+                *reinterpret_cast<uint2*>(crow) = make_uint2(code[0], code[1]);
+                *reinterpret_cast<uint2*>(crow + 8 * (p.cols / 2)) = make_uint2(code[2], code[3]);
+                const uint32_t sb4 = gather4(sb);
+                if (lane == 0)
+                    *reinterpret_cast<uint32_t*>(p.scales + (row0 / 16 + qw) * cbs + c0 / 16) = sb4;
+                if (atom && j == 0) {
+                    *reinterpret_cast<uint32_t*>(atom + 16 * (rA % 32) + 4 * (rA / 32)) = sb4;
+                    *reinterpret_cast<uint32_t*>(atom + 16 * (rB % 32) + 4 * (rB / 32)) = sb4;
+                }
+            } else {
+                // group-wise 1x16: each of the lane's two rows is a group of its own
+                const uint32_t sbA = scale_of(half_max(__vmaxu2(wmax(w[0]), wmax(w[1]))));
+                const uint32_t sbB = scale_of(half_max(__vmaxu2(wmax(w[2]), wmax(w[3]))));
+                const float invA = inv_lut[sbA], invB = inv_lut[sbB];
+                const uint32_t c0w = sbA ? encode8(w[0], invA) : 0u, c1w = sbA ? encode8(w[1], invA) : 0u;
+                const uint32_t c2w = sbB ? encode8(w[2], invB) : 0u, c3w = sbB ? encode8(w[3], invB) : 0u;
+                *reinterpret_cast<uint2*>(crow) = make_uint2(c0w, c1w);
+                *reinterpret_cast<uint2*>(crow + 8 * (p.cols / 2)) = make_uint2(c2w, c3w);
+                const uint32_t sb4A = gather4(sbA), sb4B = gather4(sbB);
+                if (j == 0) {
+                    *reinterpret_cast<uint32_t*>(p.scales + (row0 + rA) * cbs + c0 / 16) = sb4A;
+                    *reinterpret_cast<uint32_t*>(p.scales + (row0 + rB) * cbs + c0 / 16) = sb4B;
+                    if (atom) {
+                        *reinterpret_cast<uint32_t*>(atom + 16 * (rA % 32) + 4 * (rA / 32)) = sb4A;
+                        *reinterpret_cast<uint32_t*>(atom + 16 * (rB % 32) + 4 * (rB / 32)) = sb4B;
+                    }
+                }
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(S + s));
@@ -288,14 +318,20 @@ size_t quant_down_smem_bytes(int Rp) { return static_cast<size_t>(qf::layout_for
 cudaError_t launch_quant_down(const CUtensorMap& tmX, const CUtensorMap& tmW, const QuantDownArgs& a,
                               int splits, cudaStream_t stream) {
     const qf::Layout L = qf::layout_for(a.Rp);
-    // the opt-in limit is raised once to the device maximum (no per-launch host calls)
-    static const cudaError_t attr = cudaFuncSetAttribute(
-        qf::quant_down_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 232448);
-    if (attr != cudaSuccess) return attr;
+    // the opt-in limits are raised once to the device maximum (no per-launch host calls)
+    static const cudaError_t attr16 = cudaFuncSetAttribute(
+        qf::quant_down_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize, 232448);
+    static const cudaError_t attr1 = cudaFuncSetAttribute(
+        qf::quant_down_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, 232448);
+    if (attr16 != cudaSuccess) return attr16;
+    if (attr1 != cudaSuccess) return attr1;
     dim3 grid(static_cast<unsigned>(a.rows / 128), static_cast<unsigned>(splits));
     before_launch(K_QUANT, stream);
-    const cudaError_t le = launch_k(qf::quant_down_kernel, dim3(grid), dim3(qf::THREADS),
-                                    L.smem_bytes, stream, tmX, tmW, a);
+    const cudaError_t le =
+        a.block_rows == 1 ? launch_k(qf::quant_down_kernel<1>, dim3(grid), dim3(qf::THREADS), L.smem_bytes, stream,
+                                     tmX, tmW, a)
+                          : launch_k(qf::quant_down_kernel<16>, dim3(grid), dim3(qf::THREADS), L.smem_bytes,
+                                     stream, tmX, tmW, a);
     if (le != cudaSuccess) return le;
     after_launch(K_QUANT, stream);
     return cudaGetLastError();

@@ -56,6 +56,12 @@ EXPORTS = {
     "fourtune_linear_fwd": ([ctypes.POINTER(FtLinear), ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p,
                              ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t,
                              ctypes.c_void_p], ctypes.c_int),
+    "fourtune_quantize_1x16": ([ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, ctypes.c_void_p,
+                                ctypes.POINTER(FtFp4), ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p],
+                               ctypes.c_int),
+    "fourtune_linear_fwd_1x16": ([ctypes.POINTER(FtLinear), ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p,
+                                  ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t,
+                                  ctypes.c_void_p], ctypes.c_int),
     "fourtune_linear_fwd_gelu": ([ctypes.POINTER(FtLinear), ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p,
                                   ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
                                   ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p], ctypes.c_int),
@@ -135,10 +141,10 @@ class QuantizedMatrix:
     cols: int
 
     @staticmethod
-    def empty(rows: int, cols: int, device, with_sf: bool = True) -> "QuantizedMatrix":
+    def empty(rows: int, cols: int, device, with_sf: bool = True, block_rows: int = 16) -> "QuantizedMatrix":
         return QuantizedMatrix(
             codes=torch.empty(rows, cols // 2, dtype=torch.uint8, device=device),
-            scales=torch.empty(rows // 16, cols // 16, dtype=torch.uint8, device=device),
+            scales=torch.empty(rows // block_rows, cols // 16, dtype=torch.uint8, device=device),
             sf_mma=torch.empty(rows * cols // 16, dtype=torch.uint8, device=device) if with_sf else None,
             g=torch.empty(1, dtype=torch.float32, device=device), rows=rows, cols=cols)
 
@@ -171,6 +177,22 @@ def quantize_block16(x: torch.Tensor, amax: Optional[torch.Tensor] = None, with_
                                          _p(ws), nws, _stream(stream))
     _check("fourtune_quantize_block16", st)
     return q, qt, down_out
+
+
+def quantize_1x16(x: torch.Tensor, amax: Optional[torch.Tensor] = None, with_sf: bool = True, stream=None):
+    """Q(x) in group-wise 1x16 blocks (scales [rows, cols/16]) on the GPU; bf16 x."""
+    _require_cuda(x, amax)
+    if x.dim() != 2 or x.stride(1) != 1 or x.dtype != torch.bfloat16:
+        raise ValueError("x must be a row-major 2-D bf16 tensor")
+    rows, cols = x.shape
+    q = QuantizedMatrix.empty(rows, cols, x.device, with_sf=with_sf, block_rows=1)
+    nws = lib().fourtune_quantize_workspace_bytes(rows, cols, 0)
+    ws = torch.zeros(nws, dtype=torch.uint8, device=x.device)
+    qs = q.c_struct()
+    st = lib().fourtune_quantize_1x16(_p(x), rows, cols, x.stride(0), _p(amax), ctypes.byref(qs), _p(ws), nws,
+                                      _stream(stream))
+    _check("fourtune_quantize_1x16", st)
+    return q
 
 
 @dataclasses.dataclass
@@ -248,6 +270,23 @@ def linear_fwd(w: LinearWeights, x: torch.Tensor, ws: Workspace, y: Optional[tor
     st = lib().fourtune_linear_fwd(ctypes.byref(s), _p(x), M, _p(amax), _p(y), _p(t_saved), _p(ws.buf),
                                    ws.nbytes, _stream(stream))
     _check("fourtune_linear_fwd", st)
+    return y, t_saved
+
+
+def linear_fwd_1x16(w: LinearWeights, x: torch.Tensor, ws: Workspace, y: Optional[torch.Tensor] = None,
+                    t_saved: Optional[torch.Tensor] = None, amax: Optional[torch.Tensor] = None, stream=None):
+    """Eq. (2) with X quantized group-wise 1x16 (forward only).  Returns (Y, T)."""
+    _require_cuda(x)
+    M = x.shape[0]
+    if y is None:
+        y = torch.empty(M, w.N, dtype=torch.bfloat16, device=x.device)
+    R = w.r_s + w.r
+    if t_saved is None:
+        t_saved = torch.empty(M, max(R, 1), dtype=torch.float32, device=x.device)
+    s = w.c_struct()
+    st = lib().fourtune_linear_fwd_1x16(ctypes.byref(s), _p(x), M, _p(amax), _p(y), _p(t_saved), _p(ws.buf),
+                                        ws.nbytes, _stream(stream))
+    _check("fourtune_linear_fwd_1x16", st)
     return y, t_saved
 
 

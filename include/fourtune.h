@@ -175,6 +175,21 @@ ft_status fourtune_quantize_block16_noalloc(const void* x_dev, int32_t x_dtype, 
                                             float* down_out_dev, const ft_fp4* out,
                                             const ft_fp4* out_t, void* stream);
 
+/*
+ * Q(x) in group-wise 1x16 blocks: one UE4M3 scale per row and 16 consecutive columns, the
+ * granularity FourTune compares its 16x16 blocks with (section 4.3, "Impact of
+ * Quantization Granularity", Table 5).  Same two-level scaling and the same arithmetic per
+ * element as fourtune_quantize_block16; forward use only (1x16 blocks do not transpose).
+ *   x_dev : bf16 [rows, cols], row stride ld elements.
+ *   out   : codes [rows, cols/2], scales [rows, cols/16] (one byte per group), g, and
+ *           sf_mma (optional; the tensor-core layout, per row and 16 columns as always).
+ * Shapes: rows % 128 == 0, cols % 64 == 0, ld % 8 == 0, else FT_ERR_SHAPE.  Workspace:
+ * fourtune_quantize_workspace_bytes(rows, cols, 0).
+ */
+ft_status fourtune_quantize_1x16(const void* x_dev, int64_t rows, int64_t cols, int64_t ld,
+                                 const float* amax_or_null, const ft_fp4* out, void* ws, size_t ws_bytes,
+                                 void* stream);
+
 /* Workspace bytes for fourtune_linear_fwd / fourtune_linear_bwd with M tokens. */
 size_t fourtune_linear_workspace_bytes(const ft_linear* layer, int64_t M);
 
@@ -189,6 +204,15 @@ size_t fourtune_linear_workspace_bytes(const ft_linear* layer, int64_t M);
 ft_status fourtune_linear_fwd(const ft_linear* layer, const void* x_dev, int64_t M,
                               const float* amax_or_null, void* y_dev, float* t_saved_dev,
                               void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * fourtune_linear_fwd with X quantized group-wise 1x16 (fourtune_quantize_1x16) instead
+ * of in 16x16 blocks: the Table 5 comparison, for forward-only use.  Arguments, shapes and
+ * workspace as fourtune_linear_fwd.
+ */
+ft_status fourtune_linear_fwd_1x16(const ft_linear* layer, const void* x_dev, int64_t M,
+                                   const float* amax_or_null, void* y_dev, float* t_saved_dev, void* ws,
+                                   size_t ws_bytes, void* stream);
 
 /*
  * Forward pass with GELU (tanh form) fused into the 4-bit GEMM's epilogue, for the first
