@@ -513,10 +513,13 @@ def main():
     def fwd_kernels():
         ft.linear_fwd(w, x, ws, y=y, t_saved=t)
 
+    def fwd_1x16_kernels():  # X quantized group-wise 1x16 (the Table 5 comparison, forward only)
+        ft.linear_fwd_1x16(w, x, ws, y=y, t_saved=t)
+
     def bwd_kernels():
         ft.linear_bwd(w, x, t, dy, ws, dx=dx, da=da, db=db)
 
-    graph = graph_k = graph_f = graph_b = None
+    graph = graph_k = graph_f = graph_b = graph_f1 = None
     launches_per_step = None
     if args.graph:
         # One step (forward + backward: all of the library's kernels) captured once as a
@@ -534,13 +537,16 @@ def main():
         with torch.cuda.graph(graph_k):
             one_step_with_events()
         # forward alone and backward alone, for the per-pass figures
-        graph_f, graph_b = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+        graph_f, graph_b, graph_f1 = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
         with torch.cuda.graph(graph_f):
             fwd_kernels()
         with torch.cuda.graph(graph_b):
             bwd_kernels()
+        fwd_1x16_kernels()
+        with torch.cuda.graph(graph_f1):
+            fwd_1x16_kernels()
         for _ in range(args.warmup):
-            for g_ in (graph, graph_k, graph_f, graph_b):
+            for g_ in (graph, graph_k, graph_f, graph_b, graph_f1):
                 flush.zero_()
                 g_.replay()
         torch.cuda.synchronize()
@@ -585,8 +591,9 @@ def main():
         torch.cuda.synchronize()
         ms_per_step_events = sum(ev_ks[i].elapsed_time(ev_ke[i]) for i in range(Kst)) / Kst
         # per-pass pass: the forward alone, then the backward alone, as many steps each
-        pass_ms = {"fwd": [], "bwd": []}
-        for name, g_, fn in (("fwd", graph_f, fwd_kernels), ("bwd", graph_b, bwd_kernels)):
+        pass_ms = {"fwd": [], "bwd": [], "fwd_1x16": []}
+        for name, g_, fn in (("fwd", graph_f, fwd_kernels), ("bwd", graph_b, bwd_kernels),
+                             ("fwd_1x16", graph_f1, fwd_1x16_kernels)):
             for i in range(Kst):
                 flush.zero_()
                 ev_ks[i].record()
@@ -680,6 +687,7 @@ def main():
                           "frac_with_amax": qa_gbs / hbm, "avg_launch_ms": statistics.mean(quant_ms)},
             "per_pass": {"fwd_ms": fwd_ms, "fwd_tflops": fl_f / (fwd_ms * 1e-3) / 1e12,
                          "bwd_ms": bwd_ms, "bwd_tflops": fl_b / (bwd_ms * 1e-3) / 1e12,
+                         "fwd_1x16_ms": statistics.median(pass_ms["fwd_1x16"]),
                          "timing": f"median of {Kst} replays of a forward-only / backward-only graph"},
             "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
             "gpu_launches": launches,
