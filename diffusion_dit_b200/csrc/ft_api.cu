@@ -111,7 +111,7 @@ size_t max_splits(int64_t units) {
 // Workspace of the layer calls.  Regions are 256-byte aligned.
 struct LinearWs {
     size_t status, scal, qx_codes, qx_scales, qx_sf, dn, upcat, tcat, partial;
-    size_t qg_codes, qg_scales, qg_sf, upt, dntcat, ucat, vcat, ucat_lora, gpartial, total;
+    size_t qg_codes, qg_scales, qg_sf, upt, dntcat, ucat, vcat, ucat_lora, gpartial_b, gpartial_a, total;
 };
 
 // Width of the adapter-gradient operand [hi, lo, 0]: 2r rounded up to 64.
@@ -144,7 +144,8 @@ LinearWs linear_ws(int64_t M, int64_t N, int64_t K, int R, int r) {
     w.ucat = take(static_cast<size_t>(M) * KL * 2);
     w.vcat = take(static_cast<size_t>(M) * lora_width(r) * 2);
     w.ucat_lora = take(static_cast<size_t>(M) * lora_width(r) * 2);
-    w.gpartial = take(std::max(max_splits(N / 128) * N, max_splits(K / 128) * K) * lora_width(r) * 4);
+    w.gpartial_b = take(max_splits(N / 128) * N * lora_width(r) * 4);  // dB's split partials
+    w.gpartial_a = take(max_splits(K / 128) * K * lora_width(r) * 4);  // dA's
     w.total = o;
     return w;
 }
@@ -594,13 +595,13 @@ ft_status linear_bwd_impl(const ft_linear* L, const void* x_dev, const float* t_
     // reads every element of G once and also takes max |G| (into the slot the factor
     // kernel cleared), so Q(G) needs no separate pass over G; G is then still in L2.
     const int NBW = lora_width(L->r);
-    float* gpart = reinterpret_cast<float*>(W + w.gpartial);
     ft::LoraGradArgs g{};
     g.NBW = NBW;
     g.tmem_cols = tmem_cols_for(NBW);
-    g.partial = gpart;
     g.status = status;
     const float* amax_g = amax_or_null;
+    // dB's split sum waits and runs in one launch with dA's (the two jobs of the finalize)
+    ft::LoraFinalizeJob fin_b{}, fin_a{};
     if (L->r > 0) {
         CUtensorMap tP, tV;
         FT_TRY(make_tmap(&tV, W + w.vcat, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, NBW, M, NBW * 2, 64, 64));
@@ -608,13 +609,14 @@ ft_status linear_bwd_impl(const ft_linear* L, const void* x_dev, const float* t_
         const int sp = ft::lora_grad_splits(M, N, dev.num_sms);
         g.F = N;
         g.tokens_per_split = static_cast<int>(M / sp);
+        g.partial = reinterpret_cast<float*>(W + w.gpartial_b);
         if (!amax_or_null) {
             g.amax_out = reinterpret_cast<unsigned*>(scal + SC_AMAX_G);
             amax_g = scal + SC_AMAX_G;
         }
         FT_CUDA(ft::launch_lora_grad(tP, tV, g, sp, ft::K_LORA_DB, st));
         g.amax_out = nullptr;
-        FT_CUDA(ft::launch_lora_grad_finalize(gpart, sp, N, NBW, L->r, L->lora_scale, false, db_dev, st));
+        fin_b = ft::LoraFinalizeJob{g.partial, sp, static_cast<int>(N), NBW, L->r, L->lora_scale, false, db_dev};
     }
     int splits = 1;
     FT_TRY(quantize_operand(dy_dev, M, N, N, amax_g, scal + SC_AMAX_G, R > 0, W + w.qg_codes, W + w.qg_scales,
@@ -647,8 +649,10 @@ ft_status linear_bwd_impl(const ft_linear* L, const void* x_dev, const float* t_
         const int sp = ft::lora_grad_splits(M, K, dev.num_sms);
         g.F = K;
         g.tokens_per_split = static_cast<int>(M / sp);
+        g.partial = reinterpret_cast<float*>(W + w.gpartial_a);
         FT_CUDA(ft::launch_lora_grad(tP, tV, g, sp, ft::K_LORA_DA, st));
-        FT_CUDA(ft::launch_lora_grad_finalize(gpart, sp, K, NBW, L->r, L->lora_scale, true, da_dev, st));
+        fin_a = ft::LoraFinalizeJob{g.partial, sp, static_cast<int>(K), NBW, L->r, L->lora_scale, true, da_dev};
+        FT_CUDA(ft::launch_lora_grad_finalize(fin_a, fin_b, st));
     }
     // The dX GEMM goes last: the GEMM's operand and output traffic would evict G from L2.
     FT_TRY(run_gemm(W + w.qg_codes, W + w.qg_sf, scal + SC_G_G, L->qr_t, bf(W + w.ucat), bf(W + w.dntcat), KL,

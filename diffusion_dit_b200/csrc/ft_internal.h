@@ -167,7 +167,15 @@ struct LoraGradArgs {
 int lora_grad_splits(int64_t M, int64_t F, int num_sms);
 cudaError_t launch_lora_grad(const CUtensorMap& tmP, const CUtensorMap& tmV, const LoraGradArgs& a, int splits,
                              int kind, cudaStream_t stream);
-cudaError_t launch_lora_grad_finalize(const float* partial, int splits, int64_t F, int NBW, int r, float s,
-                                      bool transpose_out, float* out, cudaStream_t stream);
+// out = s * sum over the splits (in order) of (D[f][j] + D[f][r + j]); out[f][j], or out[j][f]
+// with transpose_out.  One launch runs up to two such jobs (j1.out == nullptr: none).
+struct LoraFinalizeJob {
+    const float* partial;    // [splits, F, NBW]
+    int splits, F, NBW, r;
+    float s;
+    bool transpose_out;
+    float* out;
+};
+cudaError_t launch_lora_grad_finalize(const LoraFinalizeJob& j0, const LoraFinalizeJob& j1, cudaStream_t stream);
 
 }  // namespace ft

@@ -188,30 +188,32 @@ __global__ void __launch_bounds__(THREADS, 1)
 }
 
 // out = s * sum_split (D[f][j] + D[f][r + j]); transposed (out[j][f]) for dA.
-__global__ void lora_grad_finalize_kernel(const float* __restrict__ partial, int splits, int F, int NBW, int r,
-                                          float s, bool transpose_out, float* __restrict__ out) {
+__global__ void lora_grad_finalize_kernel(const LoraFinalizeJob j0, const LoraFinalizeJob j1) {
     pdl_trigger();
     pdl_wait();
-    const int total = F * r;
+    const int total0 = j0.F * j0.r;
+    const int total = total0 + (j1.out ? j1.F * j1.r : 0);
     for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < total; i += gridDim.x * blockDim.x) {
+        const LoraFinalizeJob& jb = i < total0 ? j0 : j1;
+        const int ii = i < total0 ? i : i - total0;
         int f, j;
-        if (transpose_out) {  // consecutive threads walk f: coalesced stores into out[j][f]
-            j = i / F;
-            f = i - j * F;
+        if (jb.transpose_out) {  // consecutive threads walk f: coalesced stores into out[j][f]
+            j = ii / jb.F;
+            f = ii - j * jb.F;
         } else {
-            f = i / r;
-            j = i - f * r;
+            f = ii / jb.r;
+            j = ii - f * jb.r;
         }
         float v = 0.0f;
-        for (int sp = 0; sp < splits; ++sp) {
-            const float* d = partial + (sp * F + f) * NBW;
-            v += d[j] + d[r + j];
+        for (int sp = 0; sp < jb.splits; ++sp) {
+            const float* d = jb.partial + (sp * jb.F + f) * jb.NBW;
+            v += d[j] + d[jb.r + j];
         }
-        v *= s;
-        if (transpose_out)
-            out[j * F + f] = v;
+        v *= jb.s;
+        if (jb.transpose_out)
+            jb.out[j * jb.F + f] = v;
         else
-            out[f * r + j] = v;
+            jb.out[f * jb.r + j] = v;
     }
 }
 
@@ -245,14 +247,12 @@ cudaError_t launch_lora_grad(const CUtensorMap& tmP, const CUtensorMap& tmV, con
     return cudaGetLastError();
 }
 
-cudaError_t launch_lora_grad_finalize(const float* partial, int splits, int64_t F, int NBW, int r, float s,
-                                      bool transpose_out, float* out, cudaStream_t stream) {
-    int64_t g = (F * r + 255) / 256;
+cudaError_t launch_lora_grad_finalize(const LoraFinalizeJob& j0, const LoraFinalizeJob& j1, cudaStream_t stream) {
+    int64_t g = (static_cast<int64_t>(j0.F) * j0.r + (j1.out ? static_cast<int64_t>(j1.F) * j1.r : 0) + 255) / 256;
     if (g > 148 * 8) g = 148 * 8;
     before_launch(K_OTHER, stream);
-    const cudaError_t le = launch_k(lg::lora_grad_finalize_kernel, dim3(static_cast<unsigned>(g)),
-                                    dim3(256), 0, stream, partial, splits, static_cast<int>(F), NBW,
-                                    r, s, transpose_out, out);
+    const cudaError_t le = launch_k(lg::lora_grad_finalize_kernel, dim3(static_cast<unsigned>(g)), dim3(256), 0,
+                                    stream, j0, j1);
     if (le != cudaSuccess) return le;
     after_launch(K_OTHER, stream);
     return cudaGetLastError();
