@@ -84,7 +84,8 @@ ft_status cuda_status(cudaError_t e) { return e == cudaSuccess ? FT_OK : FT_ERR_
     } while (0)
 #define FT_CUDA(expr) FT_TRY(cuda_status(expr))
 
-int low_rank_width(int R) { return R == 0 ? 0 : static_cast<int>(align_up(2 * static_cast<size_t>(R), 64)); }
+// Width of the GEMMs' low-rank operands [hi, lo]: 2R rounded up to the bf16 MMA's K step.
+int low_rank_width(int R) { return R == 0 ? 0 : static_cast<int>(align_up(2 * static_cast<size_t>(R), 16)); }
 
 // Width of the tensor-core down-projection: the rank rounded up to the MMA's N step.
 int padded_rank(int R) { return R == 0 ? 0 : static_cast<int>(align_up(static_cast<size_t>(R), 16)); }

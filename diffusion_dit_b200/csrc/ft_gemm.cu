@@ -93,7 +93,8 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int NB = p.N / BN;
     const int num_tiles = MB * NB;
     const int KT = p.K / 256;      // fp4 stages
-    const int KLS = p.KL / 64;     // low-rank stages
+    const int KLS = (p.KL + 63) / 64;  // low-rank stages (the last one may be partly past KL:
+                                       // TMA fills those columns with zeros, no MMA reads them)
     const int k64 = p.K / 64;      // scale atoms per 128-row band
 
     if (threadIdx.x == 0) {
@@ -217,8 +218,8 @@ __global__ void __launch_bounds__(THREADS, 1)
                     const uint32_t st = sm.stage(s);
                     const uint64_t ad = sdesc_kmajor_sw128(st);
                     const uint64_t bd = sdesc_kmajor_sw128(st + OFF_B);
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) mma_bf16(acc, ad + 2 * i, bd + 2 * i, idesc16, 1);
+                    const int nk16 = min(4, (p.KL - 64 * kl) / 16);  // K=16 steps inside KL
+                    for (int i = 0; i < nk16; ++i) mma_bf16(acc, ad + 2 * i, bd + 2 * i, idesc16, 1);
                     tc_commit(sm.bar(BAR_EMPTY(s)));
                 }
                 if (!ok) break;

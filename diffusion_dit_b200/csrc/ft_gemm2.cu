@@ -102,7 +102,8 @@ __global__ void __launch_bounds__(threads(EPI), 1)
     const int NB = p.N / BN;
     const int num_tiles = MB2 * NB;
     const int KT = p.K / 256;
-    const int KLS = p.KL / 64;
+    const int KLS = (p.KL + 63) / 64;  // low-rank stages (the last one may be partly past KL:
+                                       // TMA fills those columns with zeros, no MMA reads them)
     const int k64 = p.K / 64;
 
     if (threadIdx.x == 0) {
@@ -208,8 +209,8 @@ __global__ void __launch_bounds__(threads(EPI), 1)
                             mma_fp4_block16_pair(tmem + COL_ACC, ad + 2 * i, bd + 2 * i, idesc4, sfa_t + 4 * i,
                                                  sfb_t + 8 * i, (j | i) != 0);
                     } else {
-#pragma unroll
-                        for (int i = 0; i < 4; ++i)
+                        const int nk16 = min(4, (p.KL - 64 * (j - KT)) / 16);  // K=16 steps inside KL
+                        for (int i = 0; i < nk16; ++i)
                             mma_bf16_pair(tmem + COL_ACC, ad + 2 * i, bd + 2 * i, idesc16, 1);
                     }
                     tc_commit_pair(bar(BAR_EMPTY(s)));

@@ -47,7 +47,7 @@ struct GemmFp4Args {
     __nv_bfloat16* out;     // [M, ldo]
     int64_t ldo;
     int M, N, K;            // K: reduction length in elements (multiple of 256)
-    int KL;                 // low-rank reduction length in bf16 elements (multiple of 64), 0 = none
+    int KL;                 // low-rank reduction length in bf16 elements (multiple of 16), 0 = none
     int* status;            // device status word
     // optional GELU epilogue: also store act = bf16(gelu_tanh(out)) (same layout as out,
     // through tmAct) and take max |act| into *act_amax (float bits, cleared beforehand)
