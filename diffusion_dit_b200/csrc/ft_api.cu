@@ -207,7 +207,7 @@ ft_status quantize_operand(const void* x, int64_t rows, int64_t cols, int64_t ld
     a.cols = cols;
     a.cols_per_split = static_cast<int>(cols / s);
     a.Rp = Rp;
-    a.tmem_cols = tmem_cols_for(Rp);
+    a.tmem_cols = ft::quant_down_tmem_cols(Rp);
     a.amax = amax;
     a.codes = codes;
     a.scales = scales;

@@ -97,7 +97,7 @@ struct QuantDownArgs {
     int64_t rows, cols;      // input [rows, cols]; rows % 128 == 0, cols % 64 == 0
     int cols_per_split;      // columns per CTA slice (multiple of 64)
     int Rp;                  // down-projection width (multiple of 16, <= 256; 0 = none)
-    uint32_t tmem_cols;      // TMEM columns to allocate (power of two >= max(32, Rp))
+    uint32_t tmem_cols;      // TMEM columns to allocate: quant_down_tmem_cols(Rp)
     const float* amax;       // tensor max used for g
     uint8_t* codes;          // [rows, cols/2]
     uint8_t* scales;         // [rows/16, cols/16]
@@ -108,6 +108,7 @@ struct QuantDownArgs {
     int block_rows;          // 16: 16x16 blocks, scales [rows/16, cols/16]; 1: 1x16 groups, [rows, cols/16]
 };
 int quant_down_splits(int64_t rows, int64_t cols, int num_sms);
+uint32_t quant_down_tmem_cols(int Rp);  // room for the kernel's accumulators of Rp columns
 size_t quant_down_smem_bytes(int Rp);
 cudaError_t launch_quant_down(const CUtensorMap& tmX, const CUtensorMap& tmW, const QuantDownArgs& a,
                               int splits, cudaStream_t stream);

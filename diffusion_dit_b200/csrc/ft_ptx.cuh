@@ -464,6 +464,22 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     return out;
 }
 
+// Two fp32 products rounded to nearest in one packed instruction: (a * s, b * s).
+__device__ __forceinline__ void mul2_rn(float a, float b, float s, float& ra, float& rb) {
+    asm("{\n\t.reg .b64 x, y, z;\n\tmov.b64 x, {%2, %3};\n\tmov.b64 y, {%4, %4};\n\t"
+        "mul.rn.f32x2 z, x, y;\n\tmov.b64 {%0, %1}, z;\n\t}"
+        : "=f"(ra), "=f"(rb)
+        : "f"(a), "f"(b), "f"(s));
+}
+
+// Per 16-bit half: a bf16 whose magnitude is max(|a|, |b|) (sign bit meaningless; NaN
+// inputs are outside the domain: the other operand wins).
+__device__ __forceinline__ uint32_t absmax_bf16x2(uint32_t a, uint32_t b) {
+    uint32_t r;
+    asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
+}
+
 __device__ __forceinline__ float bf16lo_to_f32(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16hi_to_f32(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 

@@ -6,18 +6,19 @@
 // rounded up to 16, extra rows zero) one CTA takes a 128-row band and a slice of the
 // columns.  Each 128 x 64 tile arrives by TMA (128-byte swizzle) into a shared-memory
 // ring and is consumed twice:
-//   * the MMA warp multiplies it with the matching W tile on the tensor cores
-//     (tcgen05.mma kind::f16, accumulator [128 x Rp] fp32 in TMEM), giving this CTA's
-//     partial of T = X W^T;
-//   * a set of eight quantizer warps (one per 16-row block-row) reads the same tile
-//     from shared memory and emits the E2M1 codes, the compact block scales and the
-//     tensor-core scale layout (same arithmetic, bit for bit, as quant_block16_kernel
-//     in ft_quant.cu).  Two such sets take the stages in turn: a warp's work on one
-//     stage is a chain of dependent steps (loads, shuffles, scale, convert, stores), so
-//     two stages in flight double the quantizer's throughput per SM.
-// A stage is released when the MMA has finished reading it (tcgen05.commit) and the
-// eight warps of its set have arrived.  At the end four warps drain the accumulator
-// into partials[split][row][Rp]; ft_lowrank.cu sums the splits in a fixed order.
+//   * an MMA issuer multiplies it with the matching W tile on the tensor cores
+//     (tcgen05.mma kind::f16, [128 x Rp] fp32 in TMEM), giving a partial of T = X W^T.
+//     Two issuers in separate warps take alternate stages, each into its own
+//     accumulator: one thread issues a 128 x Rp x 16 MMA no faster than a 128 x 128 x 16
+//     one, so a single issuer would pace the ring;
+//   * a set of four quantizer warps (two 16-row block-rows each) copies the tile out of
+//     shared memory into registers, releases the stage, and emits the E2M1 codes, the
+//     compact block scales and the tensor-core scale layout (same arithmetic, bit for
+//     bit, as quant_block16_kernel in ft_quant.cu).  Four sets take the stages in turn.
+// A stage is released when its MMAs have finished reading it (tcgen05.commit) and the
+// four warps of its set hold its data.  At the end four warps add the two accumulators
+// (in a fixed order) into partials[split][row][Rp]; ft_lowrank.cu sums the splits in a
+// fixed order.
 #include "ft_internal.h"
 #include "ft_ptx.cuh"
 
@@ -28,12 +29,24 @@ constexpr int BM = 128;
 constexpr int BKE = 64;                 // bf16 columns per stage (one 128-byte row)
 constexpr int X_BYTES = BM * 128;       // 16 KB
 #ifndef FT_QUANT_SETS
-#define FT_QUANT_SETS 2
+#define FT_QUANT_SETS 4
 #endif
-constexpr int NQ_SET = 8;                  // quantizer warps per set: one per 16-row block-row
-constexpr int NSETS = FT_QUANT_SETS;       // sets take the stages in turn (k % NSETS)
+#ifndef FT_QUANT_SET_WARPS
+#define FT_QUANT_SET_WARPS 4
+#endif
+constexpr int NQ_SET = FT_QUANT_SET_WARPS;  // quantizer warps per set (one set per stage)
+constexpr int BR = 8 / NQ_SET;              // 16-row block-rows per quantizer warp
+constexpr int NSETS = FT_QUANT_SETS;        // sets take the stages in turn (k % NSETS)
 constexpr int NQ = NQ_SET * NSETS;         // quantizer warps
-constexpr int THREADS = 32 * (2 + NQ);     // producer, MMA, quantizers
+#ifndef FT_QUANT_MMA_WARPS
+#define FT_QUANT_MMA_WARPS 2
+#endif
+// A bf16 MMA of 128 x Rp x 16 costs the issuing thread about as much as one of 128 x 128 x 16,
+// so the down-projection's four MMAs per stage are issued by MW threads in separate warps
+// (stages alternate between them), each into its own accumulator; the epilogue adds them.
+constexpr int MW = FT_QUANT_MMA_WARPS;
+constexpr int QW0 = 1 + MW;                 // first quantizer warp
+constexpr int THREADS = 32 * (QW0 + NQ);    // producer, MMA issuers, quantizers
 constexpr int MAX_STAGES = 8;
 constexpr int BAR_BYTES = 768;           // barriers, TMEM slot, abort flag, inv table at +160
 
@@ -46,9 +59,14 @@ struct Layout {
 __host__ __device__ inline Layout layout_for(int Rp) {
     Layout L;
     L.stage_bytes = X_BYTES + Rp * 128;
+    // A stage is always consumed by the same quantizer set and the same MMA issuer (the
+    // stage count is a multiple of both): each then waits on a stage's phases one after
+    // another, so a parity wait cannot be satisfied by the phase before the one it wants.
+    constexpr int unit = (NSETS % MW == 0) ? NSETS : (MW % NSETS == 0 ? MW : NSETS * MW);
     int s = (200 * 1024) / L.stage_bytes;
-    if (s > 6) s = 6;
-    if (s < 2) s = 2;
+    if (s > MAX_STAGES) s = MAX_STAGES;
+    s -= s % unit;
+    if (s < unit) s = unit;
     L.stages = s;
     L.smem_bytes = s * L.stage_bytes + BAR_BYTES + 1024;
     return L;
@@ -91,8 +109,8 @@ __global__ void __launch_bounds__(THREADS, 1)
             mbar_init(bar(i), 1);
             mbar_init(bar(S + i), NQ_SET + (has_mma ? 1 : 0));  // one set of quantizer warps + MMA
         }
-        mbar_init(bar(2 * S), 1);
-        mbar_init(bar(2 * S + 1), 1);
+        mbar_init(bar(2 * S), MW);
+        mbar_init(bar(2 * S + 1), MW);
         *abort_flag = 0;
         fence_mbar_init();
         fence_proxy_async_smem();
@@ -132,10 +150,12 @@ __global__ void __launch_bounds__(THREADS, 1)
                 mbar_wait(bar(j % S), (j / S) & 1, &no_abort, p.status);
             }
         }
-    } else if (warp == 1) {
+    } else if (warp < QW0) {
         if (has_mma && lane == 0) {
+            const int m = warp - 1;  // this issuer takes stages k with k % MW == m
+            const uint32_t acc = tmem + m * (p.tmem_cols / MW);
             const uint32_t idesc = idesc_bf16(BM, p.Rp);
-            for (int k = 0; k < nk; ++k) {
+            for (int k = m; k < nk; k += MW) {
                 const int s = k % S;
                 if (!mbar_wait(bar(s), (k / S) & 1, abort_flag, p.status)) break;
                 tc_fence_after();
@@ -143,7 +163,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                 const uint64_t ad = sdesc_kmajor_sw128(st);
                 const uint64_t bd = sdesc_kmajor_sw128(st + X_BYTES);
 #pragma unroll
-                for (int i = 0; i < 4; ++i) mma_bf16(tmem, ad + 2 * i, bd + 2 * i, idesc, (k | i) != 0);
+                for (int i = 0; i < 4; ++i) mma_bf16(acc, ad + 2 * i, bd + 2 * i, idesc, k >= MW || i != 0);
                 tc_commit(bar(S + s));
             }
             tc_commit(bar(2 * S));
@@ -153,14 +173,17 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
     } else {
         // ---------------------------------------------------------------- quantizers
-        // Warp qw owns the 16-row block-row qw of the band; in each 128 x 64 stage it
-        // has four 16x16 blocks.  Lane L works on block j = L / 8 and holds rows
-        // l8 and l8 + 8 (l8 = L % 8) of it, 16 elements each: the block max needs three
-        // shuffle steps inside the 8-lane group, and each lane derives its block's scale
-        // once.  The per-tensor table inv[sb] = fl32(g / val(sb)) replaces the division
-        // per block; the block max / 6 uses div6_bf16 (exact for bf16 inputs).
-        const int qw = (warp - 2) % NQ_SET;  // block-row of the band
-        const int set = (warp - 2) / NQ_SET;  // this warp takes stages k with k % NSETS == set
+        // A set of NQ_SET warps quantizes one stage; warp qw of the set owns BR = 8 / NQ_SET
+        // consecutive 16-row block-rows of the band.  Lane L works on column block
+        // j = L / 8 of the stage and holds, in each of its block-rows, rows l8 and l8 + 8
+        // (l8 = L % 8), 16 elements each: a block max takes three shuffle steps inside the
+        // 8-lane group, and each lane derives its block's scale once.  The warp copies its
+        // rows out of the stage and releases the stage at once (the arithmetic runs on
+        // registers), so the ring refills while the sets compute.  The per-tensor table
+        // inv[sb] = fl32(g / val(sb)) replaces the division per block; the block max / 6
+        // uses div6_bf16 (exact for bf16 inputs).
+        const int qw = (warp - QW0) % NQ_SET;
+        const int set = (warp - QW0) / NQ_SET;  // this warp takes stages k with k % NSETS == set
         float g = 1.0f;
         bool degenerate = true;
         {
@@ -173,120 +196,144 @@ __global__ void __launch_bounds__(THREADS, 1)
                 }
             }
         }
-        if (band == 0 && split == 0 && threadIdx.x == 64) *p.g_out = g;
+        if (band == 0 && split == 0 && threadIdx.x == 32 * QW0) *p.g_out = g;
         float* inv_lut = reinterpret_cast<float*>(bar_area + 160);  // 128 floats
         {
-            const int t = threadIdx.x - 64;
+            const int t = threadIdx.x - 32 * QW0;
             if (t < 128) inv_lut[t] = (t > 0 && t < 127) ? __fdiv_rn(g, ue4m3_to_f32(t)) : 0.0f;
             asm volatile("bar.sync 1, %0;" ::"n"(32 * NQ) : "memory");  // quantizer warps only
         }
-        const int j = lane >> 3;       // block of the stage
+        const int j = lane >> 3;  // column block of the stage
         const int l8 = lane & 7;
-        const int rA = qw * 16 + l8;   // the lane's two rows inside the band
-        const int rB = rA + 8;
+        // the lane's rows inside the band: rows[2b] = block-row b's row l8, rows[2b+1] = row l8 + 8
+        int rows[2 * BR];
+#pragma unroll
+        for (int b = 0; b < BR; ++b) {
+            rows[2 * b] = (qw * BR + b) * 16 + l8;
+            rows[2 * b + 1] = rows[2 * b] + 8;
+        }
         const int64_t cbs = p.cols / 16;
         const int64_t atoms_per_band = p.cols / 64;
+        // bf16 bits of max |x| over a row's 16 elements (two 16-byte chunks): a tree of
+        // packed magnitude maxima, then the sign bits cleared (the quantizer's inputs are
+        // finite or infinite, never NaN)
+        auto row_max = [](const uint4& a, const uint4& b) -> uint32_t {
+            const uint32_t m = absmax_bf16x2(absmax_bf16x2(absmax_bf16x2(a.x, a.y), absmax_bf16x2(a.z, a.w)),
+                                             absmax_bf16x2(absmax_bf16x2(b.x, b.y), absmax_bf16x2(b.z, b.w))) &
+                               0x7FFF7FFFu;
+            return max(m & 0xFFFFu, m >> 16);
+        };
+        auto scale_of = [&](uint32_t amb) -> uint32_t {  // amb: bf16 bits of the block max
+            return degenerate ? 0u : cvt_ue4m3(__fmul_rn(div6_bf16(__uint_as_float(amb << 16)), g));
+        };
+        auto encode8 = [&](const uint4& u, float inv) {
+            float v[8];  // x * inv, each rounded to nearest in fp32 (two per instruction)
+            mul2_rn(bf16lo_to_f32(u.x), bf16hi_to_f32(u.x), inv, v[0], v[1]);
+            mul2_rn(bf16lo_to_f32(u.y), bf16hi_to_f32(u.y), inv, v[2], v[3]);
+            mul2_rn(bf16lo_to_f32(u.z), bf16hi_to_f32(u.z), inv, v[4], v[5]);
+            mul2_rn(bf16lo_to_f32(u.w), bf16hi_to_f32(u.w), inv, v[6], v[7]);
+            return cvt_e2m1x8(v);
+        };
+        // the four blocks' scale bytes of one row, gathered from the lanes with the same
+        // l8: l8, l8 + 8, l8 + 16, l8 + 24 hold blocks 0..3
+        auto gather4 = [&](uint32_t sbv) {
+            return __shfl_sync(0xffffffffu, sbv, l8) | (__shfl_sync(0xffffffffu, sbv, l8 + 8) << 8) |
+                   (__shfl_sync(0xffffffffu, sbv, l8 + 16) << 16) |
+                   (__shfl_sync(0xffffffffu, sbv, l8 + 24) << 24);
+        };
         for (int k = set; k < nk; k += NSETS) {
             const int s = k % S;
             if (!mbar_wait(bar(s), (k / S) & 1, abort_flag, p.status)) break;
             const uint8_t* tile = base + s * L.stage_bytes;
-            const int64_t c0 = col0 + k * BKE;
-            uint4 w[4];  // rows rA, rA, rB, rB; 16-byte chunks 2j, 2j + 1
-            w[0] = *reinterpret_cast<const uint4*>(tile + rA * 128 + (((2 * j) ^ (rA & 7)) << 4));
-            w[1] = *reinterpret_cast<const uint4*>(tile + rA * 128 + (((2 * j + 1) ^ (rA & 7)) << 4));
-            w[2] = *reinterpret_cast<const uint4*>(tile + rB * 128 + (((2 * j) ^ (rB & 7)) << 4));
-            w[3] = *reinterpret_cast<const uint4*>(tile + rB * 128 + (((2 * j + 1) ^ (rB & 7)) << 4));
-            uint8_t* crow = p.codes + (row0 + rA) * (p.cols / 2) + c0 / 2 + 8 * j;
-            // max |x| on the bf16 bit patterns (sign cleared: integer order = numeric order)
-            auto wmax = [](const uint4& u) {
-                return __vmaxu2(__vmaxu2(u.x & 0x7FFF7FFFu, u.y & 0x7FFF7FFFu),
-                                __vmaxu2(u.z & 0x7FFF7FFFu, u.w & 0x7FFF7FFFu));
-            };
-            auto half_max = [](uint32_t m2) { return max(m2 & 0xFFFFu, m2 >> 16); };
-            auto scale_of = [&](uint32_t amb) -> uint32_t {  // amb: bf16 bits of the block max
-                return degenerate ? 0u : cvt_ue4m3(__fmul_rn(div6_bf16(__uint_as_float(amb << 16)), g));
-            };
-            auto encode8 = [&](const uint4& u, float inv) {
-                float v[8];
-                v[0] = __fmul_rn(bf16lo_to_f32(u.x), inv); v[1] = __fmul_rn(bf16hi_to_f32(u.x), inv);
-                v[2] = __fmul_rn(bf16lo_to_f32(u.y), inv); v[3] = __fmul_rn(bf16hi_to_f32(u.y), inv);
-                v[4] = __fmul_rn(bf16lo_to_f32(u.z), inv); v[5] = __fmul_rn(bf16hi_to_f32(u.z), inv);
-                v[6] = __fmul_rn(bf16lo_to_f32(u.w), inv); v[7] = __fmul_rn(bf16hi_to_f32(u.w), inv);
-                return cvt_e2m1x8(v);
-            };
-            // the four blocks' scale bytes of this lane's rows, gathered from the lanes with
-            // the same l8: l8, l8 + 8, l8 + 16, l8 + 24 hold blocks 0..3
-            auto gather4 = [&](uint32_t sbv) {
-                return __shfl_sync(0xffffffffu, sbv, l8) | (__shfl_sync(0xffffffffu, sbv, l8 + 8) << 8) |
-                       (__shfl_sync(0xffffffffu, sbv, l8 + 16) << 16) |
-                       (__shfl_sync(0xffffffffu, sbv, l8 + 24) << 24);
-            };
-            uint8_t* atom = p.sf_mma ? p.sf_mma + (static_cast<int64_t>(band) * atoms_per_band + c0 / 64) * 512
-                                     : nullptr;
-            if constexpr (GRAN == 16) {
-                // 16x16 block: the 8 lanes of block j hold its 16 rows
-                uint32_t amb = half_max(__vmaxu2(__vmaxu2(wmax(w[0]), wmax(w[1])), __vmaxu2(wmax(w[2]), wmax(w[3]))));
-                amb = max(amb, __shfl_xor_sync(0xffffffffu, amb, 1));
-                amb = max(amb, __shfl_xor_sync(0xffffffffu, amb, 2));
-                amb = max(amb, __shfl_xor_sync(0xffffffffu, amb, 4));
-                const uint32_t sb = scale_of(amb);
-                const float inv = inv_lut[sb];
-                uint32_t code[4];  // row rA: words 0, 1; row rB: words 2, 3
+            uint4 w[2 * BR][2];  // per row: 16-byte chunks 2j, 2j + 1
 #pragma unroll
-                for (int q2 = 0; q2 < 4; ++q2) code[q2] = sb ? encode8(w[q2], inv) : 0u;
-                *reinterpret_cast<uint2*>(crow) = make_uint2(code[0], code[1]);
-                *reinterpret_cast<uint2*>(crow + 8 * (p.cols / 2)) = make_uint2(code[2], code[3]);
-                const uint32_t sb4 = gather4(sb);
-                if (lane == 0)
-                    *reinterpret_cast<uint32_t*>(p.scales + (row0 / 16 + qw) * cbs + c0 / 16) = sb4;
-                if (atom && j == 0) {
-                    *reinterpret_cast<uint32_t*>(atom + 16 * (rA % 32) + 4 * (rA / 32)) = sb4;
-                    *reinterpret_cast<uint32_t*>(atom + 16 * (rB % 32) + 4 * (rB / 32)) = sb4;
-                }
-            } else {
-                // group-wise 1x16: each of the lane's two rows is a group of its own
-                const uint32_t sbA = scale_of(half_max(__vmaxu2(wmax(w[0]), wmax(w[1]))));
-                const uint32_t sbB = scale_of(half_max(__vmaxu2(wmax(w[2]), wmax(w[3]))));
-                const float invA = inv_lut[sbA], invB = inv_lut[sbB];
-                const uint32_t c0w = sbA ? encode8(w[0], invA) : 0u, c1w = sbA ? encode8(w[1], invA) : 0u;
-                const uint32_t c2w = sbB ? encode8(w[2], invB) : 0u, c3w = sbB ? encode8(w[3], invB) : 0u;
-                *reinterpret_cast<uint2*>(crow) = make_uint2(c0w, c1w);
-                *reinterpret_cast<uint2*>(crow + 8 * (p.cols / 2)) = make_uint2(c2w, c3w);
-                const uint32_t sb4A = gather4(sbA), sb4B = gather4(sbB);
-                if (j == 0) {
-                    *reinterpret_cast<uint32_t*>(p.scales + (row0 + rA) * cbs + c0 / 16) = sb4A;
-                    *reinterpret_cast<uint32_t*>(p.scales + (row0 + rB) * cbs + c0 / 16) = sb4B;
-                    if (atom) {
-                        *reinterpret_cast<uint32_t*>(atom + 16 * (rA % 32) + 4 * (rA / 32)) = sb4A;
-                        *reinterpret_cast<uint32_t*>(atom + 16 * (rB % 32) + 4 * (rB / 32)) = sb4B;
-                    }
-                }
+            for (int i = 0; i < 2 * BR; ++i) {
+                const int r = rows[i];
+                w[i][0] = *reinterpret_cast<const uint4*>(tile + r * 128 + (((2 * j) ^ (r & 7)) << 4));
+                w[i][1] = *reinterpret_cast<const uint4*>(tile + r * 128 + (((2 * j + 1) ^ (r & 7)) << 4));
             }
+            uint32_t rmax[2 * BR];  // per row: max |x| over its 16 elements (bf16 bits)
+#pragma unroll
+            for (int i = 0; i < 2 * BR; ++i) rmax[i] = row_max(w[i][0], w[i][1]);
+            // every loaded word has been consumed: the stage goes back to the producer
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(S + s));
+
+            const int64_t c0 = col0 + k * BKE;
+            uint8_t* atom = p.sf_mma ? p.sf_mma + (static_cast<int64_t>(band) * atoms_per_band + c0 / 64) * 512
+                                     : nullptr;
+            uint32_t sb[2 * BR];  // per row: its block's (16x16) or its group's (1x16) scale
+            if constexpr (GRAN == 16) {
+#pragma unroll
+                for (int b = 0; b < BR; ++b) {
+                    uint32_t amb = max(rmax[2 * b], rmax[2 * b + 1]);
+                    amb = max(amb, __shfl_xor_sync(0xffffffffu, amb, 1));
+                    amb = max(amb, __shfl_xor_sync(0xffffffffu, amb, 2));
+                    amb = max(amb, __shfl_xor_sync(0xffffffffu, amb, 4));
+                    sb[2 * b] = sb[2 * b + 1] = scale_of(amb);
+                }
+            } else {
+#pragma unroll
+                for (int i = 0; i < 2 * BR; ++i) sb[i] = scale_of(rmax[i]);
+            }
+#pragma unroll
+            for (int i = 0; i < 2 * BR; ++i) {
+                const float inv = inv_lut[sb[i]];
+                const uint32_t lo = sb[i] ? encode8(w[i][0], inv) : 0u;
+                const uint32_t hi = sb[i] ? encode8(w[i][1], inv) : 0u;
+                *reinterpret_cast<uint2*>(p.codes + (row0 + rows[i]) * (p.cols / 2) + c0 / 2 + 8 * j) =
+                    make_uint2(lo, hi);
+            }
+            // scale words (the four blocks of a row): row i of the lane's 2 * BR rows is
+            // stored by the lanes of group j = i % 4
+#pragma unroll
+            for (int i = 0; i < 2 * BR; ++i) {
+                if (GRAN == 16 && (i & 1)) continue;  // both rows of a block-row share one word
+                const uint32_t w4 = gather4(sb[i]);
+                if constexpr (GRAN == 16) {
+                    if (lane == i / 2)
+                        *reinterpret_cast<uint32_t*>(p.scales + (row0 / 16 + qw * BR + i / 2) * cbs + c0 / 16) = w4;
+                }
+#pragma unroll
+                for (int h = 0; h < (GRAN == 16 ? 2 : 1); ++h) {
+                    const int ii = i + h;
+                    if ((ii & 3) != j) continue;
+                    const int r = rows[ii];
+                    if constexpr (GRAN == 1)
+                        *reinterpret_cast<uint32_t*>(p.scales + (row0 + r) * cbs + c0 / 16) = w4;
+                    if (atom) *reinterpret_cast<uint32_t*>(atom + 16 * (r % 32) + 4 * (r / 32)) = w4;
+                }
+            }
         }
         // ------------------------------------------------------------ T partial epilogue
-        if (has_mma && warp < 6) {
-            const int q = warp & 3;
+        if (has_mma && warp >= QW0 && warp < QW0 + 4) {
+            const int q = warp & 3;  // the TMEM lane quarter this warp may read
             if (mbar_wait(bar(2 * S), 0, abort_flag, p.status)) {
                 tc_fence_after();
                 const int64_t orow = row0 + 32 * q + lane;
                 float* dst = p.partial + (static_cast<int64_t>(split) * p.rows + orow) * p.Rp;
-                for (int c = 0; c < p.Rp; c += 16) {
-                    uint32_t v[16];
+                const int used = nk < MW ? nk : MW;  // accumulators that received stages
+                auto ld16 = [&](uint32_t col, uint32_t (&v)[16]) {
                     asm volatile(
                         "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
                         "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
                         : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]),
                           "=r"(v[6]), "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]),
                           "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
-                        : "r"(tmem + (static_cast<uint32_t>(32 * q) << 16) + c));
-                    tmem_ld_wait();
+                        : "r"(tmem + (static_cast<uint32_t>(32 * q) << 16) + col));
+                };
+                for (int c = 0; c < p.Rp; c += 16) {
+                    float t[16];
+                    for (int m = 0; m < used; ++m) {  // accumulators added in order
+                        uint32_t v[16];
+                        ld16(m * (p.tmem_cols / MW) + c, v);
+                        tmem_ld_wait();
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) t[e] = m ? __fadd_rn(t[e], __uint_as_float(v[e])) : __uint_as_float(v[e]);
+                    }
 #pragma unroll
                     for (int e = 0; e < 16; e += 4)
-                        *reinterpret_cast<float4*>(dst + c + e) =
-                            make_float4(__uint_as_float(v[e]), __uint_as_float(v[e + 1]),
-                                        __uint_as_float(v[e + 2]), __uint_as_float(v[e + 3]));
+                        *reinterpret_cast<float4*>(dst + c + e) = make_float4(t[e], t[e + 1], t[e + 2], t[e + 3]);
                 }
             }
         }
@@ -311,6 +358,15 @@ int quant_down_splits(int64_t rows, int64_t cols, int num_sms) {
     if (s > 16) s = 16;
     while (s > 1 && tiles % s) --s;
     return static_cast<int>(s);
+}
+
+uint32_t quant_down_tmem_cols(int Rp) {
+    // MW accumulators, each at a multiple of 32 columns; a power of two >= 32 in all
+    uint32_t per = 32;
+    while (per < static_cast<uint32_t>(Rp)) per += 32;
+    uint32_t c = 32;
+    while (c < per * qf::MW) c <<= 1;
+    return c;
 }
 
 size_t quant_down_smem_bytes(int Rp) { return static_cast<size_t>(qf::layout_for(Rp).smem_bytes); }
