@@ -144,13 +144,19 @@ __global__ void __launch_bounds__(threads(EPI), 1)
         // ---------------------------------------------------------------- producer
         if (lane == 0) {
             int it = 0;
+            int s = 0;        // it % STAGES
+            uint32_t ph = 0;  // (it / STAGES) & 1
+            auto acquire = [&]() { return mbar_wait(bar(BAR_EMPTY(s)), ph ^ 1, abort_flag, p.status); };
+            auto advance = [&]() {
+                ++it;
+                if (++s == STAGES) { s = 0; ph ^= 1; }
+            };
             for (int t = pair; t < num_tiles && !*abort_flag; t += num_pairs) {
                 const int mb2 = t % MB2, nb = t / MB2;
                 const int m_band = mb2 * 2 + static_cast<int>(rank);            // this CTA's A rows
                 const int n_rows = nb * BN + BN_CTA * static_cast<int>(rank);  // this CTA's B rows
-                for (int kt = 0; kt < KT; ++kt, ++it) {
-                    const int s = it % STAGES;
-                    if (!mbar_wait(bar(BAR_EMPTY(s)), ((it / STAGES) & 1) ^ 1, abort_flag, p.status)) break;
+                for (int kt = 0; kt < KT; ++kt, advance()) {
+                    if (!acquire()) break;
                     const uint32_t full = bar(BAR_FULL(s));
                     const uint32_t st = stage(s);
                     mbar_arrive_expect_tx(full, STAGE_BYTES);
@@ -165,9 +171,8 @@ __global__ void __launch_bounds__(threads(EPI), 1)
                                   full);
                 }
                 if (*abort_flag) break;
-                for (int kl = 0; kl < KLS; ++kl, ++it) {
-                    const int s = it % STAGES;
-                    if (!mbar_wait(bar(BAR_EMPTY(s)), ((it / STAGES) & 1) ^ 1, abort_flag, p.status)) break;
+                for (int kl = 0; kl < KLS; ++kl, advance()) {
+                    if (!acquire()) break;
                     const uint32_t full = bar(BAR_FULL(s));
                     const uint32_t st = stage(s);
                     mbar_arrive_expect_tx(full, A_BYTES + B_BYTES);
@@ -186,14 +191,20 @@ __global__ void __launch_bounds__(threads(EPI), 1)
         if (rank == 0 && lane == 0) {
             const uint32_t idesc4 = idesc_fp4_block16(2 * BM, BN);
             const uint32_t idesc16 = idesc_bf16(2 * BM, BN);
-            int it = 0, ti = 0;
+            // Every instruction of this thread between MMAs delays the tensor pipe: the loop
+            // keeps running stage / parity counters instead of dividing.
+            int ti = 0;
+            int s = 0;        // stage of the next k step
+            uint32_t ph = 0;  // its use parity
             for (int t = pair; t < num_tiles && !*abort_flag; t += num_pairs, ++ti) {
                 if (!mbar_wait(bar(BAR_TMEM_EMPTY), (ti & 1) ^ 1, abort_flag, p.status)) break;
                 tc_fence_after();
                 bool ok = true;
-                for (int j = 0; j < KT + KLS; ++j, ++it) {
-                    const int s = it % STAGES;
-                    if (!mbar_wait(bar(BAR_SF_READY(s)), (it / STAGES) & 1, abort_flag, p.status)) {
+                for (int j = 0; j < KT + KLS; ++j) {
+                    // one plain try_wait first: the bounded wait costs more even when the
+                    // phase is already complete
+                    const uint32_t rdy = bar(BAR_SF_READY(s));
+                    if (!mbar_try_wait(rdy, ph) && !mbar_wait(rdy, ph, abort_flag, p.status)) {
                         ok = false;
                         break;
                     }
@@ -215,6 +226,10 @@ __global__ void __launch_bounds__(threads(EPI), 1)
                     }
                     tc_commit_pair(bar(BAR_EMPTY(s)));
                     tc_commit_pair(mapa_shared(bar(BAR_EMPTY(s)), 1));
+                    if (++s == STAGES) {
+                        s = 0;
+                        ph ^= 1;
+                    }
                 }
                 if (!ok) break;
                 tc_commit_pair(bar(BAR_TMEM_FULL));
