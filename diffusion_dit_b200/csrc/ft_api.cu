@@ -226,7 +226,8 @@ ft_status quantize_operand(const void* x, int64_t rows, int64_t cols, int64_t ld
 ft_status run_gemm(const uint8_t* a_codes, const uint8_t* a_sf, const float* ga, const ft_fp4& b,
                    const __nv_bfloat16* la, const __nv_bfloat16* lb, int KL, int64_t M, int64_t N,
                    int64_t K, void* out, int* status, const DeviceInfo& dev, cudaStream_t st,
-                   void* act_out = nullptr, float* act_amax = nullptr, const void* gelu_in = nullptr) {
+                   void* act_out = nullptr, float* act_amax = nullptr, const void* gelu_in = nullptr,
+                   const ft::LoraFinalizeJob* side = nullptr) {
     // CTA pairs (256 x 256 tiles) when M allows, single CTAs (128 x 256) otherwise.
     const bool pair = (M % 256) == 0 && dev.num_sms >= 2;
     const uint32_t b_rows = pair ? 128 : 256;
@@ -262,6 +263,10 @@ ft_status run_gemm(const uint8_t* a_codes, const uint8_t* a_sf, const float* ga,
     g.act_out = bfm(act_out);
     g.act_amax = reinterpret_cast<unsigned*>(act_amax);
     g.gelu_in = bf(gelu_in);
+    if (side) {
+        g.side0 = side[0];
+        g.side1 = side[1];
+    }
     if (pair)
         FT_CUDA(ft::launch_gemm_fp4_lowrank_pair(tA, tB, tLA, tLB, tOut, tAct, g, dev.num_sms, st));
     else
@@ -601,8 +606,8 @@ ft_status linear_bwd_impl(const ft_linear* L, const void* x_dev, const float* t_
     g.tmem_cols = tmem_cols_for(NBW);
     g.status = status;
     const float* amax_g = amax_or_null;
-    // dB's split sum waits and runs in one launch with dA's (the two jobs of the finalize)
-    ft::LoraFinalizeJob fin_b{}, fin_a{};
+    // dB's and dA's split sums run on the dX GEMM's epilogue warps, before its first tile
+    ft::LoraFinalizeJob fin[2] = {};
     if (L->r > 0) {
         CUtensorMap tP, tV;
         FT_TRY(make_tmap(&tV, W + w.vcat, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, NBW, M, NBW * 2, 64, 64));
@@ -617,7 +622,7 @@ ft_status linear_bwd_impl(const ft_linear* L, const void* x_dev, const float* t_
         }
         FT_CUDA(ft::launch_lora_grad(tP, tV, g, sp, ft::K_LORA_DB, st));
         g.amax_out = nullptr;
-        fin_b = ft::LoraFinalizeJob{g.partial, sp, static_cast<int>(N), NBW, L->r, L->lora_scale, false, db_dev};
+        fin[1] = ft::LoraFinalizeJob{g.partial, sp, static_cast<int>(N), NBW, L->r, L->lora_scale, false, db_dev};
     }
     int splits = 1;
     FT_TRY(quantize_operand(dy_dev, M, N, N, amax_g, scal + SC_AMAX_G, R > 0, W + w.qg_codes, W + w.qg_scales,
@@ -652,12 +657,11 @@ ft_status linear_bwd_impl(const ft_linear* L, const void* x_dev, const float* t_
         g.tokens_per_split = static_cast<int>(M / sp);
         g.partial = reinterpret_cast<float*>(W + w.gpartial_a);
         FT_CUDA(ft::launch_lora_grad(tP, tV, g, sp, ft::K_LORA_DA, st));
-        fin_a = ft::LoraFinalizeJob{g.partial, sp, static_cast<int>(K), NBW, L->r, L->lora_scale, true, da_dev};
-        FT_CUDA(ft::launch_lora_grad_finalize(fin_a, fin_b, st));
+        fin[0] = ft::LoraFinalizeJob{g.partial, sp, static_cast<int>(K), NBW, L->r, L->lora_scale, true, da_dev};
     }
     // The dX GEMM goes last: the GEMM's operand and output traffic would evict G from L2.
     FT_TRY(run_gemm(W + w.qg_codes, W + w.qg_sf, scal + SC_G_G, L->qr_t, bf(W + w.ucat), bf(W + w.dntcat), KL,
-                    M, K, N, dx_dev, status, dev, st, nullptr, nullptr, gelu_in));
+                    M, K, N, dx_dev, status, dev, st, nullptr, nullptr, gelu_in, L->r > 0 ? fin : nullptr));
     return FT_OK;
 }
 

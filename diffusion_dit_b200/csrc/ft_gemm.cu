@@ -23,6 +23,7 @@
 // 32 (w % 4) .. +31).
 #include "ft_internal.h"
 #include "ft_ptx.cuh"
+#include "ft_sidejobs.cuh"
 
 namespace ft {
 namespace gemm {
@@ -275,6 +276,8 @@ __global__ void __launch_bounds__(THREADS, 1)
     } else {
         // ------------------------------------------------------------ epilogue
         const int q = warp & 3;  // TMEM lane quarter this warp may access
+        if (p.side0.out || p.side1.out)  // epilogue warps 2..5: 128 threads per CTA
+            lora_split_sums(p.side0, p.side1, blockIdx.x * 128 + (threadIdx.x - 64), gridDim.x * 128);
         const float ga = *p.ga, gb = *p.gb;
         const float c = 1.0f / (ga * gb);
         float hmax = 0.0f;  // max |gelu output| of this thread's elements (GELU epilogue)

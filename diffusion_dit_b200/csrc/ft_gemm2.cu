@@ -23,6 +23,7 @@
 // columns each), then 4 scale writers.
 #include "ft_internal.h"
 #include "ft_ptx.cuh"
+#include "ft_sidejobs.cuh"
 
 namespace ft {
 namespace gemm2 {
@@ -282,6 +283,9 @@ __global__ void __launch_bounds__(threads(EPI), 1)
     } else {
         // ---------------------------------------------------------------- epilogue (both CTAs)
         const int q = warp & 3;
+        if (p.side0.out || p.side1.out)
+            lora_split_sums(p.side0, p.side1, blockIdx.x * (32 * EPI_WARPS) + (threadIdx.x - 64),
+                            gridDim.x * (32 * EPI_WARPS));
         const int cbase = EPI_COLS * ((warp - 2) >> 2);  // this warp's first tile column
         const float ga = *p.ga, gb = *p.gb;
         const float c = 1.0f / (ga * gb);

@@ -39,6 +39,17 @@ cudaError_t launch_k(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t sme
 // GEMM epilogue variants, one kernel instantiation each (the plain one carries no GELU code)
 enum EpilogueKind { kEpiPlain = 0, kEpiGelu = 1, kEpiGeluBwd = 2 };
 
+// One split sum of the adapter gradients (run by lora_split_sums in ft_sidejobs.cuh):
+// out = s * sum over the splits (in order) of (D[f][j] + D[f][r + j]); out[f][j], or
+// out[j][f] with transpose_out.  out == nullptr: no job.
+struct LoraFinalizeJob {
+    const float* partial;    // [splits, F, NBW], splits <= 16
+    int splits, F, NBW, r;
+    float s;
+    bool transpose_out;
+    float* out;
+};
+
 struct GemmFp4Args {
     const uint8_t* sfa;     // tensor-core scale layout of A (rows M, cols K)
     const uint8_t* sfb;     // tensor-core scale layout of B (rows N, cols K)
@@ -56,6 +67,9 @@ struct GemmFp4Args {
     // optional GELU-backward epilogue: store bf16(bf16(out) * gelu_tanh'(gelu_in)) instead
     // of out, gelu_in bf16 with out's layout (the MLP's pre-activation P)
     const __nv_bfloat16* gelu_in;
+    // optional side jobs for the epilogue warps, run before their first tile (they wait
+    // for the first accumulator anyway): the adapter gradients' split sums
+    LoraFinalizeJob side0, side1;
 };
 
 // tmOut (and tmAct): bf16 [M, N] output, box 32 x 32, 64-byte swizzle.
@@ -168,15 +182,5 @@ struct LoraGradArgs {
 int lora_grad_splits(int64_t M, int64_t F, int num_sms);
 cudaError_t launch_lora_grad(const CUtensorMap& tmP, const CUtensorMap& tmV, const LoraGradArgs& a, int splits,
                              int kind, cudaStream_t stream);
-// out = s * sum over the splits (in order) of (D[f][j] + D[f][r + j]); out[f][j], or out[j][f]
-// with transpose_out.  One launch runs up to two such jobs (j1.out == nullptr: none).
-struct LoraFinalizeJob {
-    const float* partial;    // [splits, F, NBW]
-    int splits, F, NBW, r;
-    float s;
-    bool transpose_out;
-    float* out;
-};
-cudaError_t launch_lora_grad_finalize(const LoraFinalizeJob& j0, const LoraFinalizeJob& j1, cudaStream_t stream);
 
 }  // namespace ft

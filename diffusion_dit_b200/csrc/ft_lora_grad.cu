@@ -12,7 +12,8 @@
 // columns and are added in the final sum, keeping ~16 mantissa bits of V.
 //
 // One CTA = 128 features x a slice of the tokens; partials[split][f][NBW] fp32 are
-// summed in a fixed order by lora_grad_finalize_kernel (deterministic).
+// summed in a fixed order (deterministic) by lora_split_sums (ft_sidejobs.cuh), which
+// the dX GEMM's epilogue warps run while they wait for their first accumulator.
 //
 // When asked (amax_out), the four epilogue warps, idle until the final drain, also take
 // max |P| over every tile that lands: with dB computed first in the backward pass this
@@ -187,36 +188,6 @@ __global__ void __launch_bounds__(THREADS, 1)
     if (warp == 1) tmem_dealloc(tmem, p.tmem_cols);
 }
 
-// out = s * sum_split (D[f][j] + D[f][r + j]); transposed (out[j][f]) for dA.
-__global__ void lora_grad_finalize_kernel(const LoraFinalizeJob j0, const LoraFinalizeJob j1) {
-    pdl_trigger();
-    pdl_wait();
-    const int total0 = j0.F * j0.r;
-    const int total = total0 + (j1.out ? j1.F * j1.r : 0);
-    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < total; i += gridDim.x * blockDim.x) {
-        const LoraFinalizeJob& jb = i < total0 ? j0 : j1;
-        const int ii = i < total0 ? i : i - total0;
-        int f, j;
-        if (jb.transpose_out) {  // consecutive threads walk f: coalesced stores into out[j][f]
-            j = ii / jb.F;
-            f = ii - j * jb.F;
-        } else {
-            f = ii / jb.r;
-            j = ii - f * jb.r;
-        }
-        float v = 0.0f;
-        for (int sp = 0; sp < jb.splits; ++sp) {
-            const float* d = jb.partial + (sp * jb.F + f) * jb.NBW;
-            v += d[j] + d[jb.r + j];
-        }
-        v *= jb.s;
-        if (jb.transpose_out)
-            jb.out[j * jb.F + f] = v;
-        else
-            jb.out[f * jb.r + j] = v;
-    }
-}
-
 }  // namespace lg
 
 int lora_grad_splits(int64_t M, int64_t F, int num_sms) {
@@ -244,17 +215,6 @@ cudaError_t launch_lora_grad(const CUtensorMap& tmP, const CUtensorMap& tmV, con
                                     L.smem_bytes, stream, tmP, tmV, a);
     if (le != cudaSuccess) return le;
     after_launch(kind, stream);
-    return cudaGetLastError();
-}
-
-cudaError_t launch_lora_grad_finalize(const LoraFinalizeJob& j0, const LoraFinalizeJob& j1, cudaStream_t stream) {
-    int64_t g = (static_cast<int64_t>(j0.F) * j0.r + (j1.out ? static_cast<int64_t>(j1.F) * j1.r : 0) + 255) / 256;
-    if (g > 148 * 8) g = 148 * 8;
-    before_launch(K_OTHER, stream);
-    const cudaError_t le = launch_k(lg::lora_grad_finalize_kernel, dim3(static_cast<unsigned>(g)), dim3(256), 0,
-                                    stream, j0, j1);
-    if (le != cudaSuccess) return le;
-    after_launch(K_OTHER, stream);
     return cudaGetLastError();
 }
 
