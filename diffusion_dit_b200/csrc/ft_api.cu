@@ -111,7 +111,7 @@ size_t max_splits(int64_t units) {
 
 // Workspace of the layer calls.  Regions are 256-byte aligned.
 struct LinearWs {
-    size_t status, scal, qx_codes, qx_scales, qx_sf, dn, upcat, tcat, partial;
+    size_t status, scal, amax_parts, qx_codes, qx_scales, qx_sf, dn, upcat, tcat, partial;
     size_t qg_codes, qg_scales, qg_sf, upt, dntcat, ucat, vcat, ucat_lora, gpartial_b, gpartial_a, total;
 };
 
@@ -130,6 +130,7 @@ LinearWs linear_ws(int64_t M, int64_t N, int64_t K, int R, int r) {
     };
     w.status = take(16);
     w.scal = take(16 * sizeof(float));
+    w.amax_parts = take(ft::kPrologueCtas * sizeof(float));
     w.qx_codes = take(static_cast<size_t>(M) * K / 2);
     w.qx_scales = take(static_cast<size_t>(M) * K / 16);  // 16x16 blocks use 1/16 of it, 1x16 groups all
     w.qx_sf = take(static_cast<size_t>(M) * K / 16);
@@ -189,9 +190,10 @@ __nv_bfloat16* bfm(void* p) { return static_cast<__nv_bfloat16*>(p); }
 ft_status quantize_operand(const void* x, int64_t rows, int64_t cols, int64_t ld, const float* amax_or_null,
                            float* amax_slot, bool amax_slot_cleared, uint8_t* codes, uint8_t* scales, uint8_t* sf, float* g,
                            const void* w, int Rp, float* partial, int* splits, int* status,
-                           const DeviceInfo& dev, cudaStream_t st, int block_rows = 16) {
+                           const DeviceInfo& dev, cudaStream_t st, int block_rows = 16,
+                           const float* amax_parts = nullptr) {
     const float* amax = amax_or_null;
-    if (!amax) {
+    if (!amax && !amax_parts) {
         FT_CUDA(ft::launch_amax(x, false, rows, cols, ld, amax_slot, amax_slot_cleared, dev.num_sms, st));
         amax = amax_slot;
     }
@@ -216,6 +218,10 @@ ft_status quantize_operand(const void* x, int64_t rows, int64_t cols, int64_t ld
     a.partial = partial;
     a.status = status;
     a.block_rows = block_rows;
+    if (!amax_or_null && amax_parts) {  // the prologue's per-CTA maxima
+        a.amax_parts = amax_parts;
+        a.amax_nparts = ft::kPrologueCtas;
+    }
     FT_CUDA(ft::launch_quant_down(tX, tW, a, s, st));
     *splits = s;
     return FT_OK;
@@ -489,23 +495,30 @@ ft_status linear_fwd_impl(const ft_linear* L, const void* x_dev, int64_t M, cons
     const int Rp = padded_rank(R);
     float* partial = reinterpret_cast<float*>(W + w.partial);
 
-    // Eq. (2): the factors of this step ([Ls_down; A] and [Ls_up, B]; A, B train),
-    // then Q(X) fused with T = X [Ls_down; A]^T, then the 4-bit GEMM with the
-    // up-projections in its accumulator.
-    // The factor kernel also clears the tensor-max slot (no memset node between kernels).
+    // Eq. (2): the factors of this step ([Ls_down; A] and [Ls_up, B]; A, B train) and
+    // max |X| in one prologue launch, then Q(X) fused with T = X [Ls_down; A]^T, then
+    // the 4-bit GEMM with the up-projections in its accumulator.  The prologue leaves
+    // one max per CTA, which the quantizer reduces (no cleared slot, no separate pass);
+    // it also clears the GELU epilogue's max slot.
     ft::PrologueExtras ex;
-    if (!amax_or_null) ex.zero_slot = scal + SC_AMAX_X;
+    float* amax_parts = nullptr;
+    if (!amax_or_null) {
+        amax_parts = reinterpret_cast<float*>(W + w.amax_parts);
+        ex.max_src = bf(x_dev);
+        ex.max_rows = M;
+        ex.max_cols = K;
+        ex.max_ld = K;
+        ex.max_parts = amax_parts;
+    }
     if (h_dev) ex.zero_slot2 = h_amax_dev;
-    if (R > 0)
+    if (R > 0 || amax_parts || h_dev)
         FT_CUDA(ft::launch_build_factors(bf(L->ls_down), bf(L->lora_a), bf(L->ls_up), bf(L->lora_b), N, K,
-                                         L->r_s, L->r, Rp, KL, bfm(W + w.dn), bfm(W + w.upcat), nullptr,
-                                         nullptr, &ex, st));
-    else if (h_dev)
-        FT_CUDA(cudaMemsetAsync(h_amax_dev, 0, sizeof(float), st));
+                                         L->r_s, L->r, Rp, KL, R > 0 ? bfm(W + w.dn) : nullptr,
+                                         R > 0 ? bfm(W + w.upcat) : nullptr, nullptr, nullptr, &ex, st));
     int splits = 1;
     FT_TRY(quantize_operand(x_dev, M, K, K, amax_or_null, scal + SC_AMAX_X, R > 0, W + w.qx_codes, W + w.qx_scales,
                             W + w.qx_sf, scal + SC_G_X, W + w.dn, Rp, partial, &splits, status, dev, st,
-                            x_block_rows));
+                            x_block_rows, amax_parts));
     if (R > 0) {
         ft::LowRankFinalizeArgs f{};
         f.partial = partial;

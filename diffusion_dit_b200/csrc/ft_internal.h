@@ -120,6 +120,9 @@ struct QuantDownArgs {
     float* partial;          // [splits, rows, Rp] fp32
     int* status;
     int block_rows;          // 16: 16x16 blocks, scales [rows/16, cols/16]; 1: 1x16 groups, [rows, cols/16]
+    // when set, the tensor max is max(amax_parts[0 .. amax_nparts)) instead of *amax
+    const float* amax_parts;
+    int amax_nparts;
 };
 int quant_down_splits(int64_t rows, int64_t cols, int num_sms);
 uint32_t quant_down_tmem_cols(int Rp);  // room for the kernel's accumulators of Rp columns
@@ -155,7 +158,14 @@ struct PrologueExtras {
     __nv_bfloat16* hilo_dst = nullptr;
     float* zero_slot = nullptr;
     float* zero_slot2 = nullptr;  // a second cleared max slot (the GELU epilogue's)
+    // max |x| over a bf16 matrix [max_rows, max_cols] (row stride max_ld): every CTA of
+    // the launch writes the max over its share to max_parts[blockIdx.x]
+    // (kPrologueCtas entries, no clearing needed); the quantizer reduces them
+    const __nv_bfloat16* max_src = nullptr;
+    int64_t max_rows = 0, max_cols = 0, max_ld = 0;
+    float* max_parts = nullptr;
 };
+constexpr int kPrologueCtas = 148 * 4;  // the factor kernel's grid
 
 // Build the concatenated low-rank factors used by the forward and backward GEMMs (and
 // run the side jobs in `extra`, which may be null).  dn and upt get Rp rows (rows

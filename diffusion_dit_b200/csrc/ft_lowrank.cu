@@ -132,6 +132,42 @@ __global__ void build_factors_kernel(const __nv_bfloat16* __restrict__ ls_down,
     }
     if (x.zero_slot && t0 == 0) *x.zero_slot = 0.0f;
     if (x.zero_slot2 && t0 == 0) *x.zero_slot2 = 0.0f;
+    // side job: max |x| of the call's input (the bulk of this launch when present), one
+    // partial per CTA; four independent 16-byte loads in flight per thread per trip
+    if (x.max_src) {
+        const int64_t vpr = x.max_cols / 8;
+        const int64_t nvec = x.max_rows * vpr;
+        const int64_t gstride = static_cast<int64_t>(stride);
+        float m = 0.0f;
+        auto vmax = [&](const uint4& u) {
+            const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+                m = fmaxf(m, fmaxf(fabsf(bf16lo_to_f32(w[e])), fabsf(bf16hi_to_f32(w[e]))));
+        };
+        auto at = [&](int64_t iv) {
+            return *reinterpret_cast<const uint4*>(x.max_src + (iv / vpr) * x.max_ld + (iv % vpr) * 8);
+        };
+        int64_t i = t0;
+        for (; i + 3 * gstride < nvec; i += 4 * gstride) {
+            uint4 v[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) v[u] = at(i + u * gstride);
+#pragma unroll
+            for (int u = 0; u < 4; ++u) vmax(v[u]);
+        }
+        for (; i < nvec; i += gstride) vmax(at(i));
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        __shared__ float red[8];
+        if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            float v = 0.0f;
+            for (int w = 0; w < static_cast<int>(blockDim.x >> 5); ++w) v = fmaxf(v, red[w]);
+            x.max_parts[blockIdx.x] = v;
+        }
+    }
 }
 
 }  // namespace
@@ -160,7 +196,7 @@ cudaError_t launch_build_factors(const __nv_bfloat16* ls_down, const __nv_bfloat
                                  const PrologueExtras* extra, cudaStream_t stream) {
     const PrologueExtras x = extra ? *extra : PrologueExtras{};
     before_launch(K_OTHER, stream);
-    const cudaError_t le = launch_k(build_factors_kernel, dim3(148 * 4), dim3(256), 0, stream,
+    const cudaError_t le = launch_k(build_factors_kernel, dim3(kPrologueCtas), dim3(256), 0, stream,
                                     ls_down, lora_a, ls_up, lora_b, static_cast<int>(N),
                                     static_cast<int>(K), r_s, r, Rp, KL, dn, upcat, upt, dntcat, x);
     if (le != cudaSuccess) return le;

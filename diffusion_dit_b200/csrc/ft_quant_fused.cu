@@ -48,7 +48,8 @@ constexpr int MW = FT_QUANT_MMA_WARPS;
 constexpr int QW0 = 1 + MW;                 // first quantizer warp
 constexpr int THREADS = 32 * (QW0 + NQ);    // producer, MMA issuers, quantizers
 constexpr int MAX_STAGES = 8;
-constexpr int BAR_BYTES = 768;           // barriers, TMEM slot, abort flag, inv table at +160
+constexpr int BAR_BYTES = 768;           // barriers, TMEM slot, abort flag, inv table at +160, max scratch at +672
+static_assert(160 + 512 + 4 * NQ <= BAR_BYTES, "barrier area overflow");
 
 struct Layout {
     int stages;
@@ -187,7 +188,20 @@ __global__ void __launch_bounds__(THREADS, 1)
         float g = 1.0f;
         bool degenerate = true;
         {
-            const float amax = *p.amax;
+            float amax;
+            if (p.amax_parts) {  // max of the per-CTA maxima (exact in any order)
+                float m = 0.0f;
+                for (int i = threadIdx.x - 32 * QW0; i < p.amax_nparts; i += 32 * NQ) m = fmaxf(m, p.amax_parts[i]);
+                m = warp_max(m);
+                float* red = reinterpret_cast<float*>(bar_area + 160 + 512);  // after the inv table
+                if (lane == 0) red[warp - QW0] = m;
+                asm volatile("bar.sync 1, %0;" ::"n"(32 * NQ) : "memory");  // quantizer warps only
+                m = 0.0f;
+                for (int w = 0; w < NQ; ++w) m = fmaxf(m, red[w]);
+                amax = m;
+            } else {
+                amax = *p.amax;
+            }
             if (amax > 0.0f) {
                 const float gg = __fdiv_rn(2688.0f, amax);
                 if (isfinite(gg) && gg > 0.0f) {
