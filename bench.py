@@ -655,7 +655,8 @@ def main():
         traffic = gemm_traffic() if args.workload == "qkv" else None
         # quantizer: X [M, K] and G [M, N] alternate; algorithmic bytes per element:
         # 2 (read bf16) + 0.5 (codes) + 1/256 (block scales).  The tensor max of X is one
-        # more read of X by its own kernel; max |G| is taken by the dB kernel.
+        # more read of X, by the forward's prologue kernel (which also builds the low-rank
+        # factors: its whole duration counts); max |G| is taken by the dB kernel.
         elems = [M * K, M * N] * Kst
         qbytes = sum(e * (2.0 + 0.5 + 1.0 / 256) for e in elems)
         q_gbs = qbytes / (sum(quant_ms) * 1e-3) / 1e9

@@ -195,12 +195,14 @@ cudaError_t launch_build_factors(const __nv_bfloat16* ls_down, const __nv_bfloat
                                  __nv_bfloat16* upcat, __nv_bfloat16* upt, __nv_bfloat16* dntcat,
                                  const PrologueExtras* extra, cudaStream_t stream) {
     const PrologueExtras x = extra ? *extra : PrologueExtras{};
-    before_launch(K_OTHER, stream);
+    // with the tensor-max job the launch is the call's max pass (timed as such)
+    const int kind = x.max_src ? K_AMAX : K_OTHER;
+    before_launch(kind, stream);
     const cudaError_t le = launch_k(build_factors_kernel, dim3(kPrologueCtas), dim3(256), 0, stream,
                                     ls_down, lora_a, ls_up, lora_b, static_cast<int>(N),
                                     static_cast<int>(K), r_s, r, Rp, KL, dn, upcat, upt, dntcat, x);
     if (le != cudaSuccess) return le;
-    after_launch(K_OTHER, stream);
+    after_launch(kind, stream);
     return cudaGetLastError();
 }
 

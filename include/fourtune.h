@@ -307,8 +307,8 @@ ft_status fourtune_encode_ue4m3(const float* v_dev, int64_t n, uint8_t* out_dev,
  */
 #define FT_KERNEL_GEMM 0      /* 4-bit GEMM with the low-rank tail (forward and dX) */
 #define FT_KERNEL_QUANT 1     /* 16x16 block quantizer */
-#define FT_KERNEL_AMAX 2      /* tensor max */
-#define FT_KERNEL_LOWRANK 3   /* low-rank down-projection */
+#define FT_KERNEL_AMAX 2      /* tensor max pass (the layer forward's: its prologue, which also builds the factors) */
+#define FT_KERNEL_LOWRANK 3   /* low-rank split sum */
 #define FT_KERNEL_LORA_DB 4   /* adapter gradient dB */
 #define FT_KERNEL_LORA_DA 5   /* adapter gradient dA */
 #define FT_KERNEL_KINDS 6
