@@ -435,27 +435,39 @@ __device__ __forceinline__ float ue4m3_to_f32(uint32_t code) {
 // it stays cheap next to the tile's MMAs; the polynomial steps are explicitly rounded.
 // The stand-alone kernels use these same functions, so they and the epilogue agree bit
 // for bit.  For |2u| beyond the fp32 exp range the sigmoid goes to 0 or 1 as it should
-// (__fdividef(x, inf) = 0).
-__device__ __forceinline__ float gelu_tanh_u(float p) {
-    const float k = 0.7978845608028654f;  // sqrt(2 / pi)
-    const float p3 = __fmul_rn(__fmul_rn(p, p), p);
-    return __fmul_rn(k, __fadd_rn(p, __fmul_rn(0.044715f, p3)));
+// (__fdividef(x, inf) = 0).  The derivative: dP = dH * gelu'(P) with s = sigmoid(2u),
+// gelu' = s + 2 p s (1 - s) u'; with e = exp(-2u), s = 1 / (1 + e) and 1 - s = e s (one
+// exponential and one reciprocal: the special-function pipe bounds that epilogue), the
+// exponent capped at 80 so e stays finite (then s ~ 1e-35 and e s = 1 to within rounding).
+// The arithmetic runs on packed fp32 pairs (the GELU epilogues are issue-bound: two
+// elements per instruction), each lane rounded to nearest as __fmul_rn / __fadd_rn do;
+// only the exponential and the divisions are per element.
+struct F2 {
+    float a, b;
+};
+__device__ __forceinline__ F2 f2_mul(F2 x, F2 y) {
+    F2 r;
+    asm("{\n\t.reg .b64 p, q, z;\n\tmov.b64 p, {%2, %3};\n\tmov.b64 q, {%4, %5};\n\t"
+        "mul.rn.f32x2 z, p, q;\n\tmov.b64 {%0, %1}, z;\n\t}"
+        : "=f"(r.a), "=f"(r.b)
+        : "f"(x.a), "f"(x.b), "f"(y.a), "f"(y.b));
+    return r;
 }
-
-__device__ __forceinline__ float gelu_tanh_f(float p) {
-    return __fdividef(p, __fadd_rn(1.0f, __expf(__fmul_rn(-2.0f, gelu_tanh_u(p)))));
+__device__ __forceinline__ F2 f2_add(F2 x, F2 y) {
+    F2 r;
+    asm("{\n\t.reg .b64 p, q, z;\n\tmov.b64 p, {%2, %3};\n\tmov.b64 q, {%4, %5};\n\t"
+        "add.rn.f32x2 z, p, q;\n\tmov.b64 {%0, %1}, z;\n\t}"
+        : "=f"(r.a), "=f"(r.b)
+        : "f"(x.a), "f"(x.b), "f"(y.a), "f"(y.b));
+    return r;
 }
+__device__ __forceinline__ F2 f2(float v) { return F2{v, v}; }
 
-// dP = dH * gelu'(P); with s = sigmoid(2u): gelu' = s + 2 p s (1 - s) u', and
-// 1 - s = sigmoid(-2u) taken directly (no inf / inf for large |u|).
-__device__ __forceinline__ float gelu_tanh_bwd_f(float p, float dh) {
-    const float k = 0.7978845608028654f;
-    const float u = gelu_tanh_u(p);
-    const float sg = __fdividef(1.0f, __fadd_rn(1.0f, __expf(__fmul_rn(-2.0f, u))));
-    const float one_minus = __fdividef(1.0f, __fadd_rn(1.0f, __expf(__fmul_rn(2.0f, u))));
-    const float du = __fmul_rn(k, __fadd_rn(1.0f, __fmul_rn(3.0f * 0.044715f, __fmul_rn(p, p))));
-    const float g = __fadd_rn(sg, __fmul_rn(__fmul_rn(__fmul_rn(__fmul_rn(2.0f, p), sg), one_minus), du));
-    return __fmul_rn(dh, g);
+// u = sqrt(2/pi) (p + 0.044715 p^3) of both lanes, each step rounded; p2 = p * p is
+// returned for reuse
+__device__ __forceinline__ F2 gelu_tanh_u2(F2 p, F2& p2) {
+    p2 = f2_mul(p, p);
+    return f2_mul(f2(0.7978845608028654f), f2_add(p, f2_mul(f2(0.044715f), f2_mul(p2, p))));
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
@@ -485,14 +497,28 @@ __device__ __forceinline__ float bf16hi_to_f32(uint32_t w) { return __uint_as_fl
 
 // Two packed bf16 gradients dh -> bf16(dh * gelu_tanh'(p)) each (p: two packed bf16).
 __device__ __forceinline__ uint32_t gelu_bwd_bf16x2(uint32_t dh, uint32_t p) {
-    return pack_bf16x2(gelu_tanh_bwd_f(bf16lo_to_f32(p), bf16lo_to_f32(dh)),
-                       gelu_tanh_bwd_f(bf16hi_to_f32(p), bf16hi_to_f32(dh)));
+    const F2 P{bf16lo_to_f32(p), bf16hi_to_f32(p)};
+    F2 pp;
+    const F2 u = gelu_tanh_u2(P, pp);
+    const F2 m2u = f2_mul(f2(-2.0f), u);
+    const F2 e{__expf(fminf(m2u.a, 80.0f)), __expf(fminf(m2u.b, 80.0f))};
+    const F2 den = f2_add(f2(1.0f), e);
+    const F2 sg{__fdividef(1.0f, den.a), __fdividef(1.0f, den.b)};
+    const F2 one_minus = f2_mul(e, sg);
+    const F2 du = f2_mul(f2(0.7978845608028654f), f2_add(f2(1.0f), f2_mul(f2(3.0f * 0.044715f), pp)));
+    const F2 g = f2_add(sg, f2_mul(f2_mul(f2_mul(f2_mul(f2(2.0f), P), sg), one_minus), du));
+    const F2 r = f2_mul(F2{bf16lo_to_f32(dh), bf16hi_to_f32(dh)}, g);
+    return pack_bf16x2(r.a, r.b);
 }
 
 // Two packed bf16 -> bf16(gelu_tanh(.)) each, packed the same way; hmax takes the larger
 // of itself and the two results' magnitudes (fmaxf: a NaN never wins).
 __device__ __forceinline__ uint32_t gelu_bf16x2(uint32_t w, float& hmax) {
-    const uint32_t r = pack_bf16x2(gelu_tanh_f(bf16lo_to_f32(w)), gelu_tanh_f(bf16hi_to_f32(w)));
+    const F2 P{bf16lo_to_f32(w), bf16hi_to_f32(w)};
+    F2 pp;
+    const F2 m2u = f2_mul(f2(-2.0f), gelu_tanh_u2(P, pp));
+    const F2 den = f2_add(f2(1.0f), F2{__expf(m2u.a), __expf(m2u.b)});
+    const uint32_t r = pack_bf16x2(__fdividef(P.a, den.a), __fdividef(P.b, den.b));
     hmax = fmaxf(hmax, fmaxf(fabsf(bf16lo_to_f32(r)), fabsf(bf16hi_to_f32(r))));
     return r;
 }
