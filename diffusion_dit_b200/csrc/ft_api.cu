@@ -672,9 +672,20 @@ ft_status linear_bwd_impl(const ft_linear* L, const void* x_dev, const float* t_
         FT_CUDA(ft::launch_lora_grad(tP, tV, g, sp, ft::K_LORA_DA, st));
         fin[0] = ft::LoraFinalizeJob{g.partial, sp, static_cast<int>(K), NBW, L->r, L->lora_scale, true, da_dev};
     }
+    // dA's and dB's split sums: on the dX GEMM's epilogue warps when they fit in the time
+    // those warps wait for their first accumulator (about a k step of 256 per 0.35 us, an
+    // output per thread ~0.4 us when the loads miss L1: kept within half of the first
+    // tile), else in a launch of their own before the GEMM.
+    bool side = false;
+    if (L->r > 0) {
+        const double outputs = static_cast<double>(N + K) * L->r;
+        const double per_thread = outputs / (static_cast<double>(dev.num_sms) * 128.0);
+        side = 2.0 * per_thread <= static_cast<double>(N / 256);
+        if (!side) FT_CUDA(ft::launch_lora_grad_finalize(fin[0], fin[1], st));
+    }
     // The dX GEMM goes last: the GEMM's operand and output traffic would evict G from L2.
     FT_TRY(run_gemm(W + w.qg_codes, W + w.qg_sf, scal + SC_G_G, L->qr_t, bf(W + w.ucat), bf(W + w.dntcat), KL,
-                    M, K, N, dx_dev, status, dev, st, nullptr, nullptr, gelu_in, L->r > 0 ? fin : nullptr));
+                    M, K, N, dx_dev, status, dev, st, nullptr, nullptr, gelu_in, side ? fin : nullptr));
     return FT_OK;
 }
 

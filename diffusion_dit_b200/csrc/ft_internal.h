@@ -50,6 +50,9 @@ struct LoraFinalizeJob {
     float* out;
 };
 
+// The two split sums in a launch of their own (lora_split_sums on every thread).
+cudaError_t launch_lora_grad_finalize(const LoraFinalizeJob& j0, const LoraFinalizeJob& j1, cudaStream_t stream);
+
 struct GemmFp4Args {
     const uint8_t* sfa;     // tensor-core scale layout of A (rows M, cols K)
     const uint8_t* sfb;     // tensor-core scale layout of B (rows N, cols K)

@@ -20,6 +20,7 @@
 // gives the tensor max of G for Q(G) without a separate pass over G.
 #include "ft_internal.h"
 #include "ft_ptx.cuh"
+#include "ft_sidejobs.cuh"
 
 namespace ft {
 namespace lg {
@@ -188,6 +189,14 @@ __global__ void __launch_bounds__(THREADS, 1)
     if (warp == 1) tmem_dealloc(tmem, p.tmem_cols);
 }
 
+// The split sums in a launch of their own (when the dX GEMM's epilogue warps could not
+// finish them within its first tile): the same routine, so the same sums bit for bit.
+__global__ void lora_grad_finalize_kernel(const LoraFinalizeJob j0, const LoraFinalizeJob j1) {
+    pdl_trigger();
+    pdl_wait();
+    lora_split_sums(j0, j1, blockIdx.x * blockDim.x + threadIdx.x, gridDim.x * blockDim.x);
+}
+
 }  // namespace lg
 
 int lora_grad_splits(int64_t M, int64_t F, int num_sms) {
@@ -215,6 +224,19 @@ cudaError_t launch_lora_grad(const CUtensorMap& tmP, const CUtensorMap& tmV, con
                                     L.smem_bytes, stream, tmP, tmV, a);
     if (le != cudaSuccess) return le;
     after_launch(kind, stream);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_lora_grad_finalize(const LoraFinalizeJob& j0, const LoraFinalizeJob& j1, cudaStream_t stream) {
+    int64_t g = ((j0.out ? static_cast<int64_t>(j0.F) * j0.r : 0) + (j1.out ? static_cast<int64_t>(j1.F) * j1.r : 0) +
+                 255) / 256;
+    if (g > 148 * 8) g = 148 * 8;
+    if (g < 1) g = 1;
+    before_launch(K_OTHER, stream);
+    const cudaError_t le = launch_k(lg::lora_grad_finalize_kernel, dim3(static_cast<unsigned>(g)), dim3(256), 0,
+                                    stream, j0, j1);
+    if (le != cudaSuccess) return le;
+    after_launch(K_OTHER, stream);
     return cudaGetLastError();
 }
 
