@@ -114,3 +114,42 @@ def test_repeated_calls_are_deterministic():
     dx2, da2, db2 = ft.linear_bwd(w, x, t2, dy, ws)
     assert torch.equal(y1, y2) and torch.equal(dx1, dx2)
     assert torch.equal(da1, da2) and torch.equal(db1, db2)
+
+
+# r = 32 with K = 2048: dA's and dB's split sums are too much work for the dX GEMM's
+# epilogue warps before its first tile (N = 512: two k steps), so they run in a launch of
+# their own; the gradients must meet the same bar.
+WIDE_R = wl.LayerSpec(name="wide_r_256x2048x512", M=256, K=2048, N=512, r_s=16, r=32, alpha=32.0,
+                      n_outlier_cols=10, outlier_gain=20.0, w_std=0.02, plant_rank=4, plant_sigma=6.0,
+                      b_std=0.01, dy_std=1e-2)
+
+
+def test_backward_with_separate_split_sums_matches_oracle():
+    test_backward_matches_oracle(WIDE_R)
+
+
+def test_given_max_equal_to_the_true_max_gives_the_same_forward():
+    # the prologue's per-CTA maxima (reduced by the quantizer) and a caller's max of the
+    # same value are two routes to one g: Y and T must agree bit for bit
+    ft = _ft()
+    inp, _, w = _setup(MID)
+    ws = ft.Workspace(w, MID.M, "cuda")
+    x = inp.x.cuda()
+    y0, t0 = ft.linear_fwd(w, x, ws)
+    y0, t0 = y0.clone(), t0.clone()
+    amax = x.float().abs().max().reshape(1)
+    y1, t1 = ft.linear_fwd(w, x, ws, amax=amax)
+    torch.cuda.synchronize()
+    assert ws.device_status() == 0
+    assert torch.equal(y0, y1) and torch.equal(t0, t1)
+
+
+# M = 384 (one-CTA GEMM kernel) with split sums small enough for its epilogue warps
+# ((N + K) r = 12288 outputs; N = 1024: four k steps in the dX GEMM's first tile)
+SIDE_ONE_CTA = wl.LayerSpec(name="side_one_cta_384x512x1024", M=384, K=512, N=1024, r_s=16, r=8, alpha=8.0,
+                            n_outlier_cols=3, outlier_gain=20.0, w_std=0.02, plant_rank=4, plant_sigma=6.0,
+                            b_std=0.01, dy_std=1e-2)
+
+
+def test_backward_one_cta_gemm_with_side_split_sums_matches_oracle():
+    test_backward_matches_oracle(SIDE_ONE_CTA)
