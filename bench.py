@@ -519,7 +519,20 @@ def main():
     def bwd_kernels():
         ft.linear_bwd(w, x, t, dy, ws, dx=dx, da=da, db=db)
 
-    graph = graph_k = graph_f = graph_b = graph_f1 = None
+    # the same layer with Q(R)^T's codes dropped: the dX GEMM transposes Q(R) on the fly
+    w_xp = ft.drop_transposed_codes(w)
+    xp_ev = (E(), E())
+    for ev in xp_ev:
+        ev.record()
+
+    def bwd_xpose_kernels():
+        ft.linear_bwd(w_xp, x, t, dy, ws, dx=dx, da=da, db=db)
+
+    def bwd_xpose_with_events():  # the dX GEMM is the backward's last GEMM launch
+        ft.time_next_launch(ft.FT_KERNEL_GEMM, xp_ev[0], xp_ev[1])
+        ft.linear_bwd(w_xp, x, t, dy, ws, dx=dx, da=da, db=db)
+
+    graph = graph_k = graph_f = graph_b = graph_f1 = graph_bx = graph_bxk = None
     launches_per_step = None
     if args.graph:
         # One step (forward + backward: all of the library's kernels) captured once as a
@@ -545,8 +558,14 @@ def main():
         fwd_1x16_kernels()
         with torch.cuda.graph(graph_f1):
             fwd_1x16_kernels()
+        bwd_xpose_kernels()
+        graph_bx, graph_bxk = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph_bx):
+            bwd_xpose_kernels()
+        with torch.cuda.graph(graph_bxk):
+            bwd_xpose_with_events()
         for _ in range(args.warmup):
-            for g_ in (graph, graph_k, graph_f, graph_b, graph_f1):
+            for g_ in (graph, graph_k, graph_f, graph_b, graph_f1, graph_bx, graph_bxk):
                 flush.zero_()
                 g_.replay()
         torch.cuda.synchronize()
@@ -591,9 +610,10 @@ def main():
         torch.cuda.synchronize()
         ms_per_step_events = sum(ev_ks[i].elapsed_time(ev_ke[i]) for i in range(Kst)) / Kst
         # per-pass pass: the forward alone, then the backward alone, as many steps each
-        pass_ms = {"fwd": [], "bwd": [], "fwd_1x16": []}
+        pass_ms = {"fwd": [], "bwd": [], "fwd_1x16": [], "bwd_xpose": []}
         for name, g_, fn in (("fwd", graph_f, fwd_kernels), ("bwd", graph_b, bwd_kernels),
-                             ("fwd_1x16", graph_f1, fwd_1x16_kernels)):
+                             ("fwd_1x16", graph_f1, fwd_1x16_kernels),
+                             ("bwd_xpose", graph_bx, bwd_xpose_kernels)):
             for i in range(Kst):
                 flush.zero_()
                 ev_ks[i].record()
@@ -604,6 +624,16 @@ def main():
                 ev_ke[i].record()
             torch.cuda.synchronize()
             pass_ms[name] = [ev_ks[i].elapsed_time(ev_ke[i]) for i in range(Kst)]
+        # the transposing dX GEMM alone, by its launch events
+        xp_gemm_ms = []
+        for i in range(Kst):
+            flush.zero_()
+            if graph_bxk is not None:
+                graph_bxk.replay()
+            else:
+                bwd_xpose_with_events()
+            torch.cuda.synchronize()
+            xp_gemm_ms.append(xp_ev[0].elapsed_time(xp_ev[1]))
     if ws.device_status() != 0:
         raise RuntimeError("device status reports a timeout in the timed region")
 
@@ -690,6 +720,13 @@ def main():
                          "bwd_ms": bwd_ms, "bwd_tflops": fl_b / (bwd_ms * 1e-3) / 1e12,
                          "fwd_1x16_ms": statistics.median(pass_ms["fwd_1x16"]),
                          "timing": f"median of {Kst} replays of a forward-only / backward-only graph"},
+            "xpose_on_the_fly": {
+                "what": "backward with Q(R)^T's codes dropped: the dX GEMM transposes Q(R)'s tiles in "
+                        "shared memory (section 3.2)",
+                "bwd_ms": statistics.median(pass_ms["bwd_xpose"]), "bwd_ms_stored_copy": bwd_ms,
+                "dx_gemm_ms": statistics.mean(xp_gemm_ms),
+                "dx_gemm_ms_stored_copy": statistics.mean(gemm_ms[1::2]),
+                "bytes_saved": N * K // 2 + N * K // 256},
             "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
             "gpu_launches": launches,
             "launch_mode": "cuda_graph_replay" if graph is not None else "stream",

@@ -172,7 +172,13 @@ ft_status check_layer(const ft_linear* L) {
     if (L->r_s % 8 || L->r % 8) return FT_ERR_SHAPE;  // factor rows move in 16-byte pieces
     if (L->N % 256 || L->K % 256) return FT_ERR_SHAPE;
     FT_TRY(check_fp4(L->qr, L->N, L->K, true));
-    FT_TRY(check_fp4(L->qr_t, L->K, L->N, true));
+    if (L->qr_t.codes) {
+        FT_TRY(check_fp4(L->qr_t, L->K, L->N, true));
+    } else {  // Q(R)^T transposed on the fly from Q(R)'s codes: only its scale layout is kept
+        if (!L->qr_t.sf_mma || !L->qr_t.g) return FT_ERR_INVALID_ARG;
+        if (L->qr_t.rows != L->K || L->qr_t.cols != L->N) return FT_ERR_SHAPE;
+        if (!aligned16(L->qr_t.sf_mma) || (reinterpret_cast<uintptr_t>(L->qr_t.g) & 3u)) return FT_ERR_ALIGN;
+    }
     if (L->r_s > 0 && (!L->ls_down || !L->ls_up)) return FT_ERR_INVALID_ARG;
     if (L->r > 0 && (!L->lora_a || !L->lora_b)) return FT_ERR_INVALID_ARG;
     if ((L->ls_down && !aligned16(L->ls_down)) || (L->ls_up && !aligned16(L->ls_up)) ||
@@ -227,19 +233,29 @@ ft_status quantize_operand(const void* x, int64_t rows, int64_t cols, int64_t ld
     return FT_OK;
 }
 
+// CTA pairs (256 x 256 tiles) when M allows, single CTAs (128 x 256) otherwise.
+bool pair_gemm(int64_t M, const DeviceInfo& dev) { return (M % 256) == 0 && dev.num_sms >= 2; }
+
 // One 4-bit GEMM with its low-rank tail: out[M, N] from A (M x K) and B (N x K); with
-// act_out, also act_out = bf16(gelu_tanh(out)) and max |act_out| into *act_amax.
+// act_out, also act_out = bf16(gelu_tanh(out)) and max |act_out| into *act_amax.  When
+// b.codes is null, b_src holds B's codes transposed ([K, N/2] bytes: the stored Q(R) for
+// the dX GEMM) and the GEMM transposes its tiles in shared memory; b.sf_mma is B's own.
 ft_status run_gemm(const uint8_t* a_codes, const uint8_t* a_sf, const float* ga, const ft_fp4& b,
                    const __nv_bfloat16* la, const __nv_bfloat16* lb, int KL, int64_t M, int64_t N,
                    int64_t K, void* out, int* status, const DeviceInfo& dev, cudaStream_t st,
                    void* act_out = nullptr, float* act_amax = nullptr, const void* gelu_in = nullptr,
-                   const ft::LoraFinalizeJob* side = nullptr) {
-    // CTA pairs (256 x 256 tiles) when M allows, single CTAs (128 x 256) otherwise.
-    const bool pair = (M % 256) == 0 && dev.num_sms >= 2;
+                   const ft::LoraFinalizeJob* side = nullptr, const uint8_t* b_src = nullptr) {
+    const bool pair = pair_gemm(M, dev);
     const uint32_t b_rows = pair ? 128 : 256;
+    const bool xpose = b.codes == nullptr;
+    if (xpose && (!b_src || act_out)) return FT_ERR_INVALID_ARG;
     CUtensorMap tA, tB, tLA, tLB;
     FT_TRY(make_tmap(&tA, a_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, K / 2, M, K / 2, 128, 128));
-    FT_TRY(make_tmap(&tB, b.codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, K / 2, N, K / 2, 128, b_rows));
+    if (xpose)  // slabs of 256 rows of B^T by this CTA's b_rows columns (b_rows / 2 bytes)
+        FT_TRY(make_tmap(&tB, b_src, CU_TENSOR_MAP_DATA_TYPE_UINT8, N / 2, K, N / 2, b_rows / 2, 256,
+                         pair ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B));
+    else
+        FT_TRY(make_tmap(&tB, b.codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, K / 2, N, K / 2, 128, b_rows));
     if (KL > 0) {
         FT_TRY(make_tmap(&tLA, la, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, KL, M, KL * 2, 64, 128));
         FT_TRY(make_tmap(&tLB, lb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, KL, N, KL * 2, 64, b_rows));
@@ -273,6 +289,7 @@ ft_status run_gemm(const uint8_t* a_codes, const uint8_t* a_sf, const float* ga,
         g.side0 = side[0];
         g.side1 = side[1];
     }
+    g.xpose = xpose ? 1 : 0;
     if (pair)
         FT_CUDA(ft::launch_gemm_fp4_lowrank_pair(tA, tB, tLA, tLB, tOut, tAct, g, dev.num_sms, st));
     else
@@ -685,7 +702,8 @@ ft_status linear_bwd_impl(const ft_linear* L, const void* x_dev, const float* t_
     }
     // The dX GEMM goes last: the GEMM's operand and output traffic would evict G from L2.
     FT_TRY(run_gemm(W + w.qg_codes, W + w.qg_sf, scal + SC_G_G, L->qr_t, bf(W + w.ucat), bf(W + w.dntcat), KL,
-                    M, K, N, dx_dev, status, dev, st, nullptr, nullptr, gelu_in, side ? fin : nullptr));
+                    M, K, N, dx_dev, status, dev, st, nullptr, nullptr, gelu_in, side ? fin : nullptr,
+                    L->qr.codes));
     return FT_OK;
 }
 

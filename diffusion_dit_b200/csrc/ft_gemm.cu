@@ -21,9 +21,14 @@
 // Warp roles (320 threads): warp 0 = TMA producer, warp 1 = MMA issuer (and TMEM
 // owner), warps 2..5 = epilogue, warps 6..9 = scale writers (warp w reaches TMEM lanes
 // 32 (w % 4) .. +31).
+//
+// With XP (the dX GEMM of section 3.2 without a stored Q(R)^T) the producer loads B's
+// untransposed slab, 256 reduction rows x 128 bytes, into the B slot and the scale writers
+// transpose it in place (ft_xpose.cuh) before they arrive on SF_READY.
 #include "ft_internal.h"
 #include "ft_ptx.cuh"
 #include "ft_sidejobs.cuh"
+#include "ft_xpose.cuh"
 
 namespace ft {
 namespace gemm {
@@ -68,11 +73,13 @@ constexpr int BAR_TMEM_FULL = 2 * STAGES;
 constexpr int BAR_TMEM_EMPTY = 2 * STAGES + 1;
 constexpr int BAR_FINAL = 2 * STAGES + 2;
 __host__ __device__ constexpr int BAR_SF_READY(int s) { return 2 * STAGES + 3 + s; }
-constexpr int NUM_BARS = 3 * STAGES + 3;
+constexpr int BAR_XREAD = 3 * STAGES + 3;  // XP: the scale warps have read the raw B slab
+constexpr int NUM_BARS = 3 * STAGES + 4;
 constexpr int OFF_TMEM_SLOT = 8 * 16;   // inside the barrier area
 constexpr int OFF_ABORT = 8 * 16 + 4;
+static_assert(8 * NUM_BARS <= OFF_TMEM_SLOT, "barriers overlap the TMEM slot");
 
-template <int EPI>
+template <int EPI, bool XP>
 __global__ void __launch_bounds__(THREADS, 1)
     gemm_fp4_lowrank_kernel(const __grid_constant__ CUtensorMap tmA,
                             const __grid_constant__ CUtensorMap tmB,
@@ -107,6 +114,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         mbar_init(sm.bar(BAR_TMEM_FULL), 1);
         mbar_init(sm.bar(BAR_TMEM_EMPTY), 4);
         mbar_init(sm.bar(BAR_FINAL), 1);
+        mbar_init(sm.bar(BAR_XREAD), 4);
         *abort_flag = 0;
         fence_mbar_init();
         fence_proxy_async_smem();
@@ -147,7 +155,10 @@ __global__ void __launch_bounds__(THREADS, 1)
                     const uint32_t st = sm.stage(s);
                     mbar_arrive_expect_tx(full, STAGE_BYTES);
                     tma_load_2d(st, &tmA, full, kt * BK_BYTES, m0);
-                    tma_load_2d(st + OFF_B, &tmB, full, kt * BK_BYTES, n0);
+                    if constexpr (XP)  // B^T rows kt*256.., the bytes of the tile's 256 columns
+                        tma_load_2d(st + OFF_B, &tmB, full, n0 / 2, kt * 256);
+                    else
+                        tma_load_2d(st + OFF_B, &tmB, full, kt * BK_BYTES, n0);
                     bulk_load(st + OFF_SFA, p.sfa + (static_cast<size_t>(mb) * k64 + kt * 4) * 512,
                               SFA_BYTES, full);
 #pragma unroll
@@ -241,6 +252,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         const int q = warp & 3;
         const uint32_t lane_base = tmem + (static_cast<uint32_t>(32 * q) << 16);
         int it = 0;
+        uint32_t xr = 0;  // XREAD phases passed
         for (int t = blockIdx.x; t < num_tiles && !*abort_flag; t += gridDim.x) {
             bool ok = true;
             for (int j = 0; j < KT + KLS; ++j, ++it) {
@@ -265,6 +277,22 @@ __global__ void __launch_bounds__(THREADS, 1)
                     tmem_st_32x32b_x16(lane_base + COL_SFA + 16 * s, va);
                     tmem_st_32x32b_x16(lane_base + COL_SFB + 32 * s, vb0);
                     tmem_st_32x32b_x16(lane_base + COL_SFB + 32 * s + 16, vb1);
+                    if constexpr (XP) {
+                        const uint32_t slab = sm.stage(s) + OFF_B;
+                        xpose::Regs<128> rg;
+                        xpose::load<128>(slab, q, lane, rg);
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(sm.bar(BAR_XREAD));
+                        xpose::transpose<128>(lane, rg);
+                        if (!mbar_wait(sm.bar(BAR_XREAD), xr & 1, abort_flag, p.status)) {
+                            tmem_st_wait();
+                            ok = false;
+                            break;
+                        }
+                        ++xr;
+                        xpose::store<128>(slab, q, lane, rg);
+                        fence_proxy_async_smem();  // ordinary stores, read next by the MMA
+                    }
                     tmem_st_wait();
                 }
                 tc_fence_before();
@@ -390,17 +418,17 @@ __global__ void __launch_bounds__(THREADS, 1)
 
 namespace {
 
-// One epilogue variant: its own instantiation, its shared-memory opt-in set once.
-template <int EPI>
+// One variant: its own instantiation, its shared-memory opt-in set once.
+template <int EPI, bool XP>
 cudaError_t launch_variant(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmLA,
                            const CUtensorMap& tmLB, const CUtensorMap& tmOut, const CUtensorMap& tmAct,
                            const GemmFp4Args& args, int grid, cudaStream_t stream) {
     using namespace gemm;
     static const cudaError_t attr = cudaFuncSetAttribute(
-        gemm_fp4_lowrank_kernel<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+        gemm_fp4_lowrank_kernel<EPI, XP>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
     if (attr != cudaSuccess) return attr;
-    return launch_k(gemm_fp4_lowrank_kernel<EPI>, dim3(grid), dim3(THREADS), SMEM_BYTES, stream, tmA, tmB, tmLA,
-                    tmLB, tmOut, tmAct, args);
+    return launch_k(gemm_fp4_lowrank_kernel<EPI, XP>, dim3(grid), dim3(THREADS), SMEM_BYTES, stream, tmA, tmB,
+                    tmLA, tmLB, tmOut, tmAct, args);
 }
 
 }  // namespace
@@ -413,10 +441,19 @@ cudaError_t launch_gemm_fp4_lowrank(const CUtensorMap& tmA, const CUtensorMap& t
     const int tiles = (args.M / BM) * (args.N / BN);
     const int grid = tiles < num_sms ? tiles : num_sms;
     before_launch(K_GEMM, stream);
-    const cudaError_t le =
-        args.gelu_in  ? launch_variant<kEpiGeluBwd>(tmA, tmB, tmLA, tmLB, tmOut, tmAct, args, grid, stream)
-        : args.act_out ? launch_variant<kEpiGelu>(tmA, tmB, tmLA, tmLB, tmOut, tmAct, args, grid, stream)
-                       : launch_variant<kEpiPlain>(tmA, tmB, tmLA, tmLB, tmOut, tmAct, args, grid, stream);
+    // the transposing variants serve the backward's dX GEMM (plain or GELU-backward epilogue)
+    cudaError_t le;
+    if (args.xpose)
+        le = args.act_out ? cudaErrorInvalidValue
+             : args.gelu_in
+                 ? launch_variant<kEpiGeluBwd, true>(tmA, tmB, tmLA, tmLB, tmOut, tmAct, args, grid, stream)
+                 : launch_variant<kEpiPlain, true>(tmA, tmB, tmLA, tmLB, tmOut, tmAct, args, grid, stream);
+    else
+        le = args.gelu_in
+                 ? launch_variant<kEpiGeluBwd, false>(tmA, tmB, tmLA, tmLB, tmOut, tmAct, args, grid, stream)
+             : args.act_out
+                 ? launch_variant<kEpiGelu, false>(tmA, tmB, tmLA, tmLB, tmOut, tmAct, args, grid, stream)
+                 : launch_variant<kEpiPlain, false>(tmA, tmB, tmLA, tmLB, tmOut, tmAct, args, grid, stream);
     if (le != cudaSuccess) return le;
     after_launch(K_GEMM, stream);
     return cudaGetLastError();

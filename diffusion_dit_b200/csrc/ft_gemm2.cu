@@ -21,9 +21,15 @@
 // Warp roles: warp 0 = TMA producer, warp 1 = MMA issuer (even CTA) and TMEM owner, then
 // the epilogue warps (4, or 8 for the GELU epilogues: two per TMEM lane quarter, 128
 // columns each), then 4 scale writers.
+//
+// With XP (the dX GEMM of section 3.2 without a stored Q(R)^T) the producer loads B's
+// untransposed slab, 256 reduction rows x 64 bytes, into the B slot, and the scale
+// writers turn it into the K-major tile in place (ft_xpose.cuh) before they arrive on
+// SF_READY: all four read their share first, meet on the XREAD barrier, then write.
 #include "ft_internal.h"
 #include "ft_ptx.cuh"
 #include "ft_sidejobs.cuh"
+#include "ft_xpose.cuh"
 
 namespace ft {
 namespace gemm2 {
@@ -68,12 +74,34 @@ __host__ __device__ constexpr int BAR_SF_READY(int s) { return 2 * STAGES + s; }
 constexpr int BAR_TMEM_FULL = 3 * STAGES;
 constexpr int BAR_TMEM_EMPTY = 3 * STAGES + 1;
 constexpr int BAR_FINAL = 3 * STAGES + 2;
-constexpr int NUM_BARS = 3 * STAGES + 3;
+constexpr int BAR_XREAD = 3 * STAGES + 3;  // XP: the scale warps have read the raw B slab
+constexpr int NUM_BARS = 3 * STAGES + 4;
 constexpr int OFF_TMEM_SLOT = 8 * NUM_BARS;
 constexpr int OFF_ABORT = OFF_TMEM_SLOT + 4;
 static_assert(OFF_ABORT + 4 <= BAR_BYTES, "barrier area overflow");
 
-template <int EPI>
+// XP: one scale warp's share of the in-place transposition of the B slab at `slab`.
+// False if the wait for the other scale warps' reads gave up (the abort flag and status
+// are then set).
+__device__ __forceinline__ bool xpose_share(uint32_t slab, int q, int lane, uint32_t xread, uint32_t& xr,
+                                            volatile int* abort_flag, int* status) {
+    xpose::Regs<64> rg;
+    xpose::load<64>(slab, q, lane, rg);
+    __syncwarp();
+    if (lane == 0) mbar_arrive(xread);
+    xpose::transpose<64>(lane, rg);
+    if (!mbar_wait(xread, xr & 1, abort_flag, status)) return false;
+    ++xr;
+    xpose::store<64>(slab, q, lane, rg);
+    // The stores are complete in this CTA's shared memory once the proxy fence returns;
+    // the MMA reading them (issued by the even CTA) starts only after SF_READY completes,
+    // which needs this warp's arrival below, so the cta-scope arrival suffices (a
+    // cluster-scope release would cost several hundred cycles per stage).
+    fence_proxy_async_smem();
+    return true;
+}
+
+template <int EPI, bool XP>
 __global__ void __launch_bounds__(threads(EPI), 1)
     gemm_fp4_lowrank_pair_kernel(const __grid_constant__ CUtensorMap tmA,
                                  const __grid_constant__ CUtensorMap tmB,
@@ -116,6 +144,7 @@ __global__ void __launch_bounds__(threads(EPI), 1)
         mbar_init(bar(BAR_TMEM_FULL), 1);
         mbar_init(bar(BAR_TMEM_EMPTY), 2 * EPI_WARPS);  // epilogue warps x 2 CTAs (even CTA's copy used)
         mbar_init(bar(BAR_FINAL), 1);
+        mbar_init(bar(BAR_XREAD), 4);  // XP: this CTA's 4 scale warps
         *abort_flag = 0;
         fence_mbar_init();
         fence_proxy_async_smem();
@@ -162,7 +191,10 @@ __global__ void __launch_bounds__(threads(EPI), 1)
                     const uint32_t st = stage(s);
                     mbar_arrive_expect_tx(full, STAGE_BYTES);
                     tma_load_2d(st, &tmA, full, kt * BK_BYTES, m_band * BM);
-                    tma_load_2d(st + OFF_B, &tmB, full, kt * BK_BYTES, n_rows);
+                    if constexpr (XP)  // B^T rows kt*256.., bytes of this CTA's 128 columns
+                        tma_load_2d(st + OFF_B, &tmB, full, n_rows / 2, kt * 256);
+                    else
+                        tma_load_2d(st + OFF_B, &tmB, full, kt * BK_BYTES, n_rows);
                     bulk_load(st + OFF_SFA, p.sfa + (static_cast<size_t>(m_band) * k64 + kt * 4) * 512,
                               SFA_BYTES, full);
 #pragma unroll
@@ -248,6 +280,7 @@ __global__ void __launch_bounds__(threads(EPI), 1)
         const int q = warp & 3;
         const uint32_t lane_base = tmem + (static_cast<uint32_t>(32 * q) << 16);
         int it = 0;
+        uint32_t xr = 0;  // XREAD phases passed
         for (int t = pair; t < num_tiles && !*abort_flag; t += num_pairs) {
             bool ok = true;
             for (int j = 0; j < KT + KLS; ++j, ++it) {
@@ -272,6 +305,13 @@ __global__ void __launch_bounds__(threads(EPI), 1)
                     tmem_st_32x32b_x16(lane_base + COL_SFA + 16 * s, va);
                     tmem_st_32x32b_x16(lane_base + COL_SFB + 32 * s, vb0);
                     tmem_st_32x32b_x16(lane_base + COL_SFB + 32 * s + 16, vb1);
+                    if constexpr (XP) {
+                        if (!xpose_share(stage(s) + OFF_B, q, lane, bar(BAR_XREAD), xr, abort_flag, p.status)) {
+                            tmem_st_wait();
+                            ok = false;
+                            break;
+                        }
+                    }
                     tmem_st_wait();
                 }
                 tc_fence_before();
@@ -415,18 +455,19 @@ __global__ void __launch_bounds__(threads(EPI), 1)
 
 namespace {
 
-// One epilogue variant: its own instantiation, its shared-memory opt-in set once.
-template <int EPI>
+// One variant: its own instantiation, its shared-memory opt-in set once.
+template <int EPI, bool XP>
 cudaError_t launch_variant(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmLA,
                            const CUtensorMap& tmLB, const CUtensorMap& tmOut, const CUtensorMap& tmAct,
                            const GemmFp4Args& args, cudaLaunchConfig_t cfg) {
     using namespace gemm2;
     static const cudaError_t attr = cudaFuncSetAttribute(
-        gemm_fp4_lowrank_pair_kernel<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes(EPI));
+        gemm_fp4_lowrank_pair_kernel<EPI, XP>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes(EPI));
     if (attr != cudaSuccess) return attr;
     cfg.blockDim = dim3(threads(EPI));
     cfg.dynamicSmemBytes = smem_bytes(EPI);
-    return cudaLaunchKernelEx(&cfg, gemm_fp4_lowrank_pair_kernel<EPI>, tmA, tmB, tmLA, tmLB, tmOut, tmAct, args);
+    return cudaLaunchKernelEx(&cfg, gemm_fp4_lowrank_pair_kernel<EPI, XP>, tmA, tmB, tmLA, tmLB, tmOut, tmAct,
+                              args);
 }
 
 }  // namespace
@@ -452,10 +493,16 @@ cudaError_t launch_gemm_fp4_lowrank_pair(const CUtensorMap& tmA, const CUtensorM
     cfg.attrs = at;
     cfg.numAttrs = 2;
     before_launch(K_GEMM, stream);
-    const cudaError_t e =
-        args.gelu_in  ? launch_variant<kEpiGeluBwd>(tmA, tmB, tmLA, tmLB, tmOut, tmAct, args, cfg)
-        : args.act_out ? launch_variant<kEpiGelu>(tmA, tmB, tmLA, tmLB, tmOut, tmAct, args, cfg)
-                       : launch_variant<kEpiPlain>(tmA, tmB, tmLA, tmLB, tmOut, tmAct, args, cfg);
+    // the transposing variants serve the backward's dX GEMM (plain or GELU-backward epilogue)
+    cudaError_t e;
+    if (args.xpose)
+        e = args.act_out ? cudaErrorInvalidValue
+            : args.gelu_in ? launch_variant<kEpiGeluBwd, true>(tmA, tmB, tmLA, tmLB, tmOut, tmAct, args, cfg)
+                           : launch_variant<kEpiPlain, true>(tmA, tmB, tmLA, tmLB, tmOut, tmAct, args, cfg);
+    else
+        e = args.gelu_in ? launch_variant<kEpiGeluBwd, false>(tmA, tmB, tmLA, tmLB, tmOut, tmAct, args, cfg)
+            : args.act_out ? launch_variant<kEpiGelu, false>(tmA, tmB, tmLA, tmLB, tmOut, tmAct, args, cfg)
+                           : launch_variant<kEpiPlain, false>(tmA, tmB, tmLA, tmLB, tmOut, tmAct, args, cfg);
     after_launch(K_GEMM, stream);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();

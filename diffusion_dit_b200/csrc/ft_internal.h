@@ -73,16 +73,21 @@ struct GemmFp4Args {
     // optional side jobs for the epilogue warps, run before their first tile (they wait
     // for the first accumulator anyway): the adapter gradients' split sums
     LoraFinalizeJob side0, side1;
+    // non-zero: tmB holds B^T untransposed ([K rows, N/2 bytes], box 256 rows), and the
+    // scale warps transpose each tile in shared memory (ft_xpose.cuh); sfb is B's layout
+    int xpose;
 };
 
-// tmOut (and tmAct): bf16 [M, N] output, box 32 x 32, 64-byte swizzle.
+// tmOut (and tmAct): bf16 [M, N] output, box 32 x 32, 64-byte swizzle.  tmB: 128 x 256
+// (bytes x rows) with the 128-byte swizzle; with xpose, 128 bytes x 256 rows of B^T.
 cudaError_t launch_gemm_fp4_lowrank(const CUtensorMap& tmA, const CUtensorMap& tmB,
                                     const CUtensorMap& tmLA, const CUtensorMap& tmLB,
                                     const CUtensorMap& tmOut, const CUtensorMap& tmAct,
                                     const GemmFp4Args& args, int num_sms, cudaStream_t stream);
 
 // The same GEMM computed by CTA pairs (cta_group::2), 256 x 256 tiles; needs M % 256 == 0.
-// tmB / tmLB boxes are 128 rows: each CTA of a pair loads half of the tile's N.
+// tmB / tmLB boxes are 128 rows: each CTA of a pair loads half of the tile's N (with
+// xpose, tmB's box is 64 bytes x 256 rows of B^T, 64-byte swizzle; without, 128 x 128 bytes).
 cudaError_t launch_gemm_fp4_lowrank_pair(const CUtensorMap& tmA, const CUtensorMap& tmB,
                                          const CUtensorMap& tmLA, const CUtensorMap& tmLB,
                                          const CUtensorMap& tmOut, const CUtensorMap& tmAct,

@@ -133,8 +133,8 @@ def _require_cuda(*ts):
 class QuantizedMatrix:
     """Device tensors of one 16x16-block quantized matrix (see ft_fp4)."""
 
-    codes: torch.Tensor            # uint8 [rows, cols/2]
-    scales: torch.Tensor           # uint8 [rows/16, cols/16]
+    codes: Optional[torch.Tensor]   # uint8 [rows, cols/2] (None: see drop_transposed_codes)
+    scales: Optional[torch.Tensor]  # uint8 [rows/16, cols/16]
     sf_mma: Optional[torch.Tensor]  # uint8 [rows * cols / 16] or None
     g: torch.Tensor                # float32 [1]
     rows: int
@@ -149,9 +149,9 @@ class QuantizedMatrix:
             g=torch.empty(1, dtype=torch.float32, device=device), rows=rows, cols=cols)
 
     def c_struct(self) -> FtFp4:
-        return FtFp4(self.codes.data_ptr(), self.scales.data_ptr(),
-                     self.sf_mma.data_ptr() if self.sf_mma is not None else None,
-                     self.g.data_ptr(), self.rows, self.cols)
+        def ptr(t):
+            return t.data_ptr() if t is not None else None
+        return FtFp4(ptr(self.codes), ptr(self.scales), ptr(self.sf_mma), self.g.data_ptr(), self.rows, self.cols)
 
 
 def quantize_block16(x: torch.Tensor, amax: Optional[torch.Tensor] = None, with_sf: bool = False,
@@ -232,12 +232,22 @@ class LinearWeights:
 
 
 def prepare_weights(residual: torch.Tensor, ls_up: torch.Tensor, ls_down: torch.Tensor,
-                    lora_a: torch.Tensor, lora_b: torch.Tensor, lora_scale: float) -> LinearWeights:
+                    lora_a: torch.Tensor, lora_b: torch.Tensor, lora_scale: float,
+                    transpose_on_the_fly: bool = False) -> LinearWeights:
     """Q(R) offline (section 3.1) with its transposed copy (section 3.2), on the GPU.
-    ``residual`` is the fp32 (or bf16) R [N, K] on the device."""
+    ``residual`` is the fp32 (or bf16) R [N, K] on the device.  With
+    ``transpose_on_the_fly`` the transposed codes are not kept (drop_transposed_codes)."""
     qr, qr_t, _ = quantize_block16(residual.contiguous(), with_sf=True, transposed=True)
-    return LinearWeights(qr, qr_t, ls_down.contiguous(), ls_up.contiguous(), lora_a.contiguous(),
-                         lora_b.contiguous(), float(lora_scale))
+    w = LinearWeights(qr, qr_t, ls_down.contiguous(), ls_up.contiguous(), lora_a.contiguous(),
+                      lora_b.contiguous(), float(lora_scale))
+    return drop_transposed_codes(w) if transpose_on_the_fly else w
+
+
+def drop_transposed_codes(w: LinearWeights) -> LinearWeights:
+    """The same layer without Q(R)^T's codes and scale grid (N*K/2 + N*K/256 bytes): the
+    backward's dX GEMM then transposes Q(R)'s codes tile by tile in shared memory (section
+    3.2).  Q(R)^T's tensor-core scale layout and g are kept.  Shares every other tensor."""
+    return dataclasses.replace(w, qr_t=dataclasses.replace(w.qr_t, codes=None, scales=None))
 
 
 class Workspace:

@@ -88,7 +88,11 @@ typedef struct {
  * One frozen-backbone linear layer with its adapter (Eq. 1-2).
  *   qr      : Q(R), rows = N, cols = K, sf_mma required.
  *   qr_t    : Q(R)^T, rows = K, cols = N, sf_mma required (written by
- *             fourtune_quantize_block16 with an out_t argument).
+ *             fourtune_quantize_block16 with an out_t argument).  codes (and
+ *             scales) may be NULL: the backward's dX GEMM then transposes Q(R)'s
+ *             codes tile by tile in shared memory (section 3.2, transposition on
+ *             the fly), which saves the second copy of the codes (N*K/2 bytes);
+ *             sf_mma and g stay required.
  *   ls_down : bf16 [r_s, K]   (L_stab = ls_up * ls_down)
  *   ls_up   : bf16 [N, r_s]
  *   lora_a  : bf16 [r, K]
