@@ -14,8 +14,9 @@
 // complete on its own FULL barrier; its four scale warps write the scale factors into its
 // own tensor memory (tcgen05.st) and arrive on the even CTA's SF_READY barrier, which the
 // MMA issuer waits on, so SF_READY also certifies that both CTAs' operands have landed.
-// The MMA issuer's commits arrive on both CTAs' EMPTY barriers (one commit per CTA) and
-// on both TMEM_FULL barriers; each CTA drains its own 128 x 256 accumulator and releases
+// The MMA issuer's commits arrive on both CTAs' EMPTY barriers and on both TMEM_FULL
+// barriers (one commit each, multicast to the pair: half the tensor-pipe time of a commit
+// per CTA); each CTA drains its own 128 x 256 accumulator and releases
 // it on the even CTA's TMEM_EMPTY.  No load is multicast.
 //
 // Warp roles: warp 0 = TMA producer, warp 1 = MMA issuer (even CTA) and TMEM owner, then
@@ -257,16 +258,14 @@ __global__ void __launch_bounds__(threads(EPI), 1)
                         for (int i = 0; i < nk16; ++i)
                             mma_bf16_pair(tmem + COL_ACC, ad + 2 * i, bd + 2 * i, idesc16, 1);
                     }
-                    tc_commit_pair(bar(BAR_EMPTY(s)));
-                    tc_commit_pair(mapa_shared(bar(BAR_EMPTY(s)), 1));
+                    tc_commit_pair_both(bar(BAR_EMPTY(s)));
                     if (++s == STAGES) {
                         s = 0;
                         ph ^= 1;
                     }
                 }
                 if (!ok) break;
-                tc_commit_pair(bar(BAR_TMEM_FULL));
-                tc_commit_pair(mapa_shared(bar(BAR_TMEM_FULL), 1));
+                tc_commit_pair_both(bar(BAR_TMEM_FULL));
             }
             // every MMA has retired (in both CTAs' tensor memory) before the pair tears down
             tc_commit_pair(bar(BAR_FINAL));

@@ -320,6 +320,16 @@ __device__ __forceinline__ void tc_commit_pair(uint32_t bar) {
                  : "memory");
 }
 
+// The same commit arriving once on the mbarrier at this shared-memory offset in both CTAs
+// of the pair (CTA mask 0b11): one tensor-pipe commit instead of two.  An arrival, not a
+// data movement: no memory is read through the multicast.
+__device__ __forceinline__ void tc_commit_pair_both(uint32_t bar) {
+    asm volatile(
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(bar),
+        "h"(static_cast<uint16_t>(3))
+        : "memory");
+}
+
 // Shared-memory matrix descriptor, K-major, 128-byte swizzle: rows of 128 bytes, groups
 // of 8 rows 1024 bytes apart.  Stepping along K inside the 128-byte row is done by
 // advancing the start address (16-byte units).

@@ -97,6 +97,42 @@ def test_linear_rejects_bad_arguments_on_host(lib):
                nws, None) == 1
 
 
+def test_transposed_codes_may_be_absent_but_not_their_scale_layout(lib):
+    # Q(R)^T transposed on the fly in the dX GEMM: qr_t.codes (and scales) NULL is valid;
+    # qr_t's tensor-core scale layout and g stay required, with their shape and alignment.
+    # Every call returns before any device work: an accepted layer stops at the misaligned
+    # x pointer (3), or at M = 96 (2) where the case itself is an alignment error.
+    bwd = lib.fourtune_linear_bwd
+    ws = 0x1000000
+
+    def call(L, M=128, x=0x400008):
+        return bwd(ctypes.byref(L), x, 0x600000, 0x650000, M, None, 0x700000, 0x800000, 0x900000, ws,
+                   1 << 30, None)
+
+    def onfly():
+        L = _layer()
+        L.qr_t.codes = None
+        L.qr_t.scales = None
+        return L
+
+    assert call(onfly()) == 3                 # accepted: the layer check passes
+    L = onfly()
+    L.qr_t.sf_mma = None
+    assert call(L) == 1
+    L = onfly()
+    L.qr_t.g = None
+    assert call(L) == 1
+    L = onfly()
+    L.qr_t.rows = 128                         # Q(R)^T must be K x N
+    assert call(L) == 2
+    L = onfly()
+    L.qr_t.sf_mma = 0x200008                  # misaligned scale layout (accepted would give 2)
+    assert call(L, M=96, x=0x400000) == 3
+    L = onfly()
+    L.qr.codes = None                         # Q(R)'s codes are the transposition's source
+    assert call(L) == 1
+
+
 def test_workspace_grows_with_tokens(lib):
     L = _layer(N=512, K=512, r_s=16, r=8)
     a = lib.fourtune_linear_workspace_bytes(ctypes.byref(L), 128)
