@@ -1,23 +1,33 @@
 """Benchmark of the W4A4G4 triple-branch linear layer (FourTune, arXiv 2607.05711).
 
-One step = the whole hot path once over one batch: the forward (tensor max, 16x16
-block quantization of X, the low-rank down-projection, the 4-bit GEMM with the up-
-projections fused in) and the backward (the same for G, the dX GEMM through Q(R)^T,
-and the adapter gradients dA, dB).  Workload: the FLUX.1-dev attention QKV projection,
-4608 tokens (4096 image + 512 text) x 3072 -> 9216, stabilizer rank 32, LoRA rank 16,
-synthetic inputs and random-init weights of that shape (see workloads.py).
+One step = the whole hot path once over one batch, for every layer of the workload: the
+forward (tensor max, 16x16 block quantization of X fused with the low-rank down-
+projection, the 4-bit GEMM with the up-projections in its accumulator) and the backward
+(the same for G, the dX GEMM through Q(R)^T, the adapter gradients dA, dB).  Default
+workload: the linears of a FLUX.1-dev single-stream block at batch 2 x 4608 tokens --
+linear1 9216 x 3072 -> 21504 (fused QKV + MLP-up) and linear2 9216 x 15360 -> 3072,
+stabilizer rank 32, LoRA rank 64 -- forward through both, then backward through both,
+synthetic inputs (independent per layer) and random-init weights of that shape
+(workloads.py).  The same line carries the quantizer-only sweep (16x16-block quantizer
+with its fused rank-32 down-projection, bf16 4608x3072 ... 36864x21504) in GB/s against
+HBM.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload single|qkv|mlp|mlp_up|mlp_down|single_l1|single_l2]
+                    [--tokens M] [--profile]
 
-N > 1 runs data-parallel under torchrun: each rank processes its own 4608 tokens
-(weak scaling) and the adapter gradients are summed with an NCCL all-reduce.  The
-reference arm times the CPU oracle (the only reference this method has) on a bounded
-sample of the same workload.  One JSON line on rank 0.
+N > 1 runs data-parallel under torchrun: each rank processes its own batch (weak
+scaling) and the adapter gradients are summed with an NCCL all-reduce.  The reference arm
+times the CPU oracle (the only reference this method has) on a bounded sample of the same
+workload.  --tokens M replaces the token count (a smaller case for profilers);
+--profile runs the plain step only (no graphs, no side measurements), for ncu.  One JSON
+line on rank 0.
 """
 from __future__ import annotations
 
 import argparse
 import datetime
+import hashlib
 import json
 import os
 import statistics
@@ -32,10 +42,23 @@ METRIC = "W4A4G4 linear fwd+bwd TFLOPS & % FP4 roofline; quantizer GB/s vs HBM"
 NOMINAL_FP4_OVER_BF16 = 4.0   # 9 / 2.25 PFLOP/s dense (B200 spec ratio)
 NOMINAL_FP4_TFLOPS = 9000.0   # B200 dense FP4 spec
 
-# single-layer workloads (one FourTune linear, forward + backward); the default is the
-# attention QKV projection, the others are the MLP and single-stream layers
-WORKLOADS = {"qkv": "FLUX_QKV", "mlp_up": "FLUX_MLP_UP", "mlp_down": "FLUX_MLP_DOWN",
-             "single_l1": "FLUX_SS_L1", "single_l2": "FLUX_SS_L2"}
+# workload -> (description, layer specs in forward order); "mlp" is the fused MLP pair
+WORKLOADS = {
+    "single": ("flux_single_stream_block linear1 9216x3072->21504 + linear2 9216x15360->3072",
+               ["FLUX_SS_L1", "FLUX_SS_L2"]),
+    "qkv": ("flux_qkv 4608x3072->9216", ["FLUX_QKV"]),
+    "mlp_up": ("flux_mlp_up 4608x3072->12288", ["FLUX_MLP_UP"]),
+    "mlp_down": ("flux_mlp_down 4608x12288->3072", ["FLUX_MLP_DOWN"]),
+    "single_l1": ("flux_single_l1 9216x3072->21504", ["FLUX_SS_L1"]),
+    "single_l2": ("flux_single_l2 9216x15360->3072", ["FLUX_SS_L2"]),
+}
+DEFAULT_WORKLOAD = "single"
+
+# ncu DRAM read + write per launch of the 4-bit GEMM (mean over the step's GEMM launches)
+# on a workload, with the hash of the GEMM's sources the counters were taken from: the
+# figure is reported only while the sources still hash to that value.
+GEMM_DRAM_BYTES = {}
+GEMM_SOURCES = ("ft_gemm2.cu", "ft_ptx.cuh")
 
 
 def layer_flops(M, K, N, r_s, r):
@@ -62,6 +85,18 @@ def peaks():
         return float(d["hbm_gbs"]), float(d["bf16_tflops"]), "measured"
     except Exception:
         return 6650.0, 1590.0, "fallback"
+
+
+def gemm_sources_hash():
+    src = b"".join(open(os.path.join(ROOT, "diffusion_dit_b200", "csrc", f), "rb").read() for f in GEMM_SOURCES)
+    return hashlib.sha256(src).hexdigest()[:16]
+
+
+def gemm_traffic(workload):
+    rec = GEMM_DRAM_BYTES.get(workload)
+    if not rec or rec[1] != gemm_sources_hash():
+        return None
+    return rec[0]
 
 
 class ClockSampler:
@@ -113,62 +148,102 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(rows)}
 
 
-def run_reference(args, spec):
-    """The reference arm: the CPU oracle as it stands, on a bounded token sample."""
-    import numpy as np
-    import torch
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        return max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:
+        return os.cpu_count() or 1
 
-    from diffusion_dit_b200 import prep, workloads as wl
+
+def specs_of(args):
+    from diffusion_dit_b200 import workloads as wl
+    desc, names = WORKLOADS[args.workload]
+    specs = [getattr(wl, n) for n in names]
+    if args.tokens:
+        import dataclasses
+        specs = [dataclasses.replace(s, name=f"{s.name}@M{args.tokens}", M=args.tokens) for s in specs]
+        desc = f"{desc} with M={args.tokens} tokens"
+    return desc, specs
+
+
+def workload_config(args, desc, specs):
+    return {"workload": f"{desc}, fwd+bwd", "layers": [
+        {"name": s.name, "M": s.M, "K": s.K, "N": s.N, "stabilizer_rank": s.r_s, "lora_rank": s.r}
+        for s in specs], "M_tokens_per_gpu": specs[0].M,
+        "l2": "flushed between steps (512 MiB write, outside the step events); the single-stream "
+              "layers' operands are larger than L2"}
+
+
+def oracle_layers(specs, splits, rows):
+    """The oracle's view of each layer on a bounded token sample (the full weights)."""
+    from diffusion_dit_b200 import workloads as wl
     from oracle import fourtune_oracle as ora
+    out = []
+    for spec, split in zip(specs, splits):
+        inp = wl.make_layer_inputs(spec, seed=0, rows=rows)
+        layer = ora.Layer(qr=ora.quantize_residual(split.residual), ls_up=split.ls_up, ls_down=split.ls_down,
+                          lora_a=inp.lora_a, lora_b=inp.lora_b, lora_scale=spec.lora_scale)
+        out.append((inp, layer))
+    return out
+
+
+def oracle_pass(layers):
+    from oracle import fourtune_oracle as ora
+    for inp, layer in layers:
+        ora.linear_fwd(inp.x, layer)
+    for inp, layer in reversed(layers):
+        ora.linear_bwd(inp.x, inp.dy, layer)
+
+
+def sample_flops(specs, rows):
+    return sum(sum(layer_flops(rows, s.K, s.N, s.r_s, s.r)) for s in specs)
+
+
+def run_reference(args, desc, specs):
+    """The reference arm: the CPU oracle as it stands, on a bounded token sample."""
+    from diffusion_dit_b200 import prep
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
     rows = args.ref_rows
-    inp = wl.make_layer_inputs(spec, seed=0, rows=rows)
-    split = prep.svd_split(inp.w, spec.r_s)
-    layer = ora.Layer(qr=ora.quantize_residual(split.residual), ls_up=split.ls_up, ls_down=split.ls_down,
-                      lora_a=inp.lora_a, lora_b=inp.lora_b, lora_scale=spec.lora_scale)
+    from diffusion_dit_b200 import workloads as wl
+    splits = [prep.svd_split(wl.make_layer_inputs(s, seed=0, rows=rows).w, s.r_s) for s in specs]
+    layers = oracle_layers(specs, splits, rows)
     threads = blas_threads()
-
-    def one():
-        ora.linear_fwd(inp.x, layer)
-        ora.linear_bwd(inp.x, inp.dy, layer)
-
     for _ in range(args.warmup):
-        one()
+        oracle_pass(layers)
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        one()
+        oracle_pass(layers)
     dt = (time.perf_counter() - t0) / args.steps
-    fp4, bf = layer_flops(rows, spec.K, spec.N, spec.r_s, spec.r)
-    value = (fp4 + bf) / dt / 1e12
-    sample = f"{rows} of {spec.M} tokens, full weights; oracle quantize+fwd+bwd (fp64 products)"
+    value = sample_flops(specs, rows) / dt / 1e12
+    sample = (f"{rows} tokens of each layer's {specs[0].M}, full weights; oracle quantize + fwd + bwd "
+              f"(fp64 products) through every layer")
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": workload_config(spec),
+            "config": workload_config(args, desc, specs),
             "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
 
-def gemm_traffic():
-    """DRAM bytes per launch of the 4-bit GEMM from the committed ncu summary, or None
-    when the kernel's sources have changed since those counters were taken."""
-    import hashlib
-    import re
-    here = os.path.dirname(os.path.abspath(__file__))
-    try:
-        text = open(os.path.join(here, "profiles", "gemm_fp4_lowrank_pair_kernel.md")).read()
-        m = re.search(r"traffic_bytes_per_launch: (\d+) sources_sha256_16: ([0-9a-f]{16})", text)
-        src = b"".join(open(os.path.join(here, "diffusion_dit_b200", "csrc", f), "rb").read()
-                       for f in ("ft_gemm2.cu", "ft_ptx.cuh"))
-    except OSError:
-        return None
-    if not m or hashlib.sha256(src).hexdigest()[:16] != m.group(2):
-        return None
-    return int(m.group(1))
+def cpu_baseline(specs, splits, budget_s=12.0, rows=128):
+    """The oracle timed on the host cores on a bounded sample (rank 0, N = 1)."""
+    layers = oracle_layers(specs, splits, rows)
+    n, t0 = 0, time.perf_counter()
+    while True:
+        oracle_pass(layers)
+        n += 1
+        if time.perf_counter() - t0 >= budget_s:
+            break
+    dt = (time.perf_counter() - t0) / n
+    return {"value": sample_flops(specs, rows) / dt / 1e12, "unit": "TFLOP/s", "cores": blas_threads(),
+            "kind": "oracle",
+            "sample": f"{rows} of {specs[0].M} tokens of every layer with the full weights, {n} oracle passes "
+                      f"(quantize + fwd + bwd, fp64 products) in {time.perf_counter() - t0:.1f} s"}
 
 
 def cublaslt_nvfp4_tflops(M, N, K, iters=20):
@@ -200,44 +275,6 @@ def cublaslt_nvfp4_tflops(M, N, K, iters=20):
         return 2.0 * M * N * K / (statistics.median(ts) * 1e-3) / 1e12
     except Exception:
         return None
-
-
-def blas_threads():
-    try:
-        from threadpoolctl import threadpool_info
-        return max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
-    except Exception:
-        return os.cpu_count() or 1
-
-
-def workload_config(spec):
-    return {"workload": f"{spec.name} fwd+bwd", "M_tokens_per_gpu": spec.M, "K": spec.K, "N": spec.N,
-            "stabilizer_rank": spec.r_s, "lora_rank": spec.r,
-            "l2": "flushed between steps (512 MiB write, outside the step events)"}
-
-
-def cpu_baseline(spec, budget_s=12.0, rows=512):
-    """The oracle timed on the host cores on a bounded sample (rank 0, N = 1)."""
-    import torch  # noqa: F401
-
-    from diffusion_dit_b200 import prep, workloads as wl
-    from oracle import fourtune_oracle as ora
-    inp = wl.make_layer_inputs(spec, seed=0, rows=rows)
-    split = prep.svd_split(inp.w, spec.r_s)
-    layer = ora.Layer(qr=ora.quantize_residual(split.residual), ls_up=split.ls_up, ls_down=split.ls_down,
-                      lora_a=inp.lora_a, lora_b=inp.lora_b, lora_scale=spec.lora_scale)
-    n, t0 = 0, time.perf_counter()
-    while True:
-        ora.linear_fwd(inp.x, layer)
-        ora.linear_bwd(inp.x, inp.dy, layer)
-        n += 1
-        if time.perf_counter() - t0 >= budget_s:
-            break
-    dt = (time.perf_counter() - t0) / n
-    fp4, bf = layer_flops(rows, spec.K, spec.N, spec.r_s, spec.r)
-    return {"value": (fp4 + bf) / dt / 1e12, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
-            "sample": f"{rows} of {spec.M} tokens with the full weights, {n} oracle passes "
-                      f"(quantize + fwd + bwd, fp64 products) in {time.perf_counter() - t0:.1f} s"}
 
 
 def run_mlp_pair(args):
@@ -415,39 +452,138 @@ def run_mlp_pair(args):
     print(json.dumps(line), flush=True)
 
 
-def main():
-    ap = argparse.ArgumentParser()
-    ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
-    ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--ref-rows", type=int, default=256)
-    ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--graph", dest="graph", action="store_true", default=True,
-                    help="replay each step as a captured CUDA graph (default)")
-    ap.add_argument("--no-graph", dest="graph", action="store_false")
-    ap.add_argument("--workload", default="qkv", choices=sorted(WORKLOADS) + ["mlp"],
-                    help="single-layer workload (default: the attention QKV projection), or mlp: "
-                         "the MLP pair with GELU, fused")
-    args = ap.parse_args()
-    args.warmup = max(args.warmup, 3)
-    if args.workload == "mlp" and args.impl == "ours":
-        if int(os.environ.get("WORLD_SIZE", "1")) > 1:
-            raise SystemExit("--workload mlp runs on one GPU")
-        run_mlp_pair(args)
-        return
+class LayerRun:
+    """One layer of the step: its weights (prepared once, offline), workspace, synthetic
+    inputs resident on the device, and outputs."""
 
+    def __init__(self, spec, dev, seed):
+        import torch
+
+        from diffusion_dit_b200 import fourtune as ft
+        from diffusion_dit_b200 import prep, workloads as wl
+        self.spec = spec
+        inp = wl.make_layer_inputs(spec, seed=seed)
+        self.inp = inp
+        self.split = prep.svd_split(inp.w, spec.r_s)
+        self.w = ft.prepare_weights(self.split.residual.to(dev), self.split.ls_up.to(dev),
+                                    self.split.ls_down.to(dev), inp.lora_a.to(dev), inp.lora_b.to(dev),
+                                    spec.lora_scale)
+        self.w_xp = ft.drop_transposed_codes(self.w)
+        M, K, N, R = spec.M, spec.K, spec.N, spec.r_s + spec.r
+        self.ws = ft.Workspace(self.w, M, dev)
+        self.x = inp.x.to(dev)
+        self.dy = inp.dy.to(dev)
+        bf, f32 = torch.bfloat16, torch.float32
+        self.y = torch.empty(M, N, dtype=bf, device=dev)
+        self.t = torch.empty(M, R, dtype=f32, device=dev)
+        self.dx = torch.empty(M, K, dtype=bf, device=dev)
+        self.da = torch.empty(spec.r, K, dtype=f32, device=dev)
+        self.db = torch.empty(N, spec.r, dtype=f32, device=dev)
+
+    def fwd(self, x1x16=False):
+        from diffusion_dit_b200 import fourtune as ft
+        (ft.linear_fwd_1x16 if x1x16 else ft.linear_fwd)(self.w, self.x, self.ws, y=self.y, t_saved=self.t)
+
+    def bwd(self, xpose=False):
+        from diffusion_dit_b200 import fourtune as ft
+        ft.linear_bwd(self.w_xp if xpose else self.w, self.x, self.t, self.dy, self.ws, dx=self.dx, da=self.da,
+                      db=self.db)
+
+    def flops(self):
+        s = self.spec
+        return layer_flops(s.M, s.K, s.N, s.r_s, s.r)
+
+
+def quant_sweep(dev, warmup, reps, flush):
+    """The quantizer-only workload: Q(x) in 16x16 blocks with the fused rank-32
+    down-projection x A^T, on bf16 inputs of the sweep's shapes, through
+    fourtune_quantize_block16.  Timed as a CUDA graph of the whole call: with the call's
+    own tensor max (one extra read of x), and with a caller-supplied max; and the fused
+    quantizer kernel alone, by its launch events.  GB/s = algorithmic bytes (read x 2 B,
+    write codes 0.5 B and block scales 1/256 B per element, x A^T 4 B per row and rank)
+    / time; with the max pass, 2 B more per element."""
+    import torch
+
+    from diffusion_dit_b200 import fourtune as ft
     from diffusion_dit_b200 import workloads as wl
-    spec = getattr(wl, WORKLOADS.get(args.workload, "FLUX_MLP_UP"))
-    if args.impl == "reference":
-        run_reference(args, spec)
-        return
+    hbm, _, _ = peaks()
+    E = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+    out = []
+    for qs in wl.QUANT_SWEEP:
+        x, down = wl.make_quant_input(qs, seed=0)
+        x, down = x.to(dev), down.to(dev)
+        rows, cols, r = qs.rows, qs.cols, qs.r_down
+        q = ft.QuantizedMatrix.empty(rows, cols, dev, with_sf=False)
+        t = torch.empty(rows, r, dtype=torch.float32, device=dev)
+        amax = x.abs().amax().float().reshape(1)
+        nws = ft.lib().fourtune_quantize_workspace_bytes(rows, cols, r)
+        ws = torch.zeros(nws, dtype=torch.uint8, device=dev)
 
+        def call(given):
+            ft.quantize_block16_into(x, q, ws, amax=amax if given else None, down=down, down_out=t)
+
+        kev = (E(), E())
+        for e in kev:
+            e.record()
+        torch.cuda.synchronize()
+
+        def call_events():
+            ft.time_next_launch(ft.FT_KERNEL_QUANT, *kev)
+            call(False)
+
+        graphs = {}
+        for name, fn in (("own_max", lambda: call(False)), ("given_max", lambda: call(True)),
+                         ("events", call_events)):
+            fn()
+            torch.cuda.synchronize()
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                fn()
+            for _ in range(warmup):
+                flush.zero_()
+                g.replay()
+            graphs[name] = g
+        torch.cuda.synchronize()
+        s_, e_ = E(), E()
+        res = {}
+        for name in ("own_max", "given_max", "events"):
+            ts = []
+            for _ in range(reps):
+                flush.zero_()
+                s_.record()
+                graphs[name].replay()
+                e_.record()
+                torch.cuda.synchronize()
+                ts.append(kev[0].elapsed_time(kev[1]) if name == "events" else s_.elapsed_time(e_))
+            res[name] = statistics.median(ts)
+        n = rows * cols
+        base = n * (2.0 + 0.5 + 1.0 / 256) + rows * r * 4.0
+        entry = {"shape": [rows, cols], "r_down": r,
+                 "call_ms": res["own_max"], "call_gbs": (base + 2.0 * n) / (res["own_max"] * 1e-3) / 1e9,
+                 "call_given_max_ms": res["given_max"],
+                 "call_given_max_gbs": base / (res["given_max"] * 1e-3) / 1e9,
+                 "kernel_ms": res["events"], "kernel_gbs": base / (res["events"] * 1e-3) / 1e9}
+        entry["frac_call"] = entry["call_gbs"] / hbm
+        entry["frac_call_given_max"] = entry["call_given_max_gbs"] / hbm
+        entry["frac_kernel"] = entry["kernel_gbs"] / hbm
+        out.append(entry)
+        del graphs, x, down, q, t, ws
+        torch.cuda.synchronize()
+        torch.cuda.empty_cache()
+    return {"what": "fourtune_quantize_block16 with the fused rank-32 down-projection, bf16 inputs "
+                    "~N(0,1) with 1% Laplace(10) entries; median of replays with L2 flushed; "
+                    "call = the whole entry point (tensor max pass, factor prologue, fused quantizer, "
+                    "split sum), given_max = the same with the caller's max, kernel = the fused "
+                    "quantizer launch alone (launch events)",
+            "peak_gbs": hbm, "shapes": out}
+
+
+def run_layers(args, desc, specs):
     import torch
     import torch.distributed as dist
 
+    from diffusion_dit_b200 import dp
     from diffusion_dit_b200 import fourtune as ft
-    from diffusion_dit_b200 import dp, prep
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -457,121 +593,119 @@ def main():
     if world > 1:
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
 
-    # --- setup (untimed): inputs of this rank's shard, offline weight prep ------
-    inp = wl.make_layer_inputs(spec, seed=rank)
-    split = prep.svd_split(inp.w, spec.r_s)
-    w = ft.prepare_weights(split.residual.to(dev), split.ls_up.to(dev), split.ls_down.to(dev),
-                           inp.lora_a.to(dev), inp.lora_b.to(dev), spec.lora_scale)
-    M, K, N = spec.M, spec.K, spec.N
-    R = spec.r_s + spec.r
-    ws = ft.Workspace(w, M, dev)
-    x = inp.x.to(dev)
-    dy = inp.dy.to(dev)
-    y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
-    t = torch.empty(M, R, dtype=torch.float32, device=dev)
-    dx = torch.empty(M, K, dtype=torch.bfloat16, device=dev)
-    da = torch.empty(spec.r, K, dtype=torch.float32, device=dev)
-    db = torch.empty(N, spec.r, dtype=torch.float32, device=dev)
+    # --- setup (untimed): this rank's synthetic inputs, offline weight prep -------------
+    layers = [LayerRun(s, dev, seed=rank + 17 * i) for i, s in enumerate(specs)]
     flush = torch.empty(512 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
 
-    def step_kernels():
-        ft.linear_fwd(w, x, ws, y=y, t_saved=t)
-        ft.linear_bwd(w, x, t, dy, ws, dx=dx, da=da, db=db)
+    def step_kernels(x1x16=False, xpose=False, fwd=True, bwd=True):
+        if fwd:
+            for L in layers:
+                L.fwd(x1x16)
+        if bwd:
+            for L in reversed(layers):
+                L.bwd(xpose)
+
+    def allreduce():
+        for L in reversed(layers):
+            dp.allreduce_adapter_grads(L.da, L.db)
 
     def step():
         step_kernels()
         if world > 1:
-            dp.allreduce_adapter_grads(da, db)
+            allreduce()
 
     for _ in range(args.warmup):
         flush.zero_()
         step()
     torch.cuda.synchronize()
-    if ws.device_status() != 0:
+    if any(L.ws.device_status() for L in layers):
         raise RuntimeError("device status reports a timeout during warm-up")
 
     Kst = args.steps
     E = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
-    ev_s, ev_e = [E() for _ in range(Kst)], [E() for _ in range(Kst)]
-    # per-launch events of the dominant kernel (the 4-bit GEMM: forward and dX), the
-    # quantizer and the tensor max; the library records them on the launch stream
-    kev = {k: ([E(), E()], [E(), E()]) for k in (ft.FT_KERNEL_GEMM, ft.FT_KERNEL_QUANT, ft.FT_KERNEL_AMAX)}
-    for ev in ev_s + ev_e + [e for b_, a_ in kev.values() for e in b_ + a_]:
+    fp4 = sum(L.flops()[0] for L in layers)
+    bf = sum(L.flops()[1] for L in layers)
+
+    if args.profile:
+        # the plain step, eagerly, for profilers: no graphs, no side measurements
+        s_, e_ = E(), E()
+        torch.cuda.synchronize()
+        s_.record()
+        for _ in range(Kst):
+            step()
+        e_.record()
+        torch.cuda.synchronize()
+        ms = s_.elapsed_time(e_) / Kst
+        if rank == 0:
+            print(json.dumps({"profile": True, "workload": desc, "ms_per_step_eager": ms,
+                              "value_eager": world * (fp4 + bf) / (ms * 1e-3) / 1e12}), flush=True)
+        if world > 1:
+            dist.barrier()
+            dist.destroy_process_group()
+        return
+
+    # per-launch events: every GEMM and quantizer launch of one step (and the forward
+    # prologue that takes max|X|), recorded by the library on the launch stream
+    GEMM, QUANT, AMAX = ft.FT_KERNEL_GEMM, ft.FT_KERNEL_QUANT, ft.FT_KERNEL_AMAX
+    nL = len(layers)
+    kev = {(k, i): (E(), E()) for k in (GEMM, QUANT) for i in range(2 * nL)}
+    kev.update({(AMAX, i): (E(), E()) for i in range(nL)})
+    xp_ev = [(E(), E()) for _ in range(nL)]
+    for ev in [e for p_ in list(kev.values()) + xp_ev for e in p_]:
         ev.record()  # torch creates the CUDA event on first record; the library needs the handle
     torch.cuda.synchronize()
 
-    def one_step_with_events():
-        for k, (b_, a_) in kev.items():
-            ft.time_next_launch(k, b_[0], a_[0])
-        ft.linear_fwd(w, x, ws, y=y, t_saved=t)
-        # the backward has no separate tensor-max launch: its adapter-gradient kernel
-        # takes max |G| on the way
-        for k in (ft.FT_KERNEL_GEMM, ft.FT_KERNEL_QUANT):
-            ft.time_next_launch(k, kev[k][0][1], kev[k][1][1])
-        ft.linear_bwd(w, x, t, dy, ws, dx=dx, da=da, db=db)
+    def step_with_events():
+        for i, L in enumerate(layers):
+            for k in (GEMM, QUANT):
+                ft.time_next_launch(k, *kev[(k, i)])
+            ft.time_next_launch(AMAX, *kev[(AMAX, i)])
+            L.fwd()
+        for j, L in enumerate(reversed(layers)):
+            for k in (GEMM, QUANT):
+                ft.time_next_launch(k, *kev[(k, nL + j)])
+            L.bwd()
 
-    def fwd_kernels():
-        ft.linear_fwd(w, x, ws, y=y, t_saved=t)
+    def bwd_xpose_with_events():  # each layer's dX GEMM is its backward's last GEMM launch
+        for j, L in enumerate(reversed(layers)):
+            ft.time_next_launch(GEMM, *xp_ev[j])
+            L.bwd(xpose=True)
 
-    def fwd_1x16_kernels():  # X quantized group-wise 1x16 (the Table 5 comparison, forward only)
-        ft.linear_fwd_1x16(w, x, ws, y=y, t_saved=t)
-
-    def bwd_kernels():
-        ft.linear_bwd(w, x, t, dy, ws, dx=dx, da=da, db=db)
-
-    # the same layer with Q(R)^T's codes dropped: the dX GEMM transposes Q(R) on the fly
-    w_xp = ft.drop_transposed_codes(w)
-    xp_ev = (E(), E())
-    for ev in xp_ev:
-        ev.record()
-
-    def bwd_xpose_kernels():
-        ft.linear_bwd(w_xp, x, t, dy, ws, dx=dx, da=da, db=db)
-
-    def bwd_xpose_with_events():  # the dX GEMM is the backward's last GEMM launch
-        ft.time_next_launch(ft.FT_KERNEL_GEMM, xp_ev[0], xp_ev[1])
-        ft.linear_bwd(w_xp, x, t, dy, ws, dx=dx, da=da, db=db)
-
-    graph = graph_k = graph_f = graph_b = graph_f1 = graph_bx = graph_bxk = None
-    launches_per_step = None
+    # Each pass is captured once as a CUDA graph and replayed: the same kernels without
+    # the host launch gaps.  Event-record nodes between kernels serialise them (~50 us per
+    # step), so the headline steps replay graphs without them and a second pass of as many
+    # steps replays the instrumented one to time the kernels.
+    variants = {"step": step_kernels, "events": step_with_events,
+                "fwd": lambda: step_kernels(bwd=False), "bwd": lambda: step_kernels(fwd=False),
+                "fwd_1x16": lambda: step_kernels(x1x16=True, bwd=False),
+                "bwd_xpose": lambda: step_kernels(xpose=True, fwd=False), "bwd_xpose_events": bwd_xpose_with_events}
+    graphs, launches_per_step = {}, None
     if args.graph:
-        # One step (forward + backward: all of the library's kernels) captured once as a
-        # CUDA graph and replayed: the same kernels, without the host launch gaps between
-        # them.  A second capture adds the per-launch timing events (graph event-record
-        # nodes); those serialise the kernels around them and cost ~50 us per step, so the
-        # headline steps replay the graph without them and a second pass of as many steps
-        # replays the instrumented one to time the kernels.
-        c0 = ft.launch_count()
-        graph = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(graph):
-            step_kernels()
-        launches_per_step = ft.launch_count() - c0
-        graph_k = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(graph_k):
-            one_step_with_events()
-        # forward alone and backward alone, for the per-pass figures
-        graph_f, graph_b, graph_f1 = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
-        with torch.cuda.graph(graph_f):
-            fwd_kernels()
-        with torch.cuda.graph(graph_b):
-            bwd_kernels()
-        fwd_1x16_kernels()
-        with torch.cuda.graph(graph_f1):
-            fwd_1x16_kernels()
-        bwd_xpose_kernels()
-        graph_bx, graph_bxk = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
-        with torch.cuda.graph(graph_bx):
-            bwd_xpose_kernels()
-        with torch.cuda.graph(graph_bxk):
-            bwd_xpose_with_events()
+        for name, fn in variants.items():
+            fn()
+            torch.cuda.synchronize()
+            c0 = ft.launch_count()
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                fn()
+            if name == "step":
+                launches_per_step = ft.launch_count() - c0
+            graphs[name] = g
         for _ in range(args.warmup):
-            for g_ in (graph, graph_k, graph_f, graph_b, graph_f1, graph_bx, graph_bxk):
+            for g in graphs.values():
                 flush.zero_()
-                g_.replay()
+                g.replay()
         torch.cuda.synchronize()
 
-    gemm_ms, quant_ms, amax_ms = [], [], []
-    ev_ks, ev_ke = [E() for _ in range(Kst)], [E() for _ in range(Kst)]
+    def run(name):
+        if name in graphs:
+            graphs[name].replay()
+        else:
+            variants[name]()
+
+    ev_s, ev_e = [E() for _ in range(Kst)], [E() for _ in range(Kst)]
+    gemm_ms, quant_ms, amax_ms, xp_gemm_ms = [], [], [], []
+    pass_ms = {}
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
@@ -580,164 +714,199 @@ def main():
         for i in range(Kst):
             flush.zero_()
             ev_s[i].record()
-            if graph is not None:
-                graph.replay()
-            else:
-                step_kernels()
+            run("step")
             if world > 1:
-                dp.allreduce_adapter_grads(da, db)
+                allreduce()
             ev_e[i].record()
         torch.cuda.synchronize()
         if world > 1:
             dist.barrier()
         torch.cuda.synchronize()
-        launches = (launches_per_step * Kst) if graph is not None else ft.launch_count() - launches0
+        launches = (launches_per_step * Kst) if launches_per_step is not None else ft.launch_count() - launches0
+        total_ms = sum(ev_s[i].elapsed_time(ev_e[i]) for i in range(Kst))
         # kernel-timing pass: the same steps with per-launch events on the launch stream
+        ev_k = []
         for i in range(Kst):
             flush.zero_()
-            ev_ks[i].record()
-            if graph_k is not None:
-                graph_k.replay()
-            else:
-                one_step_with_events()
-            ev_ke[i].record()
-            # the per-launch events are reused by every step: read them before the next one
-            torch.cuda.synchronize()
-            for k, dst in ((ft.FT_KERNEL_GEMM, gemm_ms), (ft.FT_KERNEL_QUANT, quant_ms)):
-                b_, a_ = kev[k]
-                dst.extend([b_[0].elapsed_time(a_[0]), b_[1].elapsed_time(a_[1])])
-            amax_ms.append(kev[ft.FT_KERNEL_AMAX][0][0].elapsed_time(kev[ft.FT_KERNEL_AMAX][1][0]))
-        torch.cuda.synchronize()
-        ms_per_step_events = sum(ev_ks[i].elapsed_time(ev_ke[i]) for i in range(Kst)) / Kst
-        # per-pass pass: the forward alone, then the backward alone, as many steps each
-        pass_ms = {"fwd": [], "bwd": [], "fwd_1x16": [], "bwd_xpose": []}
-        for name, g_, fn in (("fwd", graph_f, fwd_kernels), ("bwd", graph_b, bwd_kernels),
-                             ("fwd_1x16", graph_f1, fwd_1x16_kernels),
-                             ("bwd_xpose", graph_bx, bwd_xpose_kernels)):
+            ev_s[i].record()
+            run("events")
+            ev_e[i].record()
+            torch.cuda.synchronize()  # the per-launch events are reused: read them now
+            ev_k.append(ev_s[i].elapsed_time(ev_e[i]))
+            gemm_ms.append([kev[(GEMM, j)][0].elapsed_time(kev[(GEMM, j)][1]) for j in range(2 * nL)])
+            quant_ms.append([kev[(QUANT, j)][0].elapsed_time(kev[(QUANT, j)][1]) for j in range(2 * nL)])
+            amax_ms.append([kev[(AMAX, j)][0].elapsed_time(kev[(AMAX, j)][1]) for j in range(nL)])
+        # per-pass figures: forward alone, backward alone, 1x16 forward, transposing backward
+        for name in ("fwd", "bwd", "fwd_1x16", "bwd_xpose"):
+            ts = []
             for i in range(Kst):
                 flush.zero_()
-                ev_ks[i].record()
-                if g_ is not None:
-                    g_.replay()
-                else:
-                    fn()
-                ev_ke[i].record()
+                ev_s[i].record()
+                run(name)
+                ev_e[i].record()
             torch.cuda.synchronize()
-            pass_ms[name] = [ev_ks[i].elapsed_time(ev_ke[i]) for i in range(Kst)]
-        # the transposing dX GEMM alone, by its launch events
-        xp_gemm_ms = []
+            pass_ms[name] = statistics.median(ev_s[i].elapsed_time(ev_e[i]) for i in range(Kst))
         for i in range(Kst):
             flush.zero_()
-            if graph_bxk is not None:
-                graph_bxk.replay()
-            else:
-                bwd_xpose_with_events()
+            run("bwd_xpose_events")
             torch.cuda.synchronize()
-            xp_gemm_ms.append(xp_ev[0].elapsed_time(xp_ev[1]))
-    if ws.device_status() != 0:
+            xp_gemm_ms.append([b_.elapsed_time(a_) for b_, a_ in xp_ev])
+    if any(L.ws.device_status() for L in layers):
         raise RuntimeError("device status reports a timeout in the timed region")
 
-    total_ms = sum(ev_s[i].elapsed_time(ev_e[i]) for i in range(Kst))
     tm = torch.tensor([total_ms], dtype=torch.float64, device=dev)
     if world > 1:
         dist.all_reduce(tm, op=dist.ReduceOp.MAX)
     total_ms = float(tm.item())
     ms_per_step = total_ms / Kst
-    fp4, bf = layer_flops(M, K, N, spec.r_s, spec.r)
     value = world * (fp4 + bf) * Kst / (total_ms * 1e-3) / 1e12
 
-    # --- end to end through the API with host buffers (pinned), copies timed ---
-    x_h = inp.x.pin_memory()
-    dy_h = inp.dy.pin_memory()
-    da_h = torch.empty(da.shape, dtype=da.dtype).pin_memory()
-    db_h = torch.empty(db.shape, dtype=db.dtype).pin_memory()
-    e_s, e_e = [E() for _ in range(Kst)], [E() for _ in range(Kst)]
+    # --- end to end through the API: every layer's X and dY copied in from pinned host
+    # memory, dA and dB copied out, inside the timed region ----------------------------
+    hx = [L.inp.x.pin_memory() for L in layers]
+    hdy = [L.inp.dy.pin_memory() for L in layers]
+    hda = [torch.empty(L.da.shape, dtype=L.da.dtype).pin_memory() for L in layers]
+    hdb = [torch.empty(L.db.shape, dtype=L.db.dtype).pin_memory() for L in layers]
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
     for i in range(Kst):
         flush.zero_()
-        e_s[i].record()
-        x.copy_(x_h, non_blocking=True)
-        dy.copy_(dy_h, non_blocking=True)
-        ft.linear_fwd(w, x, ws, y=y, t_saved=t)
-        ft.linear_bwd(w, x, t, dy, ws, dx=dx, da=da, db=db)
-        if world > 1:
-            dp.allreduce_adapter_grads(da, db)
-        da_h.copy_(da, non_blocking=True)
-        db_h.copy_(db, non_blocking=True)
-        e_e[i].record()
+        ev_s[i].record()
+        for L, a, b in zip(layers, hx, hdy):
+            L.x.copy_(a, non_blocking=True)
+            L.dy.copy_(b, non_blocking=True)
+        step()
+        for L, a, b in zip(layers, hda, hdb):
+            a.copy_(L.da, non_blocking=True)
+            b.copy_(L.db, non_blocking=True)
+        ev_e[i].record()
     torch.cuda.synchronize()
-    e2e_ms = torch.tensor([sum(e_s[i].elapsed_time(e_e[i]) for i in range(Kst))], dtype=torch.float64,
+    e2e_ms = torch.tensor([sum(ev_s[i].elapsed_time(ev_e[i]) for i in range(Kst))], dtype=torch.float64,
                           device=dev)
     if world > 1:
         dist.all_reduce(e2e_ms, op=dist.ReduceOp.MAX)
     e2e_value = world * (fp4 + bf) * Kst / (float(e2e_ms.item()) * 1e-3) / 1e12
-    h2d = x.numel() * 2 + dy.numel() * 2
-    d2h = da.numel() * 4 + db.numel() * 4
+    h2d = sum(L.x.numel() * 2 + L.dy.numel() * 2 for L in layers)
+    d2h = sum(L.da.numel() * 4 + L.db.numel() * 4 for L in layers)
 
     if rank == 0:
         hbm, bf16_peak, src = peaks()
         fp4_peak = bf16_peak * NOMINAL_FP4_OVER_BF16
-        gemm_avg = statistics.mean(gemm_ms)
-        achieved = 2.0 * M * N * K / (gemm_avg * 1e-3) / 1e12
-        # ncu dram read + write per launch (mean of fwd and dX), captured on this workload
-        traffic = gemm_traffic() if args.workload == "qkv" else None
-        # quantizer: X [M, K] and G [M, N] alternate; algorithmic bytes per element:
-        # 2 (read bf16) + 0.5 (codes) + 1/256 (block scales).  The tensor max of X is one
-        # more read of X, by the forward's prologue kernel (which also builds the low-rank
-        # factors: its whole duration counts); max |G| is taken by the dB kernel.
-        elems = [M * K, M * N] * Kst
-        qbytes = sum(e * (2.0 + 0.5 + 1.0 / 256) for e in elems)
-        q_gbs = qbytes / (sum(quant_ms) * 1e-3) / 1e9
-        qa_gbs = (qbytes + 2.0 * M * K * Kst) / ((sum(quant_ms) + sum(amax_ms)) * 1e-3) / 1e9
-        fl_f, fl_b = pass_flops(M, K, N, spec.r_s, spec.r)
-        fwd_ms, bwd_ms = statistics.median(pass_ms["fwd"]), statistics.median(pass_ms["bwd"])
-        lt_fwd = cublaslt_nvfp4_tflops(M, N, K)
-        lt_dx = cublaslt_nvfp4_tflops(M, K, N)
-        lt_mean = (lt_fwd + lt_dx) / 2 if lt_fwd and lt_dx else None
+        # the GEMM launches of a step, in order: each layer's forward, then the backward's
+        # dX GEMMs in reverse layer order; FLOPs 2 M N K each
+        gemm_flops = [2.0 * L.spec.M * L.spec.N * L.spec.K for L in layers] * 2
+        gemm_avg = statistics.mean(sum(r) for r in gemm_ms) / len(gemm_flops)
+        achieved = statistics.mean(gemm_flops) / (gemm_avg * 1e-3) / 1e12
+        per_launch = []
+        names = [f"{L.spec.name} fwd" for L in layers] + [f"{L.spec.name} dX" for L in reversed(layers)]
+        specs_order = [L.spec for L in layers] + [L.spec for L in reversed(layers)]
+        lt = {}
+        for j, (nm, s) in enumerate(zip(names, specs_order)):
+            ms_j = statistics.mean(r[j] for r in gemm_ms)
+            shape = (s.M, s.N, s.K) if j < nL else (s.M, s.K, s.N)
+            if shape not in lt:
+                lt[shape] = cublaslt_nvfp4_tflops(*shape)
+            per_launch.append({"launch": nm, "M_N_K": list(shape), "ms": ms_j,
+                               "tflops": gemm_flops[j] / (ms_j * 1e-3) / 1e12, "cublaslt_tflops": lt[shape]})
+        lt_time = sum(gemm_flops[j] / (p["cublaslt_tflops"] * 1e12) for j, p in enumerate(per_launch)) \
+            if all(p["cublaslt_tflops"] for p in per_launch) else None
+        # quantizer launches: X of each layer (forward), G of each layer (backward)
+        q_elems = [L.spec.M * L.spec.K for L in layers] + [L.spec.M * L.spec.N for L in reversed(layers)]
+        q_rank = [L.spec.r_s + L.spec.r for L in layers] + [L.spec.r_s + L.spec.r for L in reversed(layers)]
+        q_rows = [L.spec.M for L in layers] + [L.spec.M for L in reversed(layers)]
+        q_bytes = [e * (2.0 + 0.5 + 1.0 / 256) + m * r * 4.0 for e, m, r in zip(q_elems, q_rows, q_rank)]
+        q_ms = [statistics.mean(r[j] for r in quant_ms) for j in range(2 * nL)]
+        q_gbs = sum(q_bytes) / (sum(q_ms) * 1e-3) / 1e9
+        a_ms = [statistics.mean(r[j] for r in amax_ms) for j in range(nL)]
+        qa_gbs = (sum(q_bytes) + sum(2.0 * L.spec.M * L.spec.K for L in layers)) / \
+            ((sum(q_ms) + sum(a_ms)) * 1e-3) / 1e9
+        fl_f = sum(pass_flops(L.spec.M, L.spec.K, L.spec.N, L.spec.r_s, L.spec.r)[0] for L in layers)
+        fl_b = sum(pass_flops(L.spec.M, L.spec.K, L.spec.N, L.spec.r_s, L.spec.r)[1] for L in layers)
         line = {
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": Kst,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "nvfp4(e2m1,ue4m3)+bf16", "data": "synthetic",
-            "config": dict(workload_config(spec), parallelism=f"dp{world}",
+            "config": dict(workload_config(args, desc, specs), parallelism=f"dp{world}",
                            flops_per_step={"fp4": fp4, "bf16": bf}),
-            "roofline": {"bound": "tensor", "kernel": "gemm_fp4_lowrank_pair_kernel (fwd and dX)",
+            "roofline": {"bound": "tensor", "kernel": "gemm_fp4_lowrank_pair_kernel (every forward and dX GEMM)",
                          "achieved": achieved, "peak": fp4_peak, "unit": "TFLOP/s",
-                         "frac": achieved / fp4_peak, "traffic": traffic,
+                         "frac": achieved / fp4_peak, "traffic": gemm_traffic(args.workload),
                          "peak_source": f"{src} bf16 {bf16_peak} TFLOP/s x {NOMINAL_FP4_OVER_BF16} "
                                         f"(nominal fp4/bf16 ratio)",
                          "avg_launch_ms": gemm_avg,
                          "frac_of_nominal_9pf": achieved / NOMINAL_FP4_TFLOPS,
-                         "cublaslt_nvfp4_tflops": {"fwd_shape": lt_fwd, "dx_shape": lt_dx},
-                         "frac_of_cublaslt": achieved / lt_mean if lt_mean else None,
+                         "frac_of_cublaslt": (lt_time * 1e3 / sum(p["ms"] for p in per_launch)) if lt_time else None,
+                         "launches": per_launch,
                          "timing": "CUDA events around each launch, recorded in a second pass of "
-                                   f"{Kst} steps (that pass: {ms_per_step_events:.4f} ms per step)"},
-            "quantizer": {"kernel": "quant_down_kernel (quantizer fused with the down-projection)", "achieved_gbs": q_gbs,
-                          "with_amax_pass_gbs": qa_gbs, "peak_gbs": hbm, "frac": q_gbs / hbm,
-                          "frac_with_amax": qa_gbs / hbm, "avg_launch_ms": statistics.mean(quant_ms)},
-            "per_pass": {"fwd_ms": fwd_ms, "fwd_tflops": fl_f / (fwd_ms * 1e-3) / 1e12,
-                         "bwd_ms": bwd_ms, "bwd_tflops": fl_b / (bwd_ms * 1e-3) / 1e12,
-                         "fwd_1x16_ms": statistics.median(pass_ms["fwd_1x16"]),
+                                   f"{Kst} steps (that pass: {statistics.mean(ev_k):.4f} ms per step)"},
+            "quantizer": {"kernel": "quant_down_kernel (quantizer fused with the down-projection)",
+                          "achieved_gbs": q_gbs, "with_amax_pass_gbs": qa_gbs, "peak_gbs": hbm,
+                          "frac": q_gbs / hbm, "frac_with_amax": qa_gbs / hbm,
+                          "launch_ms": q_ms, "amax_pass_ms": a_ms,
+                          "bytes_per_element": "2 (read) + 0.5 (codes) + 1/256 (block scales), + 4 R per row"},
+            "per_pass": {"fwd_ms": pass_ms["fwd"], "fwd_tflops": fl_f / (pass_ms["fwd"] * 1e-3) / 1e12,
+                         "bwd_ms": pass_ms["bwd"], "bwd_tflops": fl_b / (pass_ms["bwd"] * 1e-3) / 1e12,
+                         "fwd_1x16_ms": pass_ms["fwd_1x16"],
                          "timing": f"median of {Kst} replays of a forward-only / backward-only graph"},
             "xpose_on_the_fly": {
                 "what": "backward with Q(R)^T's codes dropped: the dX GEMM transposes Q(R)'s tiles in "
                         "shared memory (section 3.2)",
-                "bwd_ms": statistics.median(pass_ms["bwd_xpose"]), "bwd_ms_stored_copy": bwd_ms,
-                "dx_gemm_ms": statistics.mean(xp_gemm_ms),
-                "dx_gemm_ms_stored_copy": statistics.mean(gemm_ms[1::2]),
-                "bytes_saved": N * K // 2 + N * K // 256},
-            "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+                "bwd_ms": pass_ms["bwd_xpose"], "bwd_ms_stored_copy": pass_ms["bwd"],
+                "dx_gemm_ms": [statistics.mean(r[j] for r in xp_gemm_ms) for j in range(nL)],
+                "dx_gemm_ms_stored_copy": [statistics.mean(r[nL + j] for r in gemm_ms) for j in range(nL)],
+                "bytes_saved": sum(L.spec.N * L.spec.K // 2 + L.spec.N * L.spec.K // 256 for L in layers)},
+            "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "what": "each step copies every layer's X and dY in from pinned host memory and its dA "
+                            "and dB out; Y and dX stay on the device (in a training step they are the next "
+                            "layer's input and the previous layer's gradient)"},
             "gpu_launches": launches,
-            "launch_mode": "cuda_graph_replay" if graph is not None else "stream",
+            "launch_mode": "cuda_graph_replay" if graphs else "stream",
             "clocks": clocks.summary(),
         }
+        if world == 1 and not args.no_quant_sweep:
+            line["quantizer_sweep"] = quant_sweep(dev, args.warmup, min(Kst, 20), flush)
         if world == 1 and not args.no_cpu_baseline:
-            line["cpu_baseline"] = cpu_baseline(spec)
+            line["cpu_baseline"] = cpu_baseline(specs, [L.split for L in layers])
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--ref-rows", type=int, default=64)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-quant-sweep", action="store_true")
+    ap.add_argument("--graph", dest="graph", action="store_true", default=True,
+                    help="replay each step as a captured CUDA graph (default)")
+    ap.add_argument("--no-graph", dest="graph", action="store_false")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS) + ["mlp"],
+                    help="default: the FLUX single-stream block's two linears; mlp: the MLP pair with "
+                         "GELU, fused")
+    ap.add_argument("--tokens", type=int, default=0, help="replace the token count M (multiple of 256)")
+    ap.add_argument("--profile", action="store_true", help="plain eager steps only (for profilers)")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+    if args.tokens and args.tokens % 256:
+        raise SystemExit("--tokens must be a multiple of 256")
+    if args.workload == "mlp" and args.impl == "ours":
+        if int(os.environ.get("WORLD_SIZE", "1")) > 1:
+            raise SystemExit("--workload mlp runs on one GPU")
+        run_mlp_pair(args)
+        return
+    if args.workload == "mlp":
+        args.workload = "mlp_up"  # the reference arm of the pair: its first layer
+    desc, specs = specs_of(args)
+    if args.impl == "reference":
+        run_reference(args, desc, specs)
+        return
+    run_layers(args, desc, specs)
 
 
 if __name__ == "__main__":

@@ -737,7 +737,8 @@ ft_status fourtune_selftest_bounded_wait(int64_t limit_ns, void* ws, void* strea
 }
 
 ft_status fourtune_device_status(void* ws, int32_t* status_out, void* stream) {
-    if (!ws || !status_out) return FT_ERR_INVALID_ARG;
+    if (!status_out) return FT_ERR_INVALID_ARG;
+    if (!ws) FT_TRY(ft::noalloc_scratch(&ws));  // the status of fourtune_quantize_block16_noalloc
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     int32_t v = 0;
     FT_CUDA(cudaMemcpyAsync(&v, ws, sizeof(int32_t), cudaMemcpyDeviceToHost, st));

@@ -6,7 +6,13 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include "fourtune.h"
+
 namespace ft {
+
+// Device address of fourtune_quantize_block16_noalloc's fixed scratch array on the
+// current device and context, looked up on first use (ft_noalloc.cu).
+ft_status noalloc_scratch(void** out);
 
 // Instrumentation (ft_api.cu): every launcher calls before_launch(kind, stream) and
 // after_launch(kind, stream) around its kernel launch.

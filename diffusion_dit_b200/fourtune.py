@@ -179,6 +179,26 @@ def quantize_block16(x: torch.Tensor, amax: Optional[torch.Tensor] = None, with_
     return q, qt, down_out
 
 
+def quantize_block16_into(x: torch.Tensor, q: QuantizedMatrix, ws: torch.Tensor, amax: Optional[torch.Tensor] = None,
+                          down: Optional[torch.Tensor] = None, down_out: Optional[torch.Tensor] = None,
+                          q_t: Optional[QuantizedMatrix] = None, stream=None):
+    """Q(x) in 16x16 blocks into preallocated outputs with a caller workspace ``ws`` (uint8,
+    at least fourtune_quantize_workspace_bytes): allocates nothing, so it can be captured
+    in a CUDA graph.  ``down`` [r, cols] bf16 with ``down_out`` [rows, r] fp32: the fused
+    down-projection x down^T."""
+    _require_cuda(x, amax, down, down_out, ws)
+    rows, cols = x.shape
+    dt = {torch.bfloat16: FT_DTYPE_BF16, torch.float32: FT_DTYPE_F32}[x.dtype]
+    r_down = 0 if down is None else down.shape[0]
+    qs = q.c_struct()
+    qts = q_t.c_struct() if q_t is not None else None
+    st = lib().fourtune_quantize_block16(_p(x), dt, rows, cols, x.stride(0), _p(amax), _p(down), r_down,
+                                         _p(down_out), ctypes.byref(qs),
+                                         ctypes.byref(qts) if qts is not None else None,
+                                         _p(ws), ws.numel(), _stream(stream))
+    _check("fourtune_quantize_block16", st)
+
+
 def quantize_1x16(x: torch.Tensor, amax: Optional[torch.Tensor] = None, with_sf: bool = True, stream=None):
     """Q(x) in group-wise 1x16 blocks (scales [rows, cols/16]) on the GPU; bf16 x."""
     _require_cuda(x, amax)
@@ -410,17 +430,28 @@ def time_next_launch(kind: int, before: Optional[torch.cuda.Event], after: Optio
 
 class FourTuneLinearFunction(torch.autograd.Function):
     """autograd wrapper: forward Eq. (2), backward Eq. (3) + adapter gradients.
-    Gradients flow to X, lora_a and lora_b only (R and the stabilizer are frozen)."""
+
+    ``lora_a`` [r, K] and ``lora_b`` [N, r] are the adapter parameters this call uses (any
+    float dtype; the layer computes with their bf16 values), so a caller that replaces or
+    updates them is always seen; ``weights`` supplies the frozen Q(R), Q(R)^T and
+    stabilizer factors (its own lora_a / lora_b are ignored).  Gradients flow to X,
+    lora_a and lora_b only (R and the stabilizer are frozen), each in its input's dtype."""
 
     @staticmethod
     def forward(ctx, x, lora_a, lora_b, weights: LinearWeights, ws: Workspace):
-        y, t = linear_fwd(weights, x, ws)
+        if lora_a.shape != weights.lora_a.shape or lora_b.shape != weights.lora_b.shape:
+            raise ValueError("lora_a / lora_b do not match the layer's adapter shapes")
+        w = dataclasses.replace(weights, lora_a=lora_a.detach().to(torch.bfloat16).contiguous(),
+                                lora_b=lora_b.detach().to(torch.bfloat16).contiguous())
+        x = x.contiguous()
+        y, t = linear_fwd(w, x, ws)
         ctx.save_for_backward(x, t)
-        ctx.weights, ctx.ws = weights, ws
+        ctx.weights, ctx.ws = w, ws
+        ctx.dtypes = (lora_a.dtype, lora_b.dtype)
         return y
 
     @staticmethod
     def backward(ctx, dy):
         x, t = ctx.saved_tensors
-        dx, da, db = linear_bwd(ctx.weights, x, t, dy.contiguous(), ctx.ws)
-        return dx, da.to(torch.bfloat16), db.to(torch.bfloat16), None, None
+        dx, da, db = linear_bwd(ctx.weights, x, t, dy.to(torch.bfloat16).contiguous(), ctx.ws)
+        return dx, da.to(ctx.dtypes[0]), db.to(ctx.dtypes[1]), None, None

@@ -34,8 +34,12 @@
  *  - Matrices are row-major and dense (row stride == number of columns) unless an
  *    `ld` argument says otherwise.  bf16 is IEEE bfloat16 stored as 16-bit words.
  *  - The library allocates no device memory and keeps no state between calls other
- *    than a per-process cache of driver entry points.  All scratch comes from the
- *    caller's workspace `ws` of `ws_bytes` bytes (256-byte aligned); query the size first.
+ *    than per-process caches (driver entry points, device attributes).  All scratch
+ *    comes from the caller's workspace `ws` of `ws_bytes` bytes (256-byte aligned);
+ *    query the size first.  The one exception is fourtune_quantize_block16_noalloc:
+ *    its scratch is a fixed array of FT_NOALLOC_SCRATCH_BYTES in the library's own
+ *    device memory (held by every GPU that loads the library, until exit), whose
+ *    device address the library caches per device and CUDA context.
  *  - Kernels never trap.  Shapes are checked on the host before any launch.
  */
 #ifndef FOURTUNE_H_
@@ -165,11 +169,14 @@ ft_status fourtune_quantize_block16(const void* x_dev, int32_t x_dtype, int64_t 
  * and outputs are still the caller's.
  *  - A problem whose scratch (fourtune_quantize_workspace_bytes) exceeds
  *    FT_NOALLOC_SCRATCH_BYTES is refused with FT_ERR_WORKSPACE before anything runs.
- *  - The first call on a device looks up the array's device address (that device must
- *    be current) and keeps it; make that first call before any stream capture.
+ *  - The first call on a device (and again the first call in a new CUDA context of that
+ *    device, e.g. after cudaDeviceReset) looks up the array's device address, with that
+ *    device current, and keeps it; make that first call before any stream capture.
  *  - All calls share the one array and it keeps the previous call's contents (the call
  *    clears what must start at zero).  Calls whose kernels can overlap on the GPU --
  *    different streams with no ordering between them -- race and give wrong results.
+ *  - Errors detected on the device (FT_ERR_TIMEOUT) go to the array's status word, which
+ *    only the kernels set: read and clear it with fourtune_device_status(NULL, ...).
  *  - It allocates nothing: no cudaMalloc, cudaFree or allocating library routine.
  */
 #define FT_NOALLOC_SCRATCH_BYTES (8u << 20)
@@ -269,8 +276,10 @@ ft_status fourtune_linear_bwd_gelu(const ft_linear* layer, const void* x_dev, co
 
 /*
  * Reads (synchronously, on `stream`) the device status word that the kernels of the
- * last call using workspace `ws` left behind: FT_OK or FT_ERR_TIMEOUT.  *status_out is
- * a HOST pointer.  Clears the word.
+ * calls using workspace `ws` left behind since it was last read: FT_OK or
+ * FT_ERR_TIMEOUT.  *status_out is a HOST pointer.  Clears the word.  ws == NULL reads
+ * the status word of fourtune_quantize_block16_noalloc's fixed scratch array on the
+ * current device instead.
  */
 ft_status fourtune_device_status(void* ws, int32_t* status_out, void* stream);
 

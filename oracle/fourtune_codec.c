@@ -14,7 +14,7 @@
  *   - section 3.2 and Table 5: the blocks are 16x16 tiles of the stored matrix, so
  *     the transpose of a quantized matrix reuses the same codes and scales.
  *
- * Readings taken where the pages are silent (the same list is in the design notes):
+ * Readings taken where the pages are silent:
  *   - NVFP4 two-level scaling: one fp32 factor g per tensor, g = 2688 / amax_t
  *     (2688 = 6 * 448 maps the tensor max to the largest E2M1 value times the
  *     largest UE4M3 value), and one UE4M3 scale per 16x16 block;

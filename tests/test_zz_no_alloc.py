@@ -6,8 +6,9 @@ owned by another runtime.  Its scratch lives in a fixed array inside the library
 test calls it through the C ABI and checks that it gives exactly what the workspace entry
 point gives on the same inputs, on two calls in a row (the second with other data, so
 nothing left in the shared array from the first call can leak into the second), and that
-a problem too large for the array is refused.  This file is named so that pytest
-collects it last.
+a problem too large for the array is refused.  The array's status word, where a kernel
+would report a bounded wait that gave up, reads back FT_OK through fourtune_device_status
+with a NULL workspace.  This file is named so that pytest collects it last.
 """
 import ctypes
 
@@ -39,6 +40,14 @@ def _noalloc(ft, x, down):
     return q, t
 
 
+def _noalloc_status(ft):
+    v = ctypes.c_int32(-1)
+    st = ft.lib().fourtune_device_status(None, ctypes.byref(v),
+                                         ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    assert st == 0, ft.STATUS.get(st, st)
+    return int(v.value)
+
+
 def test_noalloc_matches_the_workspace_entry_point_on_two_calls():
     ft = _ft()
     for seed, (rows, cols) in ((0, (1024, 3072)), (1, (512, 1536))):
@@ -53,6 +62,8 @@ def test_noalloc_matches_the_workspace_entry_point_on_two_calls():
         assert torch.equal(q.sf_mma, q_ref.sf_mma)
         # the down-projection within the tolerance the other tests use against fp64
         assert ora.rel_frobenius(t.double().cpu().numpy(), t_ref.double().cpu().numpy()) < 1e-5
+        # the fixed array's status word (read and cleared with a NULL workspace): no timeout
+        assert _noalloc_status(ft) == 0
 
 
 def test_noalloc_refuses_problems_beyond_its_scratch():
