@@ -647,9 +647,10 @@ def run_layers(args, desc, specs):
     # per-launch events: every GEMM and quantizer launch of one step (and the forward
     # prologue that takes max|X|), recorded by the library on the launch stream
     GEMM, QUANT, AMAX = ft.FT_KERNEL_GEMM, ft.FT_KERNEL_QUANT, ft.FT_KERNEL_AMAX
+    LOWRANK, DB, DA = ft.FT_KERNEL_LOWRANK, ft.FT_KERNEL_LORA_DB, ft.FT_KERNEL_LORA_DA
     nL = len(layers)
-    kev = {(k, i): (E(), E()) for k in (GEMM, QUANT) for i in range(2 * nL)}
-    kev.update({(AMAX, i): (E(), E()) for i in range(nL)})
+    kev = {(k, i): (E(), E()) for k in (GEMM, QUANT, LOWRANK) for i in range(2 * nL)}
+    kev.update({(k, i): (E(), E()) for k in (AMAX, DB, DA) for i in range(nL)})
     xp_ev = [(E(), E()) for _ in range(nL)]
     for ev in [e for p_ in list(kev.values()) + xp_ev for e in p_]:
         ev.record()  # torch creates the CUDA event on first record; the library needs the handle
@@ -657,13 +658,15 @@ def run_layers(args, desc, specs):
 
     def step_with_events():
         for i, L in enumerate(layers):
-            for k in (GEMM, QUANT):
+            for k in (GEMM, QUANT, LOWRANK):
                 ft.time_next_launch(k, *kev[(k, i)])
             ft.time_next_launch(AMAX, *kev[(AMAX, i)])
             L.fwd()
         for j, L in enumerate(reversed(layers)):
-            for k in (GEMM, QUANT):
+            for k in (GEMM, QUANT, LOWRANK):
                 ft.time_next_launch(k, *kev[(k, nL + j)])
+            for k in (DB, DA):
+                ft.time_next_launch(k, *kev[(k, j)])
             L.bwd()
 
     def bwd_xpose_with_events():  # each layer's dX GEMM is its backward's last GEMM launch
@@ -704,7 +707,7 @@ def run_layers(args, desc, specs):
             variants[name]()
 
     ev_s, ev_e = [E() for _ in range(Kst)], [E() for _ in range(Kst)]
-    gemm_ms, quant_ms, amax_ms, xp_gemm_ms = [], [], [], []
+    gemm_ms, quant_ms, amax_ms, xp_gemm_ms, other_ms = [], [], [], [], []
     pass_ms = {}
     if world > 1:
         dist.barrier()
@@ -736,6 +739,9 @@ def run_layers(args, desc, specs):
             gemm_ms.append([kev[(GEMM, j)][0].elapsed_time(kev[(GEMM, j)][1]) for j in range(2 * nL)])
             quant_ms.append([kev[(QUANT, j)][0].elapsed_time(kev[(QUANT, j)][1]) for j in range(2 * nL)])
             amax_ms.append([kev[(AMAX, j)][0].elapsed_time(kev[(AMAX, j)][1]) for j in range(nL)])
+            other_ms.append({name: [kev[(k, j)][0].elapsed_time(kev[(k, j)][1]) for j in range(n)]
+                             for name, k, n in (("lowrank_finalize", LOWRANK, 2 * nL), ("lora_grad_db", DB, nL),
+                                                ("lora_grad_da", DA, nL))})
         # per-pass figures: forward alone, backward alone, 1x16 forward, transposing backward
         for name in ("fwd", "bwd", "fwd_1x16", "bwd_xpose"):
             ts = []
@@ -795,7 +801,7 @@ def run_layers(args, desc, specs):
         fp4_peak = bf16_peak * NOMINAL_FP4_OVER_BF16
         # the GEMM launches of a step, in order: each layer's forward, then the backward's
         # dX GEMMs in reverse layer order; FLOPs 2 M N K each
-        gemm_flops = [2.0 * L.spec.M * L.spec.N * L.spec.K for L in layers] * 2
+        gemm_flops = [2.0 * L.spec.M * L.spec.N * L.spec.K for L in layers + list(reversed(layers))]
         gemm_avg = statistics.mean(sum(r) for r in gemm_ms) / len(gemm_flops)
         achieved = statistics.mean(gemm_flops) / (gemm_avg * 1e-3) / 1e12
         per_launch = []
@@ -845,6 +851,8 @@ def run_layers(args, desc, specs):
                           "frac": q_gbs / hbm, "frac_with_amax": qa_gbs / hbm,
                           "launch_ms": q_ms, "amax_pass_ms": a_ms,
                           "bytes_per_element": "2 (read) + 0.5 (codes) + 1/256 (block scales), + 4 R per row"},
+            "other_kernels_ms": {name: [statistics.mean(r[name][j] for r in other_ms)
+                                        for j in range(len(other_ms[0][name]))] for name in other_ms[0]},
             "per_pass": {"fwd_ms": pass_ms["fwd"], "fwd_tflops": fl_f / (pass_ms["fwd"] * 1e-3) / 1e12,
                          "bwd_ms": pass_ms["bwd"], "bwd_tflops": fl_b / (pass_ms["bwd"] * 1e-3) / 1e12,
                          "fwd_1x16_ms": pass_ms["fwd_1x16"],

@@ -240,16 +240,23 @@ bool pair_gemm(int64_t M, const DeviceInfo& dev) { return (M % 256) == 0 && dev.
 // act_out, also act_out = bf16(gelu_tanh(out)) and max |act_out| into *act_amax.  When
 // b.codes is null, b_src holds B's codes transposed ([K, N/2] bytes: the stored Q(R) for
 // the dX GEMM) and the GEMM transposes its tiles in shared memory; b.sf_mma is B's own.
-ft_status run_gemm(const uint8_t* a_codes, const uint8_t* a_sf, const float* ga, const ft_fp4& b,
-                   const __nv_bfloat16* la, const __nv_bfloat16* lb, int KL, int64_t M, int64_t N,
-                   int64_t K, void* out, int* status, const DeviceInfo& dev, cudaStream_t st,
+// The pair kernel reads A's and B's scales from their compact 16x16-block grids when it
+// has them (a_grid: A's [M/16, K/16] grid, or null for 1x16 groups; B's grid is b.scales
+// unless B's codes are transposed on the fly), else from the tensor-core scale layouts
+// (a_sf, b.sf_mma), which the one-CTA kernel always uses.
+ft_status run_gemm(const uint8_t* a_codes, const uint8_t* a_sf, const uint8_t* a_grid, const float* ga,
+                   const ft_fp4& b, const __nv_bfloat16* la, const __nv_bfloat16* lb, int KL, int64_t M,
+                   int64_t N, int64_t K, void* out, int* status, const DeviceInfo& dev, cudaStream_t st,
                    void* act_out = nullptr, float* act_amax = nullptr, const void* gelu_in = nullptr,
                    const ft::LoraFinalizeJob* side = nullptr, const uint8_t* b_src = nullptr) {
     const bool pair = pair_gemm(M, dev);
     const uint32_t b_rows = pair ? 128 : 256;
     const bool xpose = b.codes == nullptr;
     if (xpose && (!b_src || act_out)) return FT_ERR_INVALID_ARG;
-    CUtensorMap tA, tB, tLA, tLB;
+    const bool grid_a = pair && a_grid != nullptr;
+    const bool grid_b = pair && !xpose && b.scales != nullptr;
+    if ((!grid_a && !a_sf) || (!grid_b && !b.sf_mma)) return FT_ERR_INVALID_ARG;
+    CUtensorMap tA, tB, tLA, tLB, tSA, tSB;
     FT_TRY(make_tmap(&tA, a_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, K / 2, M, K / 2, 128, 128));
     if (xpose)  // slabs of 256 rows of B^T by this CTA's b_rows columns (b_rows / 2 bytes)
         FT_TRY(make_tmap(&tB, b_src, CU_TENSOR_MAP_DATA_TYPE_UINT8, N / 2, K, N / 2, b_rows / 2, 256,
@@ -263,6 +270,18 @@ ft_status run_gemm(const uint8_t* a_codes, const uint8_t* a_sf, const float* ga,
         tLA = tA;
         tLB = tB;
     }
+    // scale grids: uint8 [rows/16, cols/16]; a k step takes 16 block-columns of a CTA's 8
+    // block-rows of A and of the pair tile's 16 block-rows of B (no swizzle)
+    if (grid_a)
+        FT_TRY(make_tmap(&tSA, a_grid, CU_TENSOR_MAP_DATA_TYPE_UINT8, K / 16, M / 16, K / 16, 16, 8,
+                         CU_TENSOR_MAP_SWIZZLE_NONE));
+    else
+        tSA = tA;
+    if (grid_b)
+        FT_TRY(make_tmap(&tSB, b.scales, CU_TENSOR_MAP_DATA_TYPE_UINT8, K / 16, N / 16, K / 16, 16, 16,
+                         CU_TENSOR_MAP_SWIZZLE_NONE));
+    else
+        tSB = tB;
     CUtensorMap tOut, tAct;
     FT_TRY(make_tmap(&tOut, out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, N, M, N * 2, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B));
     if (act_out)
@@ -290,8 +309,13 @@ ft_status run_gemm(const uint8_t* a_codes, const uint8_t* a_sf, const float* ga,
         g.side1 = side[1];
     }
     g.xpose = xpose ? 1 : 0;
+    g.sfc = (grid_a ? 1 : 0) | (grid_b ? 2 : 0);
+    // The tiles that run at the same time share one operand's panels and together sweep all
+    // of the other's: make the swept operand the smaller one (A is M x K codes, B N x K), so
+    // that it stays in L2 between its sweeps instead of coming from HBM again.
+    g.n_inner = N < M ? 1 : 0;
     if (pair)
-        FT_CUDA(ft::launch_gemm_fp4_lowrank_pair(tA, tB, tLA, tLB, tOut, tAct, g, dev.num_sms, st));
+        FT_CUDA(ft::launch_gemm_fp4_lowrank_pair(tA, tB, tLA, tLB, tOut, tAct, tSA, tSB, g, dev.num_sms, st));
     else
         FT_CUDA(ft::launch_gemm_fp4_lowrank(tA, tB, tLA, tLB, tOut, tAct, g, dev.num_sms, st));
     return FT_OK;
@@ -533,9 +557,12 @@ ft_status linear_fwd_impl(const ft_linear* L, const void* x_dev, int64_t M, cons
                                          L->r_s, L->r, Rp, KL, R > 0 ? bfm(W + w.dn) : nullptr,
                                          R > 0 ? bfm(W + w.upcat) : nullptr, nullptr, nullptr, &ex, st));
     int splits = 1;
+    // the pair GEMM reads Q(X)'s compact block grid; 1x16 groups and the one-CTA GEMM need
+    // the tensor-core scale layout
+    const bool x_grid = pair_gemm(M, dev) && x_block_rows == 16;
     FT_TRY(quantize_operand(x_dev, M, K, K, amax_or_null, scal + SC_AMAX_X, R > 0, W + w.qx_codes, W + w.qx_scales,
-                            W + w.qx_sf, scal + SC_G_X, W + w.dn, Rp, partial, &splits, status, dev, st,
-                            x_block_rows, amax_parts));
+                            x_grid ? nullptr : W + w.qx_sf, scal + SC_G_X, W + w.dn, Rp, partial, &splits, status,
+                            dev, st, x_block_rows, amax_parts));
     if (R > 0) {
         ft::LowRankFinalizeArgs f{};
         f.partial = partial;
@@ -552,8 +579,9 @@ ft_status linear_fwd_impl(const ft_linear* L, const void* x_dev, int64_t M, cons
         f.KL = KL;
         FT_CUDA(ft::launch_lowrank_finalize(f, st));
     }
-    return run_gemm(W + w.qx_codes, W + w.qx_sf, scal + SC_G_X, L->qr, bf(W + w.tcat), bf(W + w.upcat), KL, M,
-                    N, K, y_dev, status, dev, st, h_dev, h_amax_dev);
+    return run_gemm(W + w.qx_codes, x_grid ? nullptr : W + w.qx_sf, x_grid ? W + w.qx_scales : nullptr,
+                    scal + SC_G_X, L->qr, bf(W + w.tcat), bf(W + w.upcat), KL, M, N, K, y_dev, status, dev, st,
+                    h_dev, h_amax_dev);
 }
 
 }  // namespace
@@ -655,8 +683,10 @@ ft_status linear_bwd_impl(const ft_linear* L, const void* x_dev, const float* t_
         fin[1] = ft::LoraFinalizeJob{g.partial, sp, static_cast<int>(N), NBW, L->r, L->lora_scale, false, db_dev};
     }
     int splits = 1;
+    const bool g_grid = pair_gemm(M, dev);  // the pair GEMM reads Q(G)'s compact block grid
     FT_TRY(quantize_operand(dy_dev, M, N, N, amax_g, scal + SC_AMAX_G, R > 0, W + w.qg_codes, W + w.qg_scales,
-                            W + w.qg_sf, scal + SC_G_G, W + w.upt, Rp, partial, &splits, status, dev, st));
+                            g_grid ? nullptr : W + w.qg_sf, scal + SC_G_G, W + w.upt, Rp, partial, &splits, status,
+                            dev, st));
     if (R > 0) {
         ft::LowRankFinalizeArgs f{};
         f.partial = partial;
@@ -701,9 +731,9 @@ ft_status linear_bwd_impl(const ft_linear* L, const void* x_dev, const float* t_
         if (!side) FT_CUDA(ft::launch_lora_grad_finalize(fin[0], fin[1], st));
     }
     // The dX GEMM goes last: the GEMM's operand and output traffic would evict G from L2.
-    FT_TRY(run_gemm(W + w.qg_codes, W + w.qg_sf, scal + SC_G_G, L->qr_t, bf(W + w.ucat), bf(W + w.dntcat), KL,
-                    M, K, N, dx_dev, status, dev, st, nullptr, nullptr, gelu_in, side ? fin : nullptr,
-                    L->qr.codes));
+    FT_TRY(run_gemm(W + w.qg_codes, g_grid ? nullptr : W + w.qg_sf, g_grid ? W + w.qg_scales : nullptr,
+                    scal + SC_G_G, L->qr_t, bf(W + w.ucat), bf(W + w.dntcat), KL, M, K, N, dx_dev, status, dev, st,
+                    nullptr, nullptr, gelu_in, side ? fin : nullptr, L->qr.codes));
     return FT_OK;
 }
 

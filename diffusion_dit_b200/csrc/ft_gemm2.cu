@@ -45,6 +45,9 @@ constexpr int B_BYTES = BN_CTA * BK_BYTES;  // 16 KB
 constexpr int SFA_BYTES = 4 * 512;
 constexpr int SFB_BYTES = 2 * 4 * 512;
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;  // 38912
+// the compact grids of 16x16-block scales one k step needs (they fit in the atoms' regions)
+constexpr int SFA_GRID_BYTES = 8 * 16;   // 8 block-rows x 16 block-columns
+constexpr int SFB_GRID_BYTES = 16 * 16;  // the pair tile's 16 block-rows
 constexpr int OFF_B = A_BYTES;
 constexpr int OFF_SFA = A_BYTES + B_BYTES;
 constexpr int OFF_SFB = OFF_SFA + SFA_BYTES;
@@ -102,14 +105,23 @@ __device__ __forceinline__ bool xpose_share(uint32_t slab, int q, int lane, uint
     return true;
 }
 
-template <int EPI, bool XP>
+// SFC bit 0: A's scales come from its compact 16x16-block grid (tmSA), bit 1: B's (tmSB);
+// otherwise from the tensor-core scale layout (p.sfa / p.sfb).
+template <int EPI, bool XP, int SFC>
 __global__ void __launch_bounds__(threads(EPI), 1)
     gemm_fp4_lowrank_pair_kernel(const __grid_constant__ CUtensorMap tmA,
                                  const __grid_constant__ CUtensorMap tmB,
                                  const __grid_constant__ CUtensorMap tmLA,
                                  const __grid_constant__ CUtensorMap tmLB,
                                  const __grid_constant__ CUtensorMap tmOut,
-                                 const __grid_constant__ CUtensorMap tmAct, const GemmFp4Args p) {
+                                 const __grid_constant__ CUtensorMap tmAct,
+                                 const __grid_constant__ CUtensorMap tmSA,
+                                 const __grid_constant__ CUtensorMap tmSB, const GemmFp4Args p) {
+    constexpr bool kGridA = (SFC & 1) != 0;
+    constexpr bool kGridB = (SFC & 2) != 0;
+    // bytes one k step's scales add to a stage: a 128-row band's grid rows (8 x 16 B) or its
+    // four 512-byte atoms; the pair tile's 256 B rows: 16 x 16 B or eight atoms
+    constexpr uint32_t kSfBytes = (kGridA ? SFA_GRID_BYTES : SFA_BYTES) + (kGridB ? SFB_GRID_BYTES : SFB_BYTES);
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_u32 = smem_u32(smem_raw);
     const uint32_t pad = (1024 - (raw_u32 & 1023)) & 1023;
@@ -153,6 +165,8 @@ __global__ void __launch_bounds__(threads(EPI), 1)
     if (warp == 0 && lane == 0) {
         tma_prefetch_desc(&tmA);
         tma_prefetch_desc(&tmB);
+        if constexpr (kGridA) tma_prefetch_desc(&tmSA);
+        if constexpr (kGridB) tma_prefetch_desc(&tmSB);
         if (KLS > 0) {
             tma_prefetch_desc(&tmLA);
             tma_prefetch_desc(&tmLB);
@@ -183,26 +197,33 @@ __global__ void __launch_bounds__(threads(EPI), 1)
                 if (++s == STAGES) { s = 0; ph ^= 1; }
             };
             for (int t = pair; t < num_tiles && !*abort_flag; t += num_pairs) {
-                const int mb2 = t % MB2, nb = t / MB2;
+                const int mb2 = p.n_inner ? t / NB : t % MB2, nb = p.n_inner ? t % NB : t / MB2;
                 const int m_band = mb2 * 2 + static_cast<int>(rank);            // this CTA's A rows
                 const int n_rows = nb * BN + BN_CTA * static_cast<int>(rank);  // this CTA's B rows
                 for (int kt = 0; kt < KT; ++kt, advance()) {
                     if (!acquire()) break;
                     const uint32_t full = bar(BAR_FULL(s));
                     const uint32_t st = stage(s);
-                    mbar_arrive_expect_tx(full, STAGE_BYTES);
+                    mbar_arrive_expect_tx(full, A_BYTES + B_BYTES + kSfBytes);
                     tma_load_2d(st, &tmA, full, kt * BK_BYTES, m_band * BM);
                     if constexpr (XP)  // B^T rows kt*256.., bytes of this CTA's 128 columns
                         tma_load_2d(st + OFF_B, &tmB, full, n_rows / 2, kt * 256);
                     else
                         tma_load_2d(st + OFF_B, &tmB, full, kt * BK_BYTES, n_rows);
-                    bulk_load(st + OFF_SFA, p.sfa + (static_cast<size_t>(m_band) * k64 + kt * 4) * 512,
-                              SFA_BYTES, full);
+                    if constexpr (kGridA)  // block-rows of this CTA's 128 A rows, 16 block-columns
+                        tma_load_2d(st + OFF_SFA, &tmSA, full, kt * 16, m_band * (BM / 16));
+                    else
+                        bulk_load(st + OFF_SFA, p.sfa + (static_cast<size_t>(m_band) * k64 + kt * 4) * 512,
+                                  SFA_BYTES, full);
+                    if constexpr (kGridB) {  // the pair tile's 16 block-rows of B
+                        tma_load_2d(st + OFF_SFB, &tmSB, full, kt * 16, nb * (BN / 16));
+                    } else {
 #pragma unroll
-                    for (int rb = 0; rb < 2; ++rb)
-                        bulk_load(st + OFF_SFB + rb * 2048,
-                                  p.sfb + (static_cast<size_t>(nb * 2 + rb) * k64 + kt * 4) * 512, 2048,
-                                  full);
+                        for (int rb = 0; rb < 2; ++rb)
+                            bulk_load(st + OFF_SFB + rb * 2048,
+                                      p.sfb + (static_cast<size_t>(nb * 2 + rb) * k64 + kt * 4) * 512, 2048,
+                                      full);
+                    }
                 }
                 if (*abort_flag) break;
                 for (int kl = 0; kl < KLS; ++kl, advance()) {
@@ -288,18 +309,48 @@ __global__ void __launch_bounds__(threads(EPI), 1)
                 if (!mbar_wait(bar(BAR_FULL(s)), ph, abort_flag, p.status)) { ok = false; break; }
                 if (j < KT) {
                     const uint8_t* st = base + s * STAGE_BYTES;
+                    // va[4 i + w]: word w (rows lane + 32 w) of A's atom i (k-blocks 4i..4i+3);
+                    // vb0 / vb1: B's atoms 0-1 / 2-3, each as [rows 0-127: 4 words, rows 128-255: 4]
                     uint32_t va[16], vb0[16], vb1[16];
+                    if constexpr (kGridA) {
+                        // rows lane + 32 w lie in block-row lane / 16 + 2 w: its 16 block scales
+                        // (one 16-byte grid row) give word w of all four atoms
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const uint4 a = *reinterpret_cast<const uint4*>(st + OFF_SFA + 512 * i + 16 * lane);
-                        const uint4 b0 = *reinterpret_cast<const uint4*>(st + OFF_SFB + 512 * i + 16 * lane);
-                        const uint4 b1 =
-                            *reinterpret_cast<const uint4*>(st + OFF_SFB + 2048 + 512 * i + 16 * lane);
-                        uint32_t* vb = i < 2 ? vb0 : vb1;
-                        const int o = 8 * (i & 1);
-                        va[4 * i] = a.x; va[4 * i + 1] = a.y; va[4 * i + 2] = a.z; va[4 * i + 3] = a.w;
-                        vb[o] = b0.x; vb[o + 1] = b0.y; vb[o + 2] = b0.z; vb[o + 3] = b0.w;
-                        vb[o + 4] = b1.x; vb[o + 5] = b1.y; vb[o + 6] = b1.z; vb[o + 7] = b1.w;
+                        for (int w = 0; w < 4; ++w) {
+                            const uint4 g = *reinterpret_cast<const uint4*>(st + OFF_SFA + ((lane >> 4) + 2 * w) * 16);
+                            va[w] = g.x; va[4 + w] = g.y; va[8 + w] = g.z; va[12 + w] = g.w;
+                        }
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            const uint4 a = *reinterpret_cast<const uint4*>(st + OFF_SFA + 512 * i + 16 * lane);
+                            va[4 * i] = a.x; va[4 * i + 1] = a.y; va[4 * i + 2] = a.z; va[4 * i + 3] = a.w;
+                        }
+                    }
+                    if constexpr (kGridB) {
+#pragma unroll
+                        for (int rb = 0; rb < 2; ++rb) {
+#pragma unroll
+                            for (int w = 0; w < 4; ++w) {
+                                const uint4 g = *reinterpret_cast<const uint4*>(
+                                    st + OFF_SFB + (8 * rb + (lane >> 4) + 2 * w) * 16);
+                                vb0[4 * rb + w] = g.x;
+                                vb0[8 + 4 * rb + w] = g.y;
+                                vb1[4 * rb + w] = g.z;
+                                vb1[8 + 4 * rb + w] = g.w;
+                            }
+                        }
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            const uint4 b0 = *reinterpret_cast<const uint4*>(st + OFF_SFB + 512 * i + 16 * lane);
+                            const uint4 b1 =
+                                *reinterpret_cast<const uint4*>(st + OFF_SFB + 2048 + 512 * i + 16 * lane);
+                            uint32_t* vb = i < 2 ? vb0 : vb1;
+                            const int o = 8 * (i & 1);
+                            vb[o] = b0.x; vb[o + 1] = b0.y; vb[o + 2] = b0.z; vb[o + 3] = b0.w;
+                            vb[o + 4] = b1.x; vb[o + 5] = b1.y; vb[o + 6] = b1.z; vb[o + 7] = b1.w;
+                        }
                     }
                     tmem_st_32x32b_x16(lane_base + COL_SFA + 16 * s, va);
                     tmem_st_32x32b_x16(lane_base + COL_SFB + 32 * s, vb0);
@@ -333,7 +384,7 @@ __global__ void __launch_bounds__(threads(EPI), 1)
         int sc = 0;         // stores staged by this warp (staging buffer sc % 2)
         int ti = 0;
         for (int t = pair; t < num_tiles && !*abort_flag; t += num_pairs, ++ti) {
-            const int mb2 = t % MB2, nb = t / MB2;
+            const int mb2 = p.n_inner ? t / NB : t % MB2, nb = p.n_inner ? t % NB : t / MB2;
             if (!mbar_wait(bar(BAR_TMEM_FULL), ti & 1, abort_flag, p.status)) break;
             tc_fence_after();
             if constexpr (EPI == kEpiGeluBwd) {
@@ -455,18 +506,19 @@ __global__ void __launch_bounds__(threads(EPI), 1)
 namespace {
 
 // One variant: its own instantiation, its shared-memory opt-in set once.
-template <int EPI, bool XP>
+template <int EPI, bool XP, int SFC>
 cudaError_t launch_variant(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmLA,
                            const CUtensorMap& tmLB, const CUtensorMap& tmOut, const CUtensorMap& tmAct,
-                           const GemmFp4Args& args, cudaLaunchConfig_t cfg) {
+                           const CUtensorMap& tmSA, const CUtensorMap& tmSB, const GemmFp4Args& args,
+                           cudaLaunchConfig_t cfg) {
     using namespace gemm2;
     static const cudaError_t attr = cudaFuncSetAttribute(
-        gemm_fp4_lowrank_pair_kernel<EPI, XP>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes(EPI));
+        gemm_fp4_lowrank_pair_kernel<EPI, XP, SFC>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes(EPI));
     if (attr != cudaSuccess) return attr;
     cfg.blockDim = dim3(threads(EPI));
     cfg.dynamicSmemBytes = smem_bytes(EPI);
-    return cudaLaunchKernelEx(&cfg, gemm_fp4_lowrank_pair_kernel<EPI, XP>, tmA, tmB, tmLA, tmLB, tmOut, tmAct,
-                              args);
+    return cudaLaunchKernelEx(&cfg, gemm_fp4_lowrank_pair_kernel<EPI, XP, SFC>, tmA, tmB, tmLA, tmLB, tmOut, tmAct,
+                              tmSA, tmSB, args);
 }
 
 }  // namespace
@@ -474,6 +526,7 @@ cudaError_t launch_variant(const CUtensorMap& tmA, const CUtensorMap& tmB, const
 cudaError_t launch_gemm_fp4_lowrank_pair(const CUtensorMap& tmA, const CUtensorMap& tmB,
                                          const CUtensorMap& tmLA, const CUtensorMap& tmLB,
                                          const CUtensorMap& tmOut, const CUtensorMap& tmAct,
+                                         const CUtensorMap& tmSA, const CUtensorMap& tmSB,
                                          const GemmFp4Args& args, int num_sms, cudaStream_t stream) {
     using namespace gemm2;
     const int tiles = (args.M / (2 * BM)) * (args.N / BN);
@@ -492,16 +545,21 @@ cudaError_t launch_gemm_fp4_lowrank_pair(const CUtensorMap& tmA, const CUtensorM
     cfg.attrs = at;
     cfg.numAttrs = 2;
     before_launch(K_GEMM, stream);
-    // the transposing variants serve the backward's dX GEMM (plain or GELU-backward epilogue)
-    cudaError_t e;
-    if (args.xpose)
-        e = args.act_out ? cudaErrorInvalidValue
-            : args.gelu_in ? launch_variant<kEpiGeluBwd, true>(tmA, tmB, tmLA, tmLB, tmOut, tmAct, args, cfg)
-                           : launch_variant<kEpiPlain, true>(tmA, tmB, tmLA, tmLB, tmOut, tmAct, args, cfg);
-    else
-        e = args.gelu_in ? launch_variant<kEpiGeluBwd, false>(tmA, tmB, tmLA, tmLB, tmOut, tmAct, args, cfg)
-            : args.act_out ? launch_variant<kEpiGelu, false>(tmA, tmB, tmLA, tmLB, tmOut, tmAct, args, cfg)
-                           : launch_variant<kEpiPlain, false>(tmA, tmB, tmLA, tmLB, tmOut, tmAct, args, cfg);
+    // Instantiations: the transposing variants serve the backward's dX GEMM (plain or
+    // GELU-backward epilogue; Q(R)^T's scales from its tensor-core layout); A's scales come
+    // from the tensor-core layout only for 1x16 groups (the plain forward).
+    cudaError_t e = cudaErrorInvalidValue;
+#define FT_PAIR(E, X, S) launch_variant<E, X, S>(tmA, tmB, tmLA, tmLB, tmOut, tmAct, tmSA, tmSB, args, cfg)
+    const int sfc = args.sfc;
+    if (args.xpose) {
+        if (sfc == 1 && !args.act_out) e = args.gelu_in ? FT_PAIR(kEpiGeluBwd, true, 1) : FT_PAIR(kEpiPlain, true, 1);
+    } else if (sfc == 3) {
+        e = args.gelu_in ? FT_PAIR(kEpiGeluBwd, false, 3)
+            : args.act_out ? FT_PAIR(kEpiGelu, false, 3) : FT_PAIR(kEpiPlain, false, 3);
+    } else if (sfc == 2 && !args.gelu_in && !args.act_out) {
+        e = FT_PAIR(kEpiPlain, false, 2);
+    }
+#undef FT_PAIR
     after_launch(K_GEMM, stream);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();

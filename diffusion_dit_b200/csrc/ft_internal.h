@@ -82,6 +82,13 @@ struct GemmFp4Args {
     // non-zero: tmB holds B^T untransposed ([K rows, N/2 bytes], box 256 rows), and the
     // scale warps transpose each tile in shared memory (ft_xpose.cuh); sfb is B's layout
     int xpose;
+    // pair kernel: bit 0 set = A's scales from its compact 16x16-block grid through tmSA
+    // (uint8 [M/16, K/16], box 16 x 8), bit 1 = B's through tmSB ([N/16, K/16], box 16 x 16);
+    // a clear bit = that operand's tensor-core scale layout (sfa / sfb)
+    int sfc;
+    // pair kernel tile order: 0 = row bands fastest (consecutive tiles share B's panel and
+    // sweep all of A), 1 = column tiles fastest (they share A's panel and sweep all of B)
+    int n_inner;
 };
 
 // tmOut (and tmAct): bf16 [M, N] output, box 32 x 32, 64-byte swizzle.  tmB: 128 x 256
@@ -97,6 +104,7 @@ cudaError_t launch_gemm_fp4_lowrank(const CUtensorMap& tmA, const CUtensorMap& t
 cudaError_t launch_gemm_fp4_lowrank_pair(const CUtensorMap& tmA, const CUtensorMap& tmB,
                                          const CUtensorMap& tmLA, const CUtensorMap& tmLB,
                                          const CUtensorMap& tmOut, const CUtensorMap& tmAct,
+                                         const CUtensorMap& tmSA, const CUtensorMap& tmSB,
                                          const GemmFp4Args& args, int num_sms, cudaStream_t stream);
 
 // quantizer and helpers (ft_quant.cu)

@@ -133,7 +133,7 @@ __global__ void build_factors_kernel(const __nv_bfloat16* __restrict__ ls_down,
     if (x.zero_slot && t0 == 0) *x.zero_slot = 0.0f;
     if (x.zero_slot2 && t0 == 0) *x.zero_slot2 = 0.0f;
     // side job: max |x| of the call's input (the bulk of this launch when present), one
-    // partial per CTA; four independent 16-byte loads in flight per thread per trip
+    // partial per CTA; eight independent 16-byte loads in flight per thread per trip
     if (x.max_src) {
         const int64_t vpr = x.max_cols / 8;
         const int64_t nvec = x.max_rows * vpr;
@@ -145,16 +145,21 @@ __global__ void build_factors_kernel(const __nv_bfloat16* __restrict__ ls_down,
             for (int e = 0; e < 4; ++e)
                 m = fmaxf(m, fmaxf(fabsf(bf16lo_to_f32(w[e])), fabsf(bf16hi_to_f32(w[e]))));
         };
+        // a dense matrix (row stride == columns, as the layer calls pass it) is one flat run
+        // of 16-byte vectors: no index division per load
+        const bool flat = x.max_ld == x.max_cols;
+        const uint4* flat_src = reinterpret_cast<const uint4*>(x.max_src);
         auto at = [&](int64_t iv) {
-            return *reinterpret_cast<const uint4*>(x.max_src + (iv / vpr) * x.max_ld + (iv % vpr) * 8);
+            return flat ? flat_src[iv]
+                        : *reinterpret_cast<const uint4*>(x.max_src + (iv / vpr) * x.max_ld + (iv % vpr) * 8);
         };
         int64_t i = t0;
-        for (; i + 3 * gstride < nvec; i += 4 * gstride) {
-            uint4 v[4];
+        for (; i + 7 * gstride < nvec; i += 8 * gstride) {  // eight independent loads in flight
+            uint4 v[8];
 #pragma unroll
-            for (int u = 0; u < 4; ++u) v[u] = at(i + u * gstride);
+            for (int u = 0; u < 8; ++u) v[u] = at(i + u * gstride);
 #pragma unroll
-            for (int u = 0; u < 4; ++u) vmax(v[u]);
+            for (int u = 0; u < 8; ++u) vmax(v[u]);
         }
         for (; i < nvec; i += gstride) vmax(at(i));
 #pragma unroll

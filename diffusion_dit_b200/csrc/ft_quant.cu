@@ -64,14 +64,14 @@ __global__ void __launch_bounds__(256) amax_kernel(const T* __restrict__ x, int6
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
     float m = 0.0f;
     int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+    // a dense matrix (ld == cols) is one flat run of 8-element vectors: no index division
+    const bool flat = ld == cols;
+    auto at = [&](int64_t iv) { return flat ? x + iv * 8 : x + (iv / vec_per_row) * ld + (iv % vec_per_row) * 8; };
     // four independent 8-element loads in flight per thread per trip
     for (; i + 3 * stride < nvec; i += 4 * stride) {
         float v[4][8];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            const int64_t iu = i + u * stride;
-            load8(x + (iu / vec_per_row) * ld + (iu % vec_per_row) * 8, v[u]);
-        }
+        for (int u = 0; u < 4; ++u) load8(at(i + u * stride), v[u]);
 #pragma unroll
         for (int u = 0; u < 4; ++u)
 #pragma unroll
@@ -79,7 +79,7 @@ __global__ void __launch_bounds__(256) amax_kernel(const T* __restrict__ x, int6
     }
     for (; i < nvec; i += stride) {
         float v[8];
-        load8(x + (i / vec_per_row) * ld + (i % vec_per_row) * 8, v);
+        load8(at(i), v);
 #pragma unroll
         for (int j = 0; j < 8; ++j) m = fmaxf(m, fabsf(v[j]));
     }

@@ -226,12 +226,49 @@ class Split:
     sigma: np.ndarray      # fp64 top singular values found
 
 
+def jacobi_svd(B: np.ndarray, tol: float = 1e-15, max_sweeps: int = 60):
+    """Thin SVD of a small fp64 matrix B [p, n] (p <= n) by one-sided (Hestenes) Jacobi
+    rotations, written out: the p rows of B are rotated in pairs until every pair is
+    orthogonal (to `tol` relative), accumulating the rotations in V [p, p].  Then the row
+    norms are the singular values and B = V diag(S) Q with Q the normalised rows.  Returns
+    (U [p, p], S [p] descending, Vt [p, n]) with B = U diag(S) Vt."""
+    W = np.array(B, dtype=np.float64, copy=True)      # rows are rotated in place
+    p = W.shape[0]
+    V = np.eye(p)
+    for _ in range(max_sweeps):
+        rotated = False
+        for i in range(p - 1):
+            for j in range(i + 1, p):
+                a = W[i] @ W[i]
+                b = W[j] @ W[j]
+                c = W[i] @ W[j]
+                if abs(c) <= tol * np.sqrt(a * b) or c == 0.0:
+                    continue
+                rotated = True
+                # the rotation that zeroes the (i, j) entry of the 2x2 Gram matrix
+                zeta = (b - a) / (2.0 * c)
+                t = np.copysign(1.0, zeta) / (abs(zeta) + np.sqrt(1.0 + zeta * zeta))
+                cs = 1.0 / np.sqrt(1.0 + t * t)
+                sn = cs * t
+                wi, wj = W[i].copy(), W[j].copy()
+                W[i], W[j] = cs * wi - sn * wj, sn * wi + cs * wj
+                vi, vj = V[:, i].copy(), V[:, j].copy()
+                V[:, i], V[:, j] = cs * vi - sn * vj, sn * vi + cs * vj
+        if not rotated:
+            break
+    S = np.sqrt(np.einsum("ij,ij->i", W, W))
+    order = np.argsort(-S, kind="stable")
+    S, W, V = S[order], W[order], V[:, order]
+    Vt = W / np.where(S > 0, S, 1.0)[:, None]
+    return V, S, Vt
+
+
 def svd_split(w: torch.Tensor, r_s: int, sweeps: int = 8, oversample: int = 8,
               seed: int = 1234) -> Split:
     """Top-r_s singular triplets of W (bf16 [N, K]) by subspace iteration in fp64:
     a Gaussian start block of width r_s + oversample, ``sweeps`` power sweeps with
     a QR re-orthonormalisation after each product, then Rayleigh-Ritz (the SVD of
-    the small projected matrix).  L_stab = Ls_up Ls_down with sqrt(S) on each
+    the small projected matrix, by the one-sided Jacobi rotations of jacobi_svd).  L_stab = Ls_up Ls_down with sqrt(S) on each
     side, both stored bf16; R = W - Ls_up Ls_down in fp64, rounded once to fp32."""
     W = bf16_f64(w)
     N, K = W.shape
@@ -245,7 +282,7 @@ def svd_split(w: torch.Tensor, r_s: int, sweeps: int = 8, oversample: int = 8,
         Z, _ = np.linalg.qr(W.T @ Q)
         Q, _ = np.linalg.qr(W @ Z)
     Bsmall = Q.T @ W                      # [p, K]
-    Ub, S, Vt = np.linalg.svd(Bsmall, full_matrices=False)
+    Ub, S, Vt = jacobi_svd(Bsmall)        # Rayleigh-Ritz: the small projected problem
     U = Q @ Ub[:, :r_s]                   # [N, r_s]
     S = S[:r_s]
     V = Vt[:r_s].T                        # [K, r_s]

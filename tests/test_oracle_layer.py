@@ -34,6 +34,27 @@ def test_svd_split_reconstructs_w():
     assert np.all(np.abs(R + L - W) <= half_ulp + 1e-30)
 
 
+@pytest.mark.parametrize("shape", [(24, 512), (40, 3072), (8, 9)])
+def test_jacobi_svd_against_lapack(shape):
+    # the oracle's Rayleigh-Ritz step: singular values equal LAPACK's, the factors
+    # reconstruct the matrix and are orthonormal, on a matrix with a wide range of
+    # singular values and two nearly equal ones
+    rng = np.random.default_rng(3)
+    p, n = shape
+    U0, _ = np.linalg.qr(rng.standard_normal((p, p)))
+    V0, _ = np.linalg.qr(rng.standard_normal((n, p)))
+    sig = np.logspace(2, -3, p)
+    if p > 2:
+        sig[1] = sig[2] * (1 + 1e-9)
+    B = U0 @ np.diag(sig) @ V0.T
+    U, S, Vt = ora.jacobi_svd(B)
+    assert np.allclose(S, np.linalg.svd(B, compute_uv=False), rtol=1e-10, atol=1e-13 * sig[0])
+    assert np.allclose(U @ np.diag(S) @ Vt, B, atol=1e-11 * sig[0])
+    assert np.allclose(U.T @ U, np.eye(p), atol=1e-12)
+    assert np.allclose(Vt @ Vt.T, np.eye(p), atol=1e-10)
+    assert np.all(np.diff(S) <= 0)
+
+
 def test_svd_split_singular_values_match_lapack():
     inp = wl.make_layer_inputs(wl.PARITY_SMALL, seed=0)
     W = inp.w.double().numpy()
