@@ -45,12 +45,16 @@ cudaError_t launch_k(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t sme
 // GEMM epilogue variants, one kernel instantiation each (the plain one carries no GELU code)
 enum EpilogueKind { kEpiPlain = 0, kEpiGelu = 1, kEpiGeluBwd = 2 };
 
-// One split sum of the adapter gradients (run by lora_split_sums in ft_sidejobs.cuh):
-// out = s * sum over the splits (in order) of (D[f][j] + D[f][r + j]); out[f][j], or
-// out[j][f] with transpose_out.  out == nullptr: no job.
+// One split sum of the adapter gradients (run by lora_split_sums in ft_sidejobs.cuh): the
+// adapter-gradient kernel ran `ctas` persistent CTAs over U = (F / 128) * chunks units
+// (128-feature tile t, 64-token chunk c; unit t * chunks + c), CTA p taking units
+// [p U / ctas, (p + 1) U / ctas) and leaving the sum over each tile it touched in partial
+// slot p + t, [128][NBW] fp32.  Then
+//   out = s * sum over the CTAs that touched the tile, in order, of (D[f][j] + D[f][r + j])
+// stored as out[f][j], or out[j][f] with transpose_out.  out == nullptr: no job.
 struct LoraFinalizeJob {
-    const float* partial;    // [splits, F, NBW], splits <= 16
-    int splits, F, NBW, r;
+    const float* partial;    // [ctas + F / 128][128][NBW]
+    int ctas, chunks, F, NBW, r;
     float s;
     bool transpose_out;
     float* out;
@@ -188,6 +192,7 @@ struct PrologueExtras {
     float* max_parts = nullptr;
 };
 constexpr int kPrologueCtas = 148 * 4;  // the factor kernel's grid
+constexpr int kFactorCtas = 148;        // of which build the factors when the kernel also takes a max
 
 // Build the concatenated low-rank factors used by the forward and backward GEMMs (and
 // run the side jobs in `extra`, which may be null).  dn and upt get Rp rows (rows
@@ -202,17 +207,17 @@ cudaError_t launch_build_factors(const __nv_bfloat16* ls_down, const __nv_bfloat
 //   partial[split][f][c] = sum over the split's tokens m of P[m, f] V'[m, c]
 struct LoraGradArgs {
     int64_t F;               // features of P [M, F] (multiple of 128)
-    int tokens_per_split;    // multiple of 64
+    int chunks;              // 64-token chunks of P (M / 64)
     int NBW;                 // width of V' = [hi, lo, 0] (multiple of 64, <= 256)
-    uint32_t tmem_cols;      // power of two >= max(32, NBW)
-    float* partial;          // [splits, F, NBW]
+    uint32_t tmem_cols;      // per accumulator (two are allocated): power of two >= max(32, NBW)
+    float* partial;          // [ctas + F / 128][128][NBW] (see LoraFinalizeJob)
     int* status;
     // optional: max |P| over every element of P (each is read by exactly one CTA),
     // accumulated with atomicMax on the float's bits into a slot cleared beforehand
     unsigned* amax_out;
 };
-int lora_grad_splits(int64_t M, int64_t F, int num_sms);
-cudaError_t launch_lora_grad(const CUtensorMap& tmP, const CUtensorMap& tmV, const LoraGradArgs& a, int splits,
+int lora_grad_ctas(int64_t M, int64_t F, int num_sms);
+cudaError_t launch_lora_grad(const CUtensorMap& tmP, const CUtensorMap& tmV, const LoraGradArgs& a, int ctas,
                              int kind, cudaStream_t stream);
 
 }  // namespace ft

@@ -20,41 +20,66 @@
 namespace ft {
 namespace {
 
-// One thread per (row, j < R): fixed-order sum over the splits, then the hi/lo operands.
+// One thread per (row, 4 consecutive j < R): fixed-order sum over the splits (16-byte
+// loads), then the hi/lo operands (8-byte stores).  R, r_s and Rp are multiples of 8, so
+// a group of four never straddles the stabilizer / adapter boundary.
+__device__ __forceinline__ uint32_t bf16x2_bits(__nv_bfloat16 lo, __nv_bfloat16 hi) {
+    return static_cast<uint32_t>(__bfloat16_as_ushort(lo)) | (static_cast<uint32_t>(__bfloat16_as_ushort(hi)) << 16);
+}
+
 __global__ void lowrank_finalize_kernel(const LowRankFinalizeArgs a) {
     pdl_trigger();
     pdl_wait();
     const int rows = static_cast<int>(a.rows);
-    const int total = rows * a.R;
+    const int R4 = a.R / 4;
+    const int total = rows * R4;
     const float g = (a.cat != nullptr) ? __fmul_rn(*a.ga, *a.gb) : 1.0f;
-    const __nv_bfloat16 zero = __float2bfloat16_rn(0.0f);
+    const int r = a.R - a.r_s;
     for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < total; i += gridDim.x * blockDim.x) {
-        const int m = i / a.R;
-        const int j = i - m * a.R;
-        float v = 0.0f;
-        for (int sp = 0; sp < a.splits; ++sp) v += a.partial[(sp * rows + m) * a.Rp + j];
-        if (a.out) a.out[m * a.R + j] = v;
+        const int m = i / R4;
+        const int j = (i - m * R4) * 4;
+        float v[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+        for (int sp = 0; sp < a.splits; ++sp) {
+            const float4 pv =
+                *reinterpret_cast<const float4*>(a.partial + (static_cast<int64_t>(sp) * rows + m) * a.Rp + j);
+            v[0] += pv.x;
+            v[1] += pv.y;
+            v[2] += pv.z;
+            v[3] += pv.w;
+        }
+        if (a.out) *reinterpret_cast<float4*>(a.out + static_cast<int64_t>(m) * a.R + j) = make_float4(v[0], v[1], v[2], v[3]);
         if (a.cat) {
-            const float vs = (j >= a.r_s) ? __fmul_rn(v, a.s) : v;
-            const float gv = __fmul_rn(vs, g);
-            const __nv_bfloat16 hi = __float2bfloat16_rn(gv);
-            a.cat[m * a.KL + j] = hi;
-            a.cat[m * a.KL + a.R + j] = __float2bfloat16_rn(gv - __bfloat162float(hi));
-            if (j < a.KL - 2 * a.R) a.cat[m * a.KL + 2 * a.R + j] = zero;
+            __nv_bfloat16 hi[4], lo[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const float vs = (j >= a.r_s) ? __fmul_rn(v[q], a.s) : v[q];
+                const float gv = __fmul_rn(vs, g);
+                hi[q] = __float2bfloat16_rn(gv);
+                lo[q] = __float2bfloat16_rn(gv - __bfloat162float(hi[q]));
+            }
+            __nv_bfloat16* row = a.cat + static_cast<int64_t>(m) * a.KL;
+            *reinterpret_cast<uint2*>(row + j) = make_uint2(bf16x2_bits(hi[0], hi[1]), bf16x2_bits(hi[2], hi[3]));
+            *reinterpret_cast<uint2*>(row + a.R + j) = make_uint2(bf16x2_bits(lo[0], lo[1]), bf16x2_bits(lo[2], lo[3]));
+            if (j < a.KL - 2 * a.R) *reinterpret_cast<uint2*>(row + 2 * a.R + j) = make_uint2(0u, 0u);
         }
         if (a.lora_cat && j >= a.r_s) {  // adapter-gradient operand [hi(v), lo(v), 0] of the LoRA columns
             const int c = j - a.r_s;
-            const int r = a.R - a.r_s;
-            const __nv_bfloat16 hi = __float2bfloat16_rn(v);
-            a.lora_cat[m * a.NBW + c] = hi;
-            a.lora_cat[m * a.NBW + r + c] = __float2bfloat16_rn(v - __bfloat162float(hi));
-            for (int z = 2 * r + c; z < a.NBW; z += r) a.lora_cat[m * a.NBW + z] = zero;
+            __nv_bfloat16 hi[4], lo[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                hi[q] = __float2bfloat16_rn(v[q]);
+                lo[q] = __float2bfloat16_rn(v[q] - __bfloat162float(hi[q]));
+            }
+            __nv_bfloat16* row = a.lora_cat + static_cast<int64_t>(m) * a.NBW;
+            *reinterpret_cast<uint2*>(row + c) = make_uint2(bf16x2_bits(hi[0], hi[1]), bf16x2_bits(hi[2], hi[3]));
+            *reinterpret_cast<uint2*>(row + r + c) = make_uint2(bf16x2_bits(lo[0], lo[1]), bf16x2_bits(lo[2], lo[3]));
+            for (int z = 2 * r + c; z < a.NBW; z += r) *reinterpret_cast<uint2*>(row + z) = make_uint2(0u, 0u);
         }
     }
     if (a.cat && a.KL - 2 * a.R > a.R) {  // zero padding wider than R columns
         const int w = a.KL - 2 * a.R;
         for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < rows * w; i += gridDim.x * blockDim.x)
-            a.cat[(i / w) * a.KL + 2 * a.R + (i % w)] = zero;
+            a.cat[(i / w) * a.KL + 2 * a.R + (i % w)] = __float2bfloat16_rn(0.0f);
     }
 }
 
@@ -72,14 +97,69 @@ __global__ void build_factors_kernel(const __nv_bfloat16* __restrict__ ls_down,
                                      __nv_bfloat16* __restrict__ dntcat, const PrologueExtras x) {
     pdl_trigger();
     pdl_wait();
+    // With the tensor-max job the CTAs split the work: the first kFactorCtas build the
+    // factors (and run the side jobs), the others stream the input for its max, so the two
+    // latency-bound halves overlap instead of running one after the other in each thread.
+    const bool max_job = x.max_src != nullptr;
+    const int fctas = max_job ? kFactorCtas : static_cast<int>(gridDim.x);
+    if (max_job && static_cast<int>(blockIdx.x) >= fctas) {
+        // max |x| of the call's input, one partial per CTA; a dense matrix (row stride ==
+        // columns, as the layer calls pass it) is one flat run of 16-byte vectors
+        const int64_t vpr = x.max_cols / 8;
+        const int64_t nvec = x.max_rows * vpr;
+        const int64_t gstride = static_cast<int64_t>(gridDim.x - fctas) * blockDim.x;
+        float m = 0.0f;
+        auto vmax = [&](const uint4& u) {
+            const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+                m = fmaxf(m, fmaxf(fabsf(bf16lo_to_f32(w[e])), fabsf(bf16hi_to_f32(w[e]))));
+        };
+        const bool flat = x.max_ld == x.max_cols;
+        const uint4* flat_src = reinterpret_cast<const uint4*>(x.max_src);
+        auto at = [&](int64_t iv) {
+            return flat ? flat_src[iv]
+                        : *reinterpret_cast<const uint4*>(x.max_src + (iv / vpr) * x.max_ld + (iv % vpr) * 8);
+        };
+        int64_t i = static_cast<int64_t>(blockIdx.x - fctas) * blockDim.x + threadIdx.x;
+        for (; i + 7 * gstride < nvec; i += 8 * gstride) {  // eight independent loads in flight
+            uint4 v[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) v[u] = at(i + u * gstride);
+#pragma unroll
+            for (int u = 0; u < 8; ++u) vmax(v[u]);
+        }
+        for (; i < nvec; i += gstride) vmax(at(i));
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        __shared__ float red[8];
+        if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            float v = 0.0f;
+            for (int w = 0; w < static_cast<int>(blockDim.x >> 5); ++w) v = fmaxf(v, red[w]);
+            x.max_parts[blockIdx.x] = v;
+        }
+        return;
+    }
+    if (max_job && threadIdx.x == 0) x.max_parts[blockIdx.x] = 0.0f;  // a factor CTA's partial
+
     const int R = r_s + r;
-    const __nv_bfloat16 zero = __float2bfloat16_rn(0.0f);
-    const int stride = gridDim.x * blockDim.x;
+    const int stride = fctas * blockDim.x;
     const int t0 = blockIdx.x * blockDim.x + threadIdx.x;
     auto dn_at = [&](int j, int k) { return j < r_s ? ls_down[j * K + k] : lora_a[(j - r_s) * K + k]; };
     auto up_at = [&](int n, int j) { return j < r_s ? ls_up[n * r_s + j] : lora_b[n * r + (j - r_s)]; };
-    // Row-wise pieces move 8 elements (16 bytes) per thread; the 8-element chunks never
-    // straddle two sources because r_s, r and K are multiples of 8 (checked by the host).
+    auto pack8 = [](const __nv_bfloat16 (&e)[8]) {
+        uint4 v;
+        v.x = static_cast<uint32_t>(__bfloat16_as_ushort(e[0])) | (static_cast<uint32_t>(__bfloat16_as_ushort(e[1])) << 16);
+        v.y = static_cast<uint32_t>(__bfloat16_as_ushort(e[2])) | (static_cast<uint32_t>(__bfloat16_as_ushort(e[3])) << 16);
+        v.z = static_cast<uint32_t>(__bfloat16_as_ushort(e[4])) | (static_cast<uint32_t>(__bfloat16_as_ushort(e[5])) << 16);
+        v.w = static_cast<uint32_t>(__bfloat16_as_ushort(e[6])) | (static_cast<uint32_t>(__bfloat16_as_ushort(e[7])) << 16);
+        return v;
+    };
+    const __nv_bfloat16 zero = __float2bfloat16_rn(0.0f);
+    // Every piece moves 8 elements (16 bytes) per thread and step: r_s, r, K, N and the
+    // padded widths are multiples of 8, so a chunk never straddles two sources.
     if (dn) {
         const int kc = K / 8;
         for (int i = t0; i < Rp * kc; i += stride) {
@@ -104,75 +184,58 @@ __global__ void build_factors_kernel(const __nv_bfloat16* __restrict__ ls_down,
             *reinterpret_cast<uint4*>(upcat + n * KL + (i % cc) * 8) = v;
         }
     }
-    // Transposed pieces: one element per thread, consecutive threads along the
-    // destination row (the sources are small and stay in L2).
-    if (upt)
-        for (int i = t0; i < Rp * N; i += stride) {
-            const int j = i / N, n = i % N;
-            upt[i] = j < R ? up_at(n, j) : zero;
+    // Transposed pieces: 8 consecutive destination elements per thread (eight gathered
+    // source elements, one 16-byte store); the sources are small and stay in L2.
+    if (upt) {  // [Rp, N] = [Up^T; 0]
+        const int nc = N / 8;
+        for (int i = t0; i < Rp * nc; i += stride) {
+            const int j = i / nc, n = (i % nc) * 8;
+            __nv_bfloat16 e[8];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) e[q] = j < R ? up_at(n + q, j) : zero;
+            *reinterpret_cast<uint4*>(upt + j * N + n) = pack8(e);
         }
-    if (dntcat)
-        for (int i = t0; i < K * KL; i += stride) {
-            const int k = i / KL, c = i % KL;
-            dntcat[i] = c < R ? dn_at(c, k) : (c < 2 * R ? dn_at(c - R, k) : zero);
+    }
+    if (dntcat) {  // [K, KL] = [Dn^T, Dn^T, 0]
+        const int cc = KL / 8;
+        for (int i = t0; i < K * cc; i += stride) {
+            const int k = i / cc, c = (i % cc) * 8;
+            __nv_bfloat16 e[8];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                const int cq = c + q;
+                e[q] = cq < R ? dn_at(cq, k) : (cq < 2 * R ? dn_at(cq - R, k) : zero);
+            }
+            *reinterpret_cast<uint4*>(dntcat + k * KL + c) = pack8(e);
         }
-    // side jobs: V' = [hi(V), lo(V), 0] for dB, and the cleared tensor-max slot
+    }
+    // side jobs: V' = [hi(V), lo(V), 0] for dB (8 columns per thread: one group of hi, of
+    // lo, or of zeros, since r is a multiple of 8), and the cleared tensor-max slots
     if (x.hilo_dst) {
         const int w = x.hilo_NBW, rr = x.hilo_r;
-        for (int i = t0; i < x.hilo_M * w; i += stride) {
-            const int m = i / w, c = i - m * w;
-            __nv_bfloat16 o = zero;
+        const int wc = w / 8;
+        for (int i = t0; i < x.hilo_M * wc; i += stride) {
+            const int m = i / wc, c = (i - m * wc) * 8;
+            uint4 o = make_uint4(0, 0, 0, 0);
             if (c < 2 * rr) {
-                const float v = x.hilo_src[m * x.hilo_ld + x.hilo_c0 + (c < rr ? c : c - rr)];
-                const __nv_bfloat16 hi = __float2bfloat16_rn(v);
-                o = c < rr ? hi : __float2bfloat16_rn(v - __bfloat162float(hi));
+                const int cs = c < rr ? c : c - rr;
+                const float* src = x.hilo_src + static_cast<int64_t>(m) * x.hilo_ld + x.hilo_c0 + cs;
+                const float4 a = *reinterpret_cast<const float4*>(src);
+                const float4 b = *reinterpret_cast<const float4*>(src + 4);
+                const float v[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+                __nv_bfloat16 e[8];
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                    const __nv_bfloat16 hi = __float2bfloat16_rn(v[q]);
+                    e[q] = c < rr ? hi : __float2bfloat16_rn(v[q] - __bfloat162float(hi));
+                }
+                o = pack8(e);
             }
-            x.hilo_dst[i] = o;
+            *reinterpret_cast<uint4*>(x.hilo_dst + static_cast<int64_t>(m) * w + c) = o;
         }
     }
     if (x.zero_slot && t0 == 0) *x.zero_slot = 0.0f;
     if (x.zero_slot2 && t0 == 0) *x.zero_slot2 = 0.0f;
-    // side job: max |x| of the call's input (the bulk of this launch when present), one
-    // partial per CTA; eight independent 16-byte loads in flight per thread per trip
-    if (x.max_src) {
-        const int64_t vpr = x.max_cols / 8;
-        const int64_t nvec = x.max_rows * vpr;
-        const int64_t gstride = static_cast<int64_t>(stride);
-        float m = 0.0f;
-        auto vmax = [&](const uint4& u) {
-            const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-            for (int e = 0; e < 4; ++e)
-                m = fmaxf(m, fmaxf(fabsf(bf16lo_to_f32(w[e])), fabsf(bf16hi_to_f32(w[e]))));
-        };
-        // a dense matrix (row stride == columns, as the layer calls pass it) is one flat run
-        // of 16-byte vectors: no index division per load
-        const bool flat = x.max_ld == x.max_cols;
-        const uint4* flat_src = reinterpret_cast<const uint4*>(x.max_src);
-        auto at = [&](int64_t iv) {
-            return flat ? flat_src[iv]
-                        : *reinterpret_cast<const uint4*>(x.max_src + (iv / vpr) * x.max_ld + (iv % vpr) * 8);
-        };
-        int64_t i = t0;
-        for (; i + 7 * gstride < nvec; i += 8 * gstride) {  // eight independent loads in flight
-            uint4 v[8];
-#pragma unroll
-            for (int u = 0; u < 8; ++u) v[u] = at(i + u * gstride);
-#pragma unroll
-            for (int u = 0; u < 8; ++u) vmax(v[u]);
-        }
-        for (; i < nvec; i += gstride) vmax(at(i));
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-        __shared__ float red[8];
-        if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
-        __syncthreads();
-        if (threadIdx.x == 0) {
-            float v = 0.0f;
-            for (int w = 0; w < static_cast<int>(blockDim.x >> 5); ++w) v = fmaxf(v, red[w]);
-            x.max_parts[blockIdx.x] = v;
-        }
-    }
 }
 
 }  // namespace
@@ -187,7 +250,7 @@ static int grid_cap(int64_t work, int threads, int cap) {
 cudaError_t launch_lowrank_finalize(const LowRankFinalizeArgs& a, cudaStream_t stream) {
     before_launch(K_LOWRANK, stream);
     const cudaError_t le = launch_k(lowrank_finalize_kernel,
-                                    dim3(grid_cap(a.rows * a.R, 256, 148 * 8)), dim3(256), 0,
+                                    dim3(grid_cap(a.rows * (a.R / 4), 256, 148 * 8)), dim3(256), 0,
                                     stream, a);
     if (le != cudaSuccess) return le;
     after_launch(K_LOWRANK, stream);

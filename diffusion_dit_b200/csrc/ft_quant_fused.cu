@@ -64,7 +64,8 @@ __host__ __device__ inline Layout layout_for(int Rp) {
     // stage count is a multiple of both): each then waits on a stage's phases one after
     // another, so a parity wait cannot be satisfied by the phase before the one it wants.
     constexpr int unit = (NSETS % MW == 0) ? NSETS : (MW % NSETS == 0 ? MW : NSETS * MW);
-    int s = (200 * 1024) / L.stage_bytes;
+    // as many stages as the 227 KB of dynamic shared memory hold next to the barrier area
+    int s = (232448 - BAR_BYTES - 1024) / L.stage_bytes;
     if (s > MAX_STAGES) s = MAX_STAGES;
     s -= s % unit;
     if (s < unit) s = unit;

@@ -150,6 +150,20 @@ def test_repeated_calls_are_deterministic():
     assert torch.equal(da1, da2) and torch.equal(db1, db2)
 
 
+def _bwd_launches(spec, seed=0):
+    """Kernels one backward call launches (7 with dA's and dB's split sums in a launch of
+    their own, 6 when the dX GEMM's epilogue warps run them)."""
+    ft = _ft()
+    inp, _, w = _setup(spec, seed)
+    ws = ft.Workspace(w, spec.M, "cuda")
+    x = inp.x.cuda()
+    _, t = ft.linear_fwd(w, x, ws)
+    c0 = ft.launch_count()
+    ft.linear_bwd(w, x, t, inp.dy.cuda(), ws)
+    torch.cuda.synchronize()
+    return ft.launch_count() - c0
+
+
 # r = 32 with K = 2048: dA's and dB's split sums are too much work for the dX GEMM's
 # epilogue warps before its first tile (N = 512: two k steps), so they run in a launch of
 # their own; the gradients must meet the same bar.
@@ -159,7 +173,20 @@ WIDE_R = wl.LayerSpec(name="wide_r_256x2048x512", M=256, K=2048, N=512, r_s=16, 
 
 
 def test_backward_with_separate_split_sums_matches_oracle():
+    assert _bwd_launches(WIDE_R) == 7
     test_backward_matches_oracle(WIDE_R, 0)
+
+
+# N = 4096 (16 k steps in the dX GEMM's first tile) with r = 8: the split sums fit on the
+# pair GEMM's epilogue warps before their first accumulator
+SIDE_PAIR = wl.LayerSpec(name="side_pair_256x512x4096", M=256, K=512, N=4096, r_s=16, r=8, alpha=8.0,
+                         n_outlier_cols=3, outlier_gain=20.0, w_std=0.02, plant_rank=4, plant_sigma=6.0,
+                         b_std=0.01, dy_std=1e-2)
+
+
+def test_backward_pair_gemm_with_side_split_sums_matches_oracle():
+    assert _bwd_launches(SIDE_PAIR) == 6
+    test_backward_matches_oracle(SIDE_PAIR, 0)
 
 
 def test_given_max_equal_to_the_true_max_gives_the_same_forward():
@@ -179,13 +206,14 @@ def test_given_max_equal_to_the_true_max_gives_the_same_forward():
 
 
 # M = 384 (one-CTA GEMM kernel) with split sums small enough for its epilogue warps
-# ((N + K) r = 12288 outputs; N = 1024: four k steps in the dX GEMM's first tile)
-SIDE_ONE_CTA = wl.LayerSpec(name="side_one_cta_384x512x1024", M=384, K=512, N=1024, r_s=16, r=8, alpha=8.0,
+# ((N + K) r = 36864 outputs; N = 4096: sixteen k steps in the dX GEMM's first tile)
+SIDE_ONE_CTA = wl.LayerSpec(name="side_one_cta_384x512x4096", M=384, K=512, N=4096, r_s=16, r=8, alpha=8.0,
                             n_outlier_cols=3, outlier_gain=20.0, w_std=0.02, plant_rank=4, plant_sigma=6.0,
                             b_std=0.01, dy_std=1e-2)
 
 
 def test_backward_one_cta_gemm_with_side_split_sums_matches_oracle():
+    assert _bwd_launches(SIDE_ONE_CTA) == 6
     test_backward_matches_oracle(SIDE_ONE_CTA, 0)
 
 
