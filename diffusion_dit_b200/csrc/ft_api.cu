@@ -673,18 +673,21 @@ ft_status linear_bwd_impl(const ft_linear* L, const void* x_dev, const float* t_
         CUtensorMap tP, tV;
         FT_TRY(make_tmap(&tV, W + w.vcat, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, NBW, M, NBW * 2, 64, 64));
         FT_TRY(make_tmap(&tP, dy_dev, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, N, M, N * 2, 64, 64));
-        const int ctas = ft::lora_grad_ctas(M, N, dev.num_sms);
+        const ft::LoraSchedule sc = ft::lora_grad_schedule(M, N, dev.num_sms);
         g.F = N;
         g.chunks = static_cast<int>(M / 64);
+        g.full_tiles = sc.full_tiles;
+        g.rem_tiles = sc.rem_tiles;
+        g.rem_splits = sc.rem_splits;
         g.partial = reinterpret_cast<float*>(W + w.gpartial_b);
         if (!amax_or_null) {
             g.amax_out = reinterpret_cast<unsigned*>(scal + SC_AMAX_G);
             amax_g = scal + SC_AMAX_G;
         }
-        FT_CUDA(ft::launch_lora_grad(tP, tV, g, ctas, ft::K_LORA_DB, st));
+        FT_CUDA(ft::launch_lora_grad(tP, tV, g, ft::K_LORA_DB, st));
         g.amax_out = nullptr;
-        fin[1] = ft::LoraFinalizeJob{g.partial, ctas, g.chunks, static_cast<int>(N), NBW, L->r, L->lora_scale, false,
-                                     db_dev};
+        fin[1] = ft::LoraFinalizeJob{g.partial, sc.full_tiles, sc.rem_tiles, sc.rem_splits, static_cast<int>(N), NBW,
+                                     L->r, L->lora_scale, false, db_dev};
     }
     int splits = 1;
     const bool g_grid = pair_gemm(M, dev);  // the pair GEMM reads Q(G)'s compact block grid
@@ -716,25 +719,27 @@ ft_status linear_bwd_impl(const ft_linear* L, const void* x_dev, const float* t_
         CUtensorMap tP, tV;
         FT_TRY(make_tmap(&tV, W + w.ucat_lora, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, NBW, M, NBW * 2, 64, 64));
         FT_TRY(make_tmap(&tP, x_dev, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, K, M, K * 2, 64, 64));
-        const int ctas = ft::lora_grad_ctas(M, K, dev.num_sms);
+        const ft::LoraSchedule sc = ft::lora_grad_schedule(M, K, dev.num_sms);
         g.F = K;
         g.chunks = static_cast<int>(M / 64);
+        g.full_tiles = sc.full_tiles;
+        g.rem_tiles = sc.rem_tiles;
+        g.rem_splits = sc.rem_splits;
         g.partial = reinterpret_cast<float*>(W + w.gpartial_a);
-        FT_CUDA(ft::launch_lora_grad(tP, tV, g, ctas, ft::K_LORA_DA, st));
-        fin[0] = ft::LoraFinalizeJob{g.partial, ctas, g.chunks, static_cast<int>(K), NBW, L->r, L->lora_scale, true,
-                                     da_dev};
+        FT_CUDA(ft::launch_lora_grad(tP, tV, g, ft::K_LORA_DA, st));
+        fin[0] = ft::LoraFinalizeJob{g.partial, sc.full_tiles, sc.rem_tiles, sc.rem_splits, static_cast<int>(K), NBW,
+                                     L->r, L->lora_scale, true, da_dev};
     }
     // dA's and dB's split sums: on the dX GEMM's epilogue warps when they fit in about half
     // the time those warps wait for their first accumulator (a k step of 256 takes ~0.42 us;
-    // a thread's block of 4 x 4 outputs costs ~0.3 us per slot it adds, the slots' loads
-    // overlapping), else in a launch of their own before the GEMM.
+    // a thread's block of 4 x 4 outputs costs ~0.6 us per slot it adds: one round trip for
+    // the slot's eight loads), else in a launch of their own before the GEMM.
     bool side = false;
     if (L->r > 0) {
         const double blocks = static_cast<double>(N + K) * L->r / 16.0;
         const double workers = static_cast<double>(dev.num_sms) * (pair_gemm(M, dev) ? 256.0 : 128.0);
-        const double slots = std::max(static_cast<double>(fin[0].ctas) / (K / 128),
-                                      static_cast<double>(fin[1].ctas) / (N / 128)) + 1.0;
-        const double cost_us = std::ceil(blocks / workers) * slots * 0.3;
+        const double slots = std::max(fin[0].rem_tiles ? fin[0].rem_splits : 1, fin[1].rem_tiles ? fin[1].rem_splits : 1);
+        const double cost_us = std::ceil(blocks / workers) * slots * 0.6;
         const double first_tile_us = (static_cast<double>(N) / 256.0 + (KL + 63) / 64) * 0.42;
         side = cost_us <= 0.5 * first_tile_us;
         if (!side) FT_CUDA(ft::launch_lora_grad_finalize(fin[0], fin[1], st));

@@ -23,9 +23,14 @@
 // TMEM_EMPTY.  No load is multicast.  Tiles are visited with the smaller operand swept by
 // the tiles in flight (p.n_inner), so that it stays in L2.
 //
+// Five stages and four epilogue warps (eight for the GELU epilogues): a sixth stage (room
+// for it once the scales are compact, with the scale-factor slots in tensor memory then
+// reused five k steps apart) and eight plain epilogue warps each measured slower on the
+// FLUX single-stream layers.
+//
 // Warp roles: warp 0 = TMA producer, warp 1 = MMA issuer (even CTA) and TMEM owner, then
-// the epilogue warps (Cfg: 8, two per TMEM lane quarter, 128 columns each; 4 in the
-// transposing plain variant), then 4 scale writers.
+// the epilogue warps (4, or 8 for the GELU epilogues: two per TMEM lane quarter, 128
+// columns each), then 4 scale writers.
 //
 // With XP (the dX GEMM of section 3.2 without a stored Q(R)^T) the producer loads B's
 // untransposed slab, 256 reduction rows x 64 bytes, into the B slot, and the scale
@@ -43,64 +48,50 @@ constexpr int BM = 128;                  // rows per CTA (256 per pair)
 constexpr int BN = 256;                  // output columns per pair
 constexpr int BN_CTA = 128;              // B rows held by one CTA
 constexpr int BK_BYTES = 128;
+constexpr int STAGES = 5;
 constexpr int A_BYTES = BM * BK_BYTES;      // 16 KB
 constexpr int B_BYTES = BN_CTA * BK_BYTES;  // 16 KB
-constexpr int SFA_BYTES = 4 * 512;          // a k step's scale atoms (tensor-core layout) of 128 A rows
-constexpr int SFB_BYTES = 2 * 4 * 512;      // ... of the pair tile's 256 B rows
-// the compact grids of 16x16-block scales one k step needs
+constexpr int SFA_BYTES = 4 * 512;
+constexpr int SFB_BYTES = 2 * 4 * 512;
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;  // 38912
+// the compact grids of 16x16-block scales one k step needs (they fit in the atoms' regions)
 constexpr int SFA_GRID_BYTES = 8 * 16;   // 8 block-rows x 16 block-columns
 constexpr int SFB_GRID_BYTES = 16 * 16;  // the pair tile's 16 block-rows
 constexpr int OFF_B = A_BYTES;
 constexpr int OFF_SFA = A_BYTES + B_BYTES;
+constexpr int OFF_SFB = OFF_SFA + SFA_BYTES;
 constexpr int EPI_BYTES = 32 * 64;
+constexpr int OFF_EPI = STAGES * STAGE_BYTES;
 constexpr int BAR_BYTES = 256;
-constexpr int SMEM_LIMIT = 232448;       // 227 KB of dynamic shared memory
+constexpr int EPI_BUFS = 2;              // staging buffers per epilogue warp (one store in flight)
+// Epilogue warps per variant: 4 (one per TMEM lane quarter, all 256 columns) for the plain
+// GEMM; 8 (two per quarter, 128 columns each) for the GELU epilogues, whose arithmetic
+// needs two warps per scheduler to hide its latency.
+__host__ __device__ constexpr int epi_warps(int epi) { return epi == kEpiPlain ? 4 : 8; }
+__host__ __device__ constexpr int epi_region(int epi) { return epi_warps(epi) * EPI_BUFS * EPI_BYTES; }
+__host__ __device__ constexpr int smem_bytes(int epi) { return OFF_EPI + epi_region(epi) + BAR_BYTES + 1024; }
+__host__ __device__ constexpr int threads(int epi) { return 32 * (2 + epi_warps(epi) + 4); }
+
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t COL_ACC = 0;
+constexpr uint32_t COL_SFA = 256;                    // STAGES x 16 columns
+constexpr uint32_t COL_SFB = COL_SFA + STAGES * 16;  // STAGES x 32 columns
 
-__host__ __device__ constexpr int align1k(int v) { return (v + 1023) / 1024 * 1024; }
+static_assert(STAGE_BYTES % 1024 == 0, "stage must keep 1024-byte alignment");
+static_assert(smem_bytes(kEpiGelu) <= 232448, "exceeds 227 KB of dynamic shared memory");
+static_assert(COL_SFB + STAGES * 32 <= TMEM_COLS, "tensor memory overflow");
 
-// Layout of one instantiation.  A stage holds A's and B's codes and the k step's scales
-// (compact grids or tensor-core atoms, by SFC); as many stages as fit next to the
-// epilogue's staging buffers, up to six.  The scale factors live in tensor memory in NSF
-// slots (at most five fit beside the 256-column accumulator), reused round-robin by k
-// step: with six stages a slot is rewritten only once the MMAs that read it five steps
-// earlier have completed.  Epilogue warps: eight (two per TMEM lane quarter, 128 columns
-// each: the accumulator drains twice as fast, and the GELU arithmetic needs two warps
-// per scheduler), except the transposing plain variant, whose scale warps need the
-// registers; the plain epilogue has one staging buffer per warp, the GELU ones two.
-template <int EPI, bool XP, int SFC>
-struct Cfg {
-    static constexpr bool kGridA = (SFC & 1) != 0;
-    static constexpr bool kGridB = (SFC & 2) != 0;
-    static constexpr int SFA_SLOT = kGridA ? SFA_GRID_BYTES : SFA_BYTES;
-    static constexpr int SFB_SLOT = kGridB ? SFB_GRID_BYTES : SFB_BYTES;
-    static constexpr int OFF_SFB = OFF_SFA + SFA_SLOT;
-    static constexpr int STAGE_BYTES = align1k(A_BYTES + B_BYTES + SFA_SLOT + SFB_SLOT);
-    static constexpr int EPI_WARPS = (EPI == kEpiPlain && XP) ? 4 : 8;
-    static constexpr int EPI_BUFS = (EPI == kEpiPlain && !XP) ? 1 : 2;
-    static constexpr int EPI_REGION = EPI_WARPS * EPI_BUFS * EPI_BYTES;
-    static constexpr int STAGES_FIT = (SMEM_LIMIT - EPI_REGION - BAR_BYTES - 1024) / STAGE_BYTES;
-    static constexpr int STAGES = STAGES_FIT > 6 ? 6 : STAGES_FIT;
-    static constexpr int NSF = STAGES < 5 ? STAGES : 5;
-    static constexpr int OFF_EPI = STAGES * STAGE_BYTES;
-    static constexpr int SMEM = OFF_EPI + EPI_REGION + BAR_BYTES + 1024;
-    static constexpr int THREADS = 32 * (2 + EPI_WARPS + 4);
-    static constexpr uint32_t COL_SFA = 256;                  // NSF x 16 columns
-    static constexpr uint32_t COL_SFB = COL_SFA + NSF * 16;   // NSF x 32 columns
-    static constexpr int BAR_FULL0 = 0, BAR_EMPTY0 = STAGES, BAR_SF_READY0 = 2 * STAGES;
-    static constexpr int BAR_TMEM_FULL = 3 * STAGES;
-    static constexpr int BAR_TMEM_EMPTY = 3 * STAGES + 1;
-    static constexpr int BAR_FINAL = 3 * STAGES + 2;
-    static constexpr int BAR_XREAD = 3 * STAGES + 3;  // XP: the scale warps have read the raw B slab
-    static constexpr int NUM_BARS = 3 * STAGES + 4;
-    static constexpr int OFF_TMEM_SLOT = 8 * NUM_BARS;
-    static constexpr int OFF_ABORT = OFF_TMEM_SLOT + 4;
-    static_assert(STAGES >= 4, "too few stages");
-    static_assert(SMEM <= SMEM_LIMIT, "exceeds 227 KB of dynamic shared memory");
-    static_assert(COL_SFB + NSF * 32 <= TMEM_COLS, "tensor memory overflow");
-    static_assert(OFF_ABORT + 4 <= BAR_BYTES, "barrier area overflow");
-};
+__host__ __device__ constexpr int BAR_FULL(int s) { return s; }
+__host__ __device__ constexpr int BAR_EMPTY(int s) { return STAGES + s; }
+__host__ __device__ constexpr int BAR_SF_READY(int s) { return 2 * STAGES + s; }
+constexpr int BAR_TMEM_FULL = 3 * STAGES;
+constexpr int BAR_TMEM_EMPTY = 3 * STAGES + 1;
+constexpr int BAR_FINAL = 3 * STAGES + 2;
+constexpr int BAR_XREAD = 3 * STAGES + 3;  // XP: the scale warps have read the raw B slab
+constexpr int NUM_BARS = 3 * STAGES + 4;
+constexpr int OFF_TMEM_SLOT = 8 * NUM_BARS;
+constexpr int OFF_ABORT = OFF_TMEM_SLOT + 4;
+static_assert(OFF_ABORT + 4 <= BAR_BYTES, "barrier area overflow");
 
 // XP: one scale warp's share of the in-place transposition of the B slab at `slab`.
 // False if the wait for the other scale warps' reads gave up (the abort flag and status
@@ -126,7 +117,7 @@ __device__ __forceinline__ bool xpose_share(uint32_t slab, int q, int lane, uint
 // SFC bit 0: A's scales come from its compact 16x16-block grid (tmSA), bit 1: B's (tmSB);
 // otherwise from the tensor-core scale layout (p.sfa / p.sfb).
 template <int EPI, bool XP, int SFC>
-__global__ void __launch_bounds__(Cfg<EPI, XP, SFC>::THREADS, 1)
+__global__ void __launch_bounds__(threads(EPI), 1)
     gemm_fp4_lowrank_pair_kernel(const __grid_constant__ CUtensorMap tmA,
                                  const __grid_constant__ CUtensorMap tmB,
                                  const __grid_constant__ CUtensorMap tmLA,
@@ -135,35 +126,23 @@ __global__ void __launch_bounds__(Cfg<EPI, XP, SFC>::THREADS, 1)
                                  const __grid_constant__ CUtensorMap tmAct,
                                  const __grid_constant__ CUtensorMap tmSA,
                                  const __grid_constant__ CUtensorMap tmSB, const GemmFp4Args p) {
-    using C = Cfg<EPI, XP, SFC>;
-    constexpr bool kGridA = C::kGridA;
-    constexpr bool kGridB = C::kGridB;
-    constexpr int STAGES = C::STAGES;
-    constexpr int STAGE_BYTES = C::STAGE_BYTES;
-    constexpr int NSF = C::NSF;
-    constexpr int OFF_SFB = C::OFF_SFB;
+    constexpr bool kGridA = (SFC & 1) != 0;
+    constexpr bool kGridB = (SFC & 2) != 0;
     // bytes one k step's scales add to a stage: a 128-row band's grid rows (8 x 16 B) or its
     // four 512-byte atoms; the pair tile's 256 B rows: 16 x 16 B or eight atoms
-    constexpr uint32_t kSfBytes = C::SFA_SLOT + C::SFB_SLOT;
-    auto BAR_FULL = [](int s) { return C::BAR_FULL0 + s; };
-    auto BAR_EMPTY = [](int s) { return C::BAR_EMPTY0 + s; };
-    auto BAR_SF_READY = [](int s) { return C::BAR_SF_READY0 + s; };
-    constexpr int BAR_TMEM_FULL = C::BAR_TMEM_FULL, BAR_TMEM_EMPTY = C::BAR_TMEM_EMPTY;
-    constexpr int BAR_FINAL = C::BAR_FINAL, BAR_XREAD = C::BAR_XREAD;
+    constexpr uint32_t kSfBytes = (kGridA ? SFA_GRID_BYTES : SFA_BYTES) + (kGridB ? SFB_GRID_BYTES : SFB_BYTES);
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_u32 = smem_u32(smem_raw);
     const uint32_t pad = (1024 - (raw_u32 & 1023)) & 1023;
     uint8_t* base = smem_raw + pad;
     const uint32_t base_u32 = raw_u32 + pad;
-    constexpr int EPI_WARPS = C::EPI_WARPS;
-    constexpr int EPI_BUFS = C::EPI_BUFS;
+    constexpr int EPI_WARPS = epi_warps(EPI);
     constexpr int EPI_COLS = BN / (EPI_WARPS / 4);  // tile columns per epilogue warp
-    constexpr int OFF_EPI = C::OFF_EPI;
-    uint8_t* bar_area = base + OFF_EPI + C::EPI_REGION;
-    auto bar = [&](int i) { return base_u32 + OFF_EPI + C::EPI_REGION + 8 * i; };
+    uint8_t* bar_area = base + OFF_EPI + epi_region(EPI);
+    auto bar = [&](int i) { return base_u32 + OFF_EPI + epi_region(EPI) + 8 * i; };
     auto stage = [&](int s) { return base_u32 + s * STAGE_BYTES; };
-    volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(bar_area + C::OFF_TMEM_SLOT);
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(bar_area + C::OFF_ABORT);
+    volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(bar_area + OFF_TMEM_SLOT);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(bar_area + OFF_ABORT);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -281,7 +260,6 @@ __global__ void __launch_bounds__(Cfg<EPI, XP, SFC>::THREADS, 1)
             int ti = 0;
             int s = 0;        // stage of the next k step
             uint32_t ph = 0;  // its use parity
-            int sf = 0;       // its scale-factor slot in tensor memory (k steps round-robin over NSF)
             for (int t = pair; t < num_tiles && !*abort_flag; t += num_pairs, ++ti) {
                 if (!mbar_wait(bar(BAR_TMEM_EMPTY), (ti & 1) ^ 1, abort_flag, p.status)) break;
                 tc_fence_after();
@@ -299,8 +277,8 @@ __global__ void __launch_bounds__(Cfg<EPI, XP, SFC>::THREADS, 1)
                     const uint64_t ad = sdesc_kmajor_sw128(st);
                     const uint64_t bd = sdesc_kmajor_sw128(st + OFF_B);
                     if (j < KT) {
-                        const uint32_t sfa_t = tmem + C::COL_SFA + 16 * sf;
-                        const uint32_t sfb_t = tmem + C::COL_SFB + 32 * sf;
+                        const uint32_t sfa_t = tmem + COL_SFA + 16 * s;
+                        const uint32_t sfb_t = tmem + COL_SFB + 32 * s;
 #pragma unroll
                         for (int i = 0; i < 4; ++i)
                             mma_fp4_block16_pair(tmem + COL_ACC, ad + 2 * i, bd + 2 * i, idesc4, sfa_t + 4 * i,
@@ -315,7 +293,6 @@ __global__ void __launch_bounds__(Cfg<EPI, XP, SFC>::THREADS, 1)
                         s = 0;
                         ph ^= 1;
                     }
-                    if (++sf == NSF) sf = 0;
                 }
                 if (!ok) break;
                 tc_commit_pair_both(bar(BAR_TMEM_FULL));
@@ -338,20 +315,8 @@ __global__ void __launch_bounds__(Cfg<EPI, XP, SFC>::THREADS, 1)
             for (int j = 0; j < KT + KLS; ++j, ++it) {
                 const int s = it % STAGES;
                 const uint32_t ph = (it / STAGES) & 1;
-                const int sf = it % NSF;
                 if (!mbar_wait(bar(BAR_FULL(s)), ph, abort_flag, p.status)) { ok = false; break; }
                 if (j < KT) {
-                    if constexpr (NSF < STAGES) {
-                        // the slot was last read by k step it - NSF: wait until its MMAs have
-                        // completed (that step's release of its stage)
-                        if (it >= NSF) {
-                            const int o = it - NSF;
-                            if (!mbar_wait(bar(BAR_EMPTY(o % STAGES)), (o / STAGES) & 1, abort_flag, p.status)) {
-                                ok = false;
-                                break;
-                            }
-                        }
-                    }
                     const uint8_t* st = base + s * STAGE_BYTES;
                     // va[4 i + w]: word w (rows lane + 32 w) of A's atom i (k-blocks 4i..4i+3);
                     // vb0 / vb1: B's atoms 0-1 / 2-3, each as [rows 0-127: 4 words, rows 128-255: 4]
@@ -396,9 +361,9 @@ __global__ void __launch_bounds__(Cfg<EPI, XP, SFC>::THREADS, 1)
                             vb[o + 4] = b1.x; vb[o + 5] = b1.y; vb[o + 6] = b1.z; vb[o + 7] = b1.w;
                         }
                     }
-                    tmem_st_32x32b_x16(lane_base + C::COL_SFA + 16 * sf, va);
-                    tmem_st_32x32b_x16(lane_base + C::COL_SFB + 32 * sf, vb0);
-                    tmem_st_32x32b_x16(lane_base + C::COL_SFB + 32 * sf + 16, vb1);
+                    tmem_st_32x32b_x16(lane_base + COL_SFA + 16 * s, va);
+                    tmem_st_32x32b_x16(lane_base + COL_SFB + 32 * s, vb0);
+                    tmem_st_32x32b_x16(lane_base + COL_SFB + 32 * s + 16, vb1);
                     if constexpr (XP) {
                         if (!xpose_share(stage(s) + OFF_B, q, lane, bar(BAR_XREAD), xr, abort_flag, p.status)) {
                             tmem_st_wait();
@@ -467,15 +432,10 @@ __global__ void __launch_bounds__(Cfg<EPI, XP, SFC>::THREADS, 1)
             }
 #pragma unroll
             for (int ch = 0; ch < EPI_COLS / 32; ++ch) {
-                uint32_t stage_u32 = stage0_u32 + (sc % EPI_BUFS) * EPI_BYTES;
-                uint8_t* stage_ptr = stage0_ptr + (sc % EPI_BUFS) * EPI_BYTES;
+                uint32_t stage_u32 = stage0_u32 + (sc & 1) * EPI_BYTES;
+                uint8_t* stage_ptr = stage0_ptr + (sc & 1) * EPI_BYTES;
                 ++sc;
-                if (lane == 0) {  // this buffer's last store has read it
-                    if constexpr (EPI_BUFS == 1)
-                        bulk_wait_group_read0();
-                    else
-                        bulk_wait_group_read1();
-                }
+                if (lane == 0) bulk_wait_group_read1();  // this buffer's last store has read it
                 __syncwarp();
                 if constexpr (EPI == kEpiGeluBwd) {
                     uint4 cur[4];
@@ -561,12 +521,11 @@ cudaError_t launch_variant(const CUtensorMap& tmA, const CUtensorMap& tmB, const
                            const CUtensorMap& tmSA, const CUtensorMap& tmSB, const GemmFp4Args& args,
                            cudaLaunchConfig_t cfg) {
     using namespace gemm2;
-    using C = Cfg<EPI, XP, SFC>;
     static const cudaError_t attr = cudaFuncSetAttribute(
-        gemm_fp4_lowrank_pair_kernel<EPI, XP, SFC>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+        gemm_fp4_lowrank_pair_kernel<EPI, XP, SFC>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes(EPI));
     if (attr != cudaSuccess) return attr;
-    cfg.blockDim = dim3(C::THREADS);
-    cfg.dynamicSmemBytes = C::SMEM;
+    cfg.blockDim = dim3(threads(EPI));
+    cfg.dynamicSmemBytes = smem_bytes(EPI);
     return cudaLaunchKernelEx(&cfg, gemm_fp4_lowrank_pair_kernel<EPI, XP, SFC>, tmA, tmB, tmLA, tmLB, tmOut, tmAct,
                               tmSA, tmSB, args);
 }

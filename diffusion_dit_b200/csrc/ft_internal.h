@@ -45,16 +45,19 @@ cudaError_t launch_k(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t sme
 // GEMM epilogue variants, one kernel instantiation each (the plain one carries no GELU code)
 enum EpilogueKind { kEpiPlain = 0, kEpiGelu = 1, kEpiGeluBwd = 2 };
 
-// One split sum of the adapter gradients (run by lora_split_sums in ft_sidejobs.cuh): the
-// adapter-gradient kernel ran `ctas` persistent CTAs over U = (F / 128) * chunks units
-// (128-feature tile t, 64-token chunk c; unit t * chunks + c), CTA p taking units
-// [p U / ctas, (p + 1) U / ctas) and leaving the sum over each tile it touched in partial
-// slot p + t, [128][NBW] fp32.  Then
-//   out = s * sum over the CTAs that touched the tile, in order, of (D[f][j] + D[f][r + j])
+// The adapter-gradient kernel's CTA schedule over T tiles of 128 features: CTA b <
+// full_tiles takes tile b over all tokens; CTA full_tiles + s * rem_tiles + i takes token
+// range s (of rem_splits) of tile full_tiles + i.  CTA b writes partial slot b.
+struct LoraSchedule {
+    int full_tiles, rem_tiles, rem_splits, ctas;
+};
+
+// One split sum of the adapter gradients (run by lora_split_sums in ft_sidejobs.cuh):
+//   out = s * sum over the tile's slots, in token order, of (D[f][j] + D[f][r + j])
 // stored as out[f][j], or out[j][f] with transpose_out.  out == nullptr: no job.
 struct LoraFinalizeJob {
-    const float* partial;    // [ctas + F / 128][128][NBW]
-    int ctas, chunks, F, NBW, r;
+    const float* partial;    // [slots][128][NBW]
+    int full_tiles, rem_tiles, rem_splits, F, NBW, r;
     float s;
     bool transpose_out;
     float* out;
@@ -208,16 +211,17 @@ cudaError_t launch_build_factors(const __nv_bfloat16* ls_down, const __nv_bfloat
 struct LoraGradArgs {
     int64_t F;               // features of P [M, F] (multiple of 128)
     int chunks;              // 64-token chunks of P (M / 64)
+    int full_tiles, rem_tiles, rem_splits;  // the CTA schedule (LoraSchedule)
     int NBW;                 // width of V' = [hi, lo, 0] (multiple of 64, <= 256)
-    uint32_t tmem_cols;      // per accumulator (two are allocated): power of two >= max(32, NBW)
-    float* partial;          // [ctas + F / 128][128][NBW] (see LoraFinalizeJob)
+    uint32_t tmem_cols;      // power of two >= max(32, NBW)
+    float* partial;          // [ctas][128][NBW], slot b = CTA b
     int* status;
     // optional: max |P| over every element of P (each is read by exactly one CTA),
     // accumulated with atomicMax on the float's bits into a slot cleared beforehand
     unsigned* amax_out;
 };
-int lora_grad_ctas(int64_t M, int64_t F, int num_sms);
-cudaError_t launch_lora_grad(const CUtensorMap& tmP, const CUtensorMap& tmV, const LoraGradArgs& a, int ctas,
-                             int kind, cudaStream_t stream);
+LoraSchedule lora_grad_schedule(int64_t M, int64_t F, int num_sms);
+cudaError_t launch_lora_grad(const CUtensorMap& tmP, const CUtensorMap& tmV, const LoraGradArgs& a, int kind,
+                             cudaStream_t stream);
 
 }  // namespace ft

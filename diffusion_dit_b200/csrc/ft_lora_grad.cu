@@ -11,20 +11,20 @@
 // up to 64) is MN-major too; the hi and lo halves land in separate accumulator
 // columns and are added in the final sum, keeping ~16 mantissa bits of V.
 //
-// Work is balanced over persistent CTAs (at most one per SM): the units (128-feature
-// tile t, 64-token chunk c) are numbered u = t C + c (C chunks per tile) and CTA p of P
-// takes the run [p U / P, (p + 1) U / P) of the U = T C units.  A run is cut into
-// segments where it crosses a tile boundary; each segment's sum over its tokens goes to
-// partial slot p + t (unique: a CTA's tiles t0..t1 give slots p + t0 .. p + t1, and the
-// next CTA starts at tile t1 or later), [128 features][NBW] fp32.  The accumulator is
-// double-buffered in tensor memory so that one segment drains while the next fills.
-// lora_split_sums (ft_sidejobs.cuh) adds, for each tile, the slots of the CTAs that
-// covered it, in token order (deterministic); the dX GEMM's epilogue warps run it while
-// they wait for their first accumulator, or a launch of its own does.
+// Schedule (lora_grad_schedule): one CTA per SM at a time, in lockstep over the tokens
+// -- the CTAs running together read the same 64-token rows of P, each its own 128
+// features, so every row of P streams from HBM whole.  Phase 1: q = T / P rounds of whole
+// tiles (T tiles of 128 features, P SMs), CTA b < qP taking tile b over all tokens.
+// Phase 2: the R = T - qP remaining tiles, each split over S2 = P / R token ranges (at
+// most 16), CTA qP + s R + i taking range s of tile qP + i, so that the CTAs of one range
+// run together.  CTA b leaves its sum in partial slot b, [128 features][NBW] fp32;
+// lora_split_sums (ft_sidejobs.cuh) adds a tile's slots in token order (deterministic).
+// The dX GEMM's epilogue warps run those sums while they wait for their first
+// accumulator, or a launch of its own does.
 //
-// When asked (amax_out), the four epilogue warps also take max |P| over every tile that
-// lands: with dB computed first in the backward pass this gives the tensor max of G for
-// Q(G) without a separate pass over G.
+// When asked (amax_out), the four epilogue warps, idle until the final drain, also take
+// max |P| over every tile that lands: with dB computed first in the backward pass this
+// gives the tensor max of G for Q(G) without a separate pass over G.
 #include "ft_internal.h"
 #include "ft_ptx.cuh"
 #include "ft_sidejobs.cuh"
@@ -66,20 +66,30 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int S = L.stages;
     uint8_t* bar_area = base + S * L.stage_bytes;
     auto bar = [&](int i) { return base_u32 + S * L.stage_bytes + 8 * i; };
-    // barriers: FULL [0, S), EMPTY [S, 2S), ACC_FULL 2S + b, ACC_EMPTY 2S + 2 + b (b = the
-    // accumulator buffer), FINAL 2S + 4
-    volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(bar_area + 8 * (2 * MAX_STAGES + 5));
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(bar_area + 8 * (2 * MAX_STAGES + 5) + 4);
-    const int ACC_FULL = 2 * S, ACC_EMPTY = 2 * S + 2, FINAL = 2 * S + 4;
+    volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(bar_area + 8 * (2 * MAX_STAGES + 2));
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(bar_area + 8 * (2 * MAX_STAGES + 2) + 4);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    // this CTA's run of units and the tile it starts in
-    const int64_t U = static_cast<int64_t>(p.F / BF) * p.chunks;
-    const int64_t u0 = static_cast<int64_t>(blockIdx.x) * U / gridDim.x;
-    const int64_t u1 = static_cast<int64_t>(blockIdx.x + 1) * U / gridDim.x;
-    const int nk = static_cast<int>(u1 - u0);
-    const int t_first = static_cast<int>(u0 / p.chunks);
+    // this CTA's tile and token range (see the schedule above)
+    int tile, c0, c1;
+    {
+        const int b = blockIdx.x;
+        if (b < p.full_tiles) {
+            tile = b;
+            c0 = 0;
+            c1 = p.chunks;
+        } else {
+            const int rr = b - p.full_tiles;
+            const int s = rr / p.rem_tiles;
+            tile = p.full_tiles + (rr - s * p.rem_tiles);
+            c0 = static_cast<int>(static_cast<int64_t>(s) * p.chunks / p.rem_splits);
+            c1 = static_cast<int>(static_cast<int64_t>(s + 1) * p.chunks / p.rem_splits);
+        }
+    }
+    const int f0 = tile * BF;
+    const int m0 = c0 * BMT;
+    const int nk = c1 - c0;
     const int nchunk = p.NBW / 64;
 
     if (threadIdx.x == 0) {
@@ -87,11 +97,8 @@ __global__ void __launch_bounds__(THREADS, 1)
             mbar_init(bar(i), 1);
             mbar_init(bar(S + i), 1 + (p.amax_out ? 4 : 0));  // MMA commit (+ 4 max warps)
         }
-        for (int b = 0; b < 2; ++b) {
-            mbar_init(bar(ACC_FULL + b), 1);   // the MMA issuer's commit after a segment's last unit
-            mbar_init(bar(ACC_EMPTY + b), 4);  // the four drain warps
-        }
-        mbar_init(bar(FINAL), 1);
+        mbar_init(bar(2 * S), 1);
+        mbar_init(bar(2 * S + 1), 1);
         *abort_flag = 0;
         fence_mbar_init();
         fence_proxy_async_smem();
@@ -101,7 +108,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         tma_prefetch_desc(&tmV);
     }
     if (warp == 1) {
-        tmem_alloc(smem_u32(const_cast<uint32_t*>(tmem_slot)), 2 * p.tmem_cols);  // two accumulators
+        tmem_alloc(smem_u32(const_cast<uint32_t*>(tmem_slot)), p.tmem_cols);
         tmem_relinquish();
     }
     tc_fence_before();
@@ -122,9 +129,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                 if (!mbar_wait(bar(S + s), ((k / S) & 1) ^ 1, abort_flag, p.status)) break;
                 const uint32_t st = base_u32 + s * L.stage_bytes;
                 mbar_arrive_expect_tx(bar(s), tx);
-                const int64_t u = u0 + k;
-                const int f0 = static_cast<int>(u / p.chunks) * BF;
-                const int mm = static_cast<int>(u % p.chunks) * BMT;
+                const int mm = m0 + k * BMT;
                 tma_load_2d(st, &tmP, bar(s), f0, mm);
                 tma_load_2d(st + A_BYTES / 2, &tmP, bar(s), f0 + 64, mm);
                 for (int c = 0; c < nchunk; ++c)
@@ -138,18 +143,8 @@ __global__ void __launch_bounds__(THREADS, 1)
     } else if (warp == 1) {
         if (lane == 0) {
             const uint32_t idesc = idesc_bf16(BF, p.NBW, /*a_mn=*/true, /*b_mn=*/true);
-            int seg = 0;  // segment of this CTA the next unit belongs to
             for (int k = 0; k < nk; ++k) {
                 const int s = k % S;
-                const int64_t u = u0 + k;
-                const bool first = k == 0 || u % p.chunks == 0;
-                const bool last = k == nk - 1 || (u + 1) % p.chunks == 0;
-                if (first && k > 0) ++seg;
-                const uint32_t acc = tmem + static_cast<uint32_t>(seg & 1) * p.tmem_cols;
-                // a buffer is reused two segments later, once its drain has finished
-                if (first && seg >= 2 &&
-                    !mbar_wait(bar(ACC_EMPTY + (seg & 1)), ((seg >> 1) - 1) & 1, abort_flag, p.status))
-                    break;
                 if (!mbar_wait(bar(s), (k / S) & 1, abort_flag, p.status)) break;
                 tc_fence_after();
                 const uint32_t st = base_u32 + s * L.stage_bytes;
@@ -159,47 +154,22 @@ __global__ void __launch_bounds__(THREADS, 1)
                 const uint64_t bd = sdesc_mnmajor_sw128(st + A_BYTES, BMT * 128, 1024);
 #pragma unroll
                 for (int i = 0; i < BMT / 16; ++i)  // 16 tokens per MMA = two 8-row groups
-                    mma_bf16(acc, ad + (2048 >> 4) * i, bd + (2048 >> 4) * i, idesc, !first || i != 0);
+                    mma_bf16(tmem, ad + (2048 >> 4) * i, bd + (2048 >> 4) * i, idesc, (k | i) != 0);
                 tc_commit(bar(S + s));
-                if (last) tc_commit(bar(ACC_FULL + (seg & 1)));
             }
-            tc_commit(bar(FINAL));
+            tc_commit(bar(2 * S));
+            tc_commit(bar(2 * S + 1));
             volatile int no_abort = 0;
-            mbar_wait(bar(FINAL), 0, &no_abort, p.status);
+            mbar_wait(bar(2 * S + 1), 0, &no_abort, p.status);
         }
     } else {
-        // ---------------------------------------------------------------- max + drains
-        const int q = warp & 3;  // the TMEM lane quarter this warp reads: features 32 q ..
-        // a finished segment: its 128 features x NBW sums go to partial slot blockIdx.x + t
-        auto drain = [&](int seg) -> bool {
-            if (!mbar_wait(bar(ACC_FULL + (seg & 1)), (seg >> 1) & 1, abort_flag, p.status)) return false;
-            tc_fence_after();
-            const int64_t slot = static_cast<int64_t>(blockIdx.x) + t_first + seg;
-            float* dst = p.partial + (slot * BF + 32 * q + lane) * p.NBW;
-            const uint32_t acc = tmem + static_cast<uint32_t>(seg & 1) * p.tmem_cols;
-            for (int c = 0; c < p.NBW; c += 32) {
-                uint32_t v[32];
-                tmem_ld_32x32b_x32(acc + (static_cast<uint32_t>(32 * q) << 16) + c, v);
-                tmem_ld_wait();
-#pragma unroll
-                for (int e = 0; e < 32; e += 4)
-                    *reinterpret_cast<float4*>(dst + c + e) =
-                        make_float4(__uint_as_float(v[e]), __uint_as_float(v[e + 1]),
-                                    __uint_as_float(v[e + 2]), __uint_as_float(v[e + 3]));
-            }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar(ACC_EMPTY + (seg & 1)));
-            return true;
-        };
-        float m = 0.0f;
-        const int t = threadIdx.x - 64;  // 0..127
-        int seg = 0;
-        for (int k = 0; k < nk; ++k) {
-            const int64_t u = u0 + k;
-            if (p.amax_out) {
-                // max |x| of each landed P tile (16 KB: 8 x 16 bytes per thread), fp32 fmaxf
-                // as in amax_kernel (a NaN never wins); the stage is released after the read
+        const int q = warp & 3;
+        if (p.amax_out) {
+            // max |x| of each landed P tile (16 KB: 8 x 16 bytes per thread), fp32 fmaxf
+            // as in amax_kernel (a NaN never wins); the stage is released after the read
+            float m = 0.0f;
+            const int t = threadIdx.x - 64;  // 0..127
+            for (int k = 0; k < nk; ++k) {
                 const int s = k % S;
                 if (!mbar_wait(bar(s), (k / S) & 1, abort_flag, p.status)) break;
                 const uint8_t* tile = base + s * L.stage_bytes;
@@ -214,22 +184,30 @@ __global__ void __launch_bounds__(THREADS, 1)
                 __syncwarp();
                 if (lane == 0) mbar_arrive(bar(S + s));
             }
-            if (k == nk - 1 || (u + 1) % p.chunks == 0) {
-                if (!drain(seg)) break;
-                ++seg;
-            }
-        }
-        if (p.amax_out) {
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
             if (lane == 0) atomicMax(p.amax_out, __float_as_uint(m));
+        }
+        if (mbar_wait(bar(2 * S), 0, abort_flag, p.status)) {
+            tc_fence_after();
+            float* dst = p.partial + (static_cast<int64_t>(blockIdx.x) * BF + 32 * q + lane) * p.NBW;
+            for (int c = 0; c < p.NBW; c += 32) {
+                uint32_t v[32];
+                tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(32 * q) << 16) + c, v);
+                tmem_ld_wait();
+#pragma unroll
+                for (int e = 0; e < 32; e += 4)
+                    *reinterpret_cast<float4*>(dst + c + e) =
+                        make_float4(__uint_as_float(v[e]), __uint_as_float(v[e + 1]),
+                                    __uint_as_float(v[e + 2]), __uint_as_float(v[e + 3]));
+            }
         }
     }
 
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (warp == 1) tmem_dealloc(tmem, 2 * p.tmem_cols);
+    if (warp == 1) tmem_dealloc(tmem, p.tmem_cols);
 }
 
 // The split sums in a launch of their own (when the dX GEMM's epilogue warps could not
@@ -242,22 +220,30 @@ __global__ void lora_grad_finalize_kernel(const LoraFinalizeJob j0, const LoraFi
 
 }  // namespace lg
 
-int lora_grad_ctas(int64_t M, int64_t F, int num_sms) {
-    // one persistent CTA per SM (at most kMaxSms, which the workspace query assumes), never
-    // more than there are units
-    if (num_sms > 160) num_sms = 160;
-    const int64_t units = (F / lg::BF) * (M / lg::BMT);
-    return static_cast<int>(units < num_sms ? units : num_sms);
+LoraSchedule lora_grad_schedule(int64_t M, int64_t F, int num_sms) {
+    if (num_sms > 160) num_sms = 160;  // the workspace queries size the slots for at most 160 SMs
+    LoraSchedule sc{};
+    const int T = static_cast<int>(F / lg::BF);
+    const int C = static_cast<int>(M / lg::BMT);
+    sc.full_tiles = (T / num_sms) * num_sms;
+    sc.rem_tiles = T - sc.full_tiles;
+    int s2 = sc.rem_tiles ? num_sms / sc.rem_tiles : 0;
+    if (sc.rem_tiles && s2 < 1) s2 = 1;
+    if (s2 > 16) s2 = 16;
+    if (s2 > C) s2 = C;
+    sc.rem_splits = s2;
+    sc.ctas = sc.full_tiles + sc.rem_tiles * s2;
+    return sc;
 }
 
-cudaError_t launch_lora_grad(const CUtensorMap& tmP, const CUtensorMap& tmV, const LoraGradArgs& a, int ctas,
-                             int kind, cudaStream_t stream) {
+cudaError_t launch_lora_grad(const CUtensorMap& tmP, const CUtensorMap& tmV, const LoraGradArgs& a, int kind,
+                             cudaStream_t stream) {
     const lg::Layout L = lg::layout_for(a.NBW);
     // the opt-in limit is raised once to the device maximum (no per-launch host calls)
     static const cudaError_t attr = cudaFuncSetAttribute(
         lg::lora_grad_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 232448);
     if (attr != cudaSuccess) return attr;
-    dim3 grid(static_cast<unsigned>(ctas));
+    dim3 grid(static_cast<unsigned>(a.full_tiles + a.rem_tiles * a.rem_splits));
     before_launch(kind, stream);
     const cudaError_t le = launch_k(lg::lora_grad_kernel, dim3(grid), dim3(lg::THREADS),
                                     L.smem_bytes, stream, tmP, tmV, a);

@@ -160,28 +160,54 @@ __global__ void build_factors_kernel(const __nv_bfloat16* __restrict__ ls_down,
     const __nv_bfloat16 zero = __float2bfloat16_rn(0.0f);
     // Every piece moves 8 elements (16 bytes) per thread and step: r_s, r, K, N and the
     // padded widths are multiples of 8, so a chunk never straddles two sources.
+    // The row copies issue four independent 16-byte loads before their stores (a thread's
+    // chunks are otherwise one L2 round trip each, one after the other).
     if (dn) {
         const int kc = K / 8;
-        for (int i = t0; i < Rp * kc; i += stride) {
-            const int j = i / kc, k = (i % kc) * 8;
-            uint4 v = make_uint4(0, 0, 0, 0);
-            if (j < r_s) v = *reinterpret_cast<const uint4*>(ls_down + j * K + k);
-            else if (j < R) v = *reinterpret_cast<const uint4*>(lora_a + (j - r_s) * K + k);
-            *reinterpret_cast<uint4*>(dn + j * K + k) = v;
+        const int total = Rp * kc;
+        for (int i0 = t0; i0 < total; i0 += 4 * stride) {
+            uint4 v[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int i = i0 + u * stride;
+                v[u] = make_uint4(0, 0, 0, 0);
+                if (i < total) {
+                    const int j = i / kc, k = (i % kc) * 8;
+                    if (j < r_s) v[u] = *reinterpret_cast<const uint4*>(ls_down + j * K + k);
+                    else if (j < R) v[u] = *reinterpret_cast<const uint4*>(lora_a + (j - r_s) * K + k);
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int i = i0 + u * stride;
+                if (i < total) *reinterpret_cast<uint4*>(dn + (i / kc) * K + (i % kc) * 8) = v[u];
+            }
         }
     }
     if (upcat) {
         const int cc = KL / 8;
-        for (int i = t0; i < N * cc; i += stride) {
-            const int n = i / cc;
-            int c = (i % cc) * 8;
-            uint4 v = make_uint4(0, 0, 0, 0);
-            if (c < 2 * R) {
-                if (c >= R) c -= R;
-                v = c < r_s ? *reinterpret_cast<const uint4*>(ls_up + n * r_s + c)
-                            : *reinterpret_cast<const uint4*>(lora_b + n * r + (c - r_s));
+        const int total = N * cc;
+        for (int i0 = t0; i0 < total; i0 += 4 * stride) {
+            uint4 v[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int i = i0 + u * stride;
+                v[u] = make_uint4(0, 0, 0, 0);
+                if (i < total) {
+                    const int n = i / cc;
+                    int c = (i % cc) * 8;
+                    if (c < 2 * R) {
+                        if (c >= R) c -= R;
+                        v[u] = c < r_s ? *reinterpret_cast<const uint4*>(ls_up + n * r_s + c)
+                                       : *reinterpret_cast<const uint4*>(lora_b + n * r + (c - r_s));
+                    }
+                }
             }
-            *reinterpret_cast<uint4*>(upcat + n * KL + (i % cc) * 8) = v;
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int i = i0 + u * stride;
+                if (i < total) *reinterpret_cast<uint4*>(upcat + (i / cc) * KL + (i % cc) * 8) = v[u];
+            }
         }
     }
     // Transposed pieces: 8 consecutive destination elements per thread (eight gathered

@@ -7,17 +7,15 @@
 namespace ft {
 
 // The adapter gradients' split sums (FourTune, arXiv 2607.05711, section 3.2: dA and dB
-// are the only weight gradients): for output (f, j) of tile t = f / 128, the CTAs p that
-// covered tile t are those whose unit runs [p U / P, (p + 1) U / P) meet
-// [t C, (t + 1) C) (C = chunks, U = (F / 128) C, P = ctas): p_lo .. p_hi below, in token
-// order, each with its slot p + t;
-//   out = s * sum over them, in order, of (D[f][j] + D[f][r + j])
+// are the only weight gradients).  A tile t < full_tiles has one slot (t); a later tile
+// has rem_splits slots, full_tiles + s * rem_tiles + (t - full_tiles) for token range s
+// (LoraSchedule in ft_internal.h).  Then
+//   out = s * sum over the tile's slots, in token order, of (D[f][j] + D[f][r + j])
 // stored as out[f][j], or out[j][f] with transpose_out.  Thread `worker` of `nworkers`
 // takes every nworkers-th block of 4 features x 4 columns of the two jobs (j.out ==
 // nullptr: no job): per slot it issues eight independent 16-byte loads (four features'
-// high and low halves), so an output costs a fraction of an L2 round trip, and it stores
-// 16-byte rows (along j for out[f][j], along f for out[j][f]).  The sums are those of a
-// separate pass bit for bit.
+// high and low halves), and it stores 16-byte rows (along j for out[f][j], along f for
+// out[j][f]).  The sums are those of a separate pass bit for bit.
 __device__ __forceinline__ void lora_split_sums(const LoraFinalizeJob& j0, const LoraFinalizeJob& j1,
                                                 int worker, int nworkers) {
     const int n0 = j0.out ? (j0.F / 4) * (j0.r / 4) : 0;
@@ -36,21 +34,25 @@ __device__ __forceinline__ void lora_split_sums(const LoraFinalizeJob& j0, const
         }
         const int f = 4 * fq, j = 4 * jq;
         const int t = f >> 7;
-        const int64_t P = jb.ctas;
-        const int64_t U = static_cast<int64_t>(jb.F >> 7) * jb.chunks;
-        // the largest p with p U / P <= x is ceil((x + 1) P / U) - 1
-        const int64_t lo_x = static_cast<int64_t>(t) * jb.chunks, hi_x = lo_x + jb.chunks - 1;
-        const int p_lo = static_cast<int>(((lo_x + 1) * P + U - 1) / U - 1);
-        const int p_hi = static_cast<int>(((hi_x + 1) * P + U - 1) / U - 1);
-        const float* d0 = jb.partial + (static_cast<int64_t>(t) * 128 + (f & 127)) * jb.NBW + j;
+        int slot0, nslots, slot_step;
+        if (t < jb.full_tiles) {
+            slot0 = t;
+            nslots = 1;
+            slot_step = 0;
+        } else {
+            slot0 = t;  // full_tiles + 0 * rem_tiles + (t - full_tiles)
+            nslots = jb.rem_splits;
+            slot_step = jb.rem_tiles;
+        }
         const int64_t slot_stride = static_cast<int64_t>(128) * jb.NBW;
+        const float* d0 = jb.partial + (static_cast<int64_t>(slot0) * 128 + (f & 127)) * jb.NBW + j;
         float v[4][4];  // [feature f + a][column j + b]
 #pragma unroll
         for (int a = 0; a < 4; ++a)
 #pragma unroll
             for (int b = 0; b < 4; ++b) v[a][b] = 0.0f;
-        for (int p = p_lo; p <= p_hi; ++p) {
-            const float* d = d0 + static_cast<int64_t>(p) * slot_stride;
+        for (int k = 0; k < nslots; ++k) {
+            const float* d = d0 + static_cast<int64_t>(k) * slot_step * slot_stride;
             float4 h[4], l[4];
 #pragma unroll
             for (int a = 0; a < 4; ++a) {

@@ -206,8 +206,8 @@ def test_given_max_equal_to_the_true_max_gives_the_same_forward():
 
 
 # M = 384 (one-CTA GEMM kernel) with split sums small enough for its epilogue warps
-# ((N + K) r = 36864 outputs; N = 4096: sixteen k steps in the dX GEMM's first tile)
-SIDE_ONE_CTA = wl.LayerSpec(name="side_one_cta_384x512x4096", M=384, K=512, N=4096, r_s=16, r=8, alpha=8.0,
+# ((N + K) r = 69632 outputs; N = 8192: 32 k steps in the dX GEMM's first tile)
+SIDE_ONE_CTA = wl.LayerSpec(name="side_one_cta_384x512x8192", M=384, K=512, N=8192, r_s=16, r=8, alpha=8.0,
                             n_outlier_cols=3, outlier_gain=20.0, w_std=0.02, plant_rank=4, plant_sigma=6.0,
                             b_std=0.01, dy_std=1e-2)
 
