@@ -456,17 +456,21 @@ class LayerRun:
     """One layer of the step: its weights (prepared once, offline), workspace, synthetic
     inputs resident on the device, and outputs."""
 
-    def __init__(self, spec, dev, seed):
+    def __init__(self, spec, dev, seed, weight_spec=None, weight_seed=None):
+        """spec: this rank's shape (its token count M); the frozen weights and the adapter
+        are drawn from weight_spec / weight_seed (the same on every rank: they are
+        replicated), the inputs X and dY from spec / seed."""
         import torch
 
         from diffusion_dit_b200 import fourtune as ft
         from diffusion_dit_b200 import prep, workloads as wl
         self.spec = spec
         inp = wl.make_layer_inputs(spec, seed=seed)
+        wdraw = inp if weight_spec is None else wl.make_layer_inputs(weight_spec, seed=weight_seed)
         self.inp = inp
-        self.split = prep.svd_split(inp.w, spec.r_s)
+        self.split = prep.svd_split(wdraw.w, spec.r_s)
         self.w = ft.prepare_weights(self.split.residual.to(dev), self.split.ls_up.to(dev),
-                                    self.split.ls_down.to(dev), inp.lora_a.to(dev), inp.lora_b.to(dev),
+                                    self.split.ls_down.to(dev), wdraw.lora_a.to(dev), wdraw.lora_b.to(dev),
                                     spec.lora_scale)
         self.w_xp = ft.drop_transposed_codes(self.w)
         M, K, N, R = spec.M, spec.K, spec.N, spec.r_s + spec.r
@@ -594,7 +598,16 @@ def run_layers(args, desc, specs):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
 
     # --- setup (untimed): this rank's synthetic inputs, offline weight prep -------------
-    layers = [LayerRun(s, dev, seed=rank + 17 * i) for i, s in enumerate(specs)]
+    # Weak scaling: every rank a full batch of the workload.  Strong scaling: the ranks
+    # split the workload's batch into token shards (dp.token_shard, multiples of the pair
+    # GEMM's 256 rows).  The frozen weights and the adapter are the same on every rank.
+    import dataclasses
+    rank_specs = specs
+    if args.scaling == "strong" and world > 1:
+        lo, hi = dp.token_shard(specs[0].M, world, rank, multiple=256)
+        rank_specs = [dataclasses.replace(s, M=hi - lo) for s in specs]
+    layers = [LayerRun(rs, dev, seed=1000 + 31 * rank + i, weight_spec=s, weight_seed=17 * i)
+              for i, (rs, s) in enumerate(zip(rank_specs, specs))]
     flush = torch.empty(512 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
 
     def step_kernels(x1x16=False, xpose=False, fwd=True, bwd=True):
@@ -625,6 +638,11 @@ def run_layers(args, desc, specs):
     E = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
     fp4 = sum(L.flops()[0] for L in layers)
     bf = sum(L.flops()[1] for L in layers)
+    # whole-job FLOPs per step: every rank's own batch (weak) or the one global batch (strong)
+    if args.scaling == "strong":
+        job_flops = sum(sum(layer_flops(s.M, s.K, s.N, s.r_s, s.r)) for s in specs)
+    else:
+        job_flops = world * (fp4 + bf)
 
     if args.profile:
         # the plain step, eagerly, for profilers: no graphs, no side measurements
@@ -638,7 +656,7 @@ def run_layers(args, desc, specs):
         ms = s_.elapsed_time(e_) / Kst
         if rank == 0:
             print(json.dumps({"profile": True, "workload": desc, "ms_per_step_eager": ms,
-                              "value_eager": world * (fp4 + bf) / (ms * 1e-3) / 1e12}), flush=True)
+                              "value_eager": job_flops / (ms * 1e-3) / 1e12}), flush=True)
         if world > 1:
             dist.barrier()
             dist.destroy_process_group()
@@ -765,7 +783,7 @@ def run_layers(args, desc, specs):
         dist.all_reduce(tm, op=dist.ReduceOp.MAX)
     total_ms = float(tm.item())
     ms_per_step = total_ms / Kst
-    value = world * (fp4 + bf) * Kst / (total_ms * 1e-3) / 1e12
+    value = job_flops * Kst / (total_ms * 1e-3) / 1e12
 
     # --- end to end through the API: every layer's X and dY copied in from pinned host
     # memory, dA and dB copied out, inside the timed region ----------------------------
@@ -792,7 +810,7 @@ def run_layers(args, desc, specs):
                           device=dev)
     if world > 1:
         dist.all_reduce(e2e_ms, op=dist.ReduceOp.MAX)
-    e2e_value = world * (fp4 + bf) * Kst / (float(e2e_ms.item()) * 1e-3) / 1e12
+    e2e_value = job_flops * Kst / (float(e2e_ms.item()) * 1e-3) / 1e12
     h2d = sum(L.x.numel() * 2 + L.dy.numel() * 2 for L in layers)
     d2h = sum(L.da.numel() * 4 + L.db.numel() * 4 for L in layers)
 
@@ -831,10 +849,12 @@ def run_layers(args, desc, specs):
         fl_b = sum(pass_flops(L.spec.M, L.spec.K, L.spec.N, L.spec.r_s, L.spec.r)[1] for L in layers)
         line = {
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": Kst,
-            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+            "scaling": "strong" if args.scaling == "strong" and world > 1 else "weak",
             "vs_baseline": None, "dtype": "nvfp4(e2m1,ue4m3)+bf16", "data": "synthetic",
             "config": dict(workload_config(args, desc, specs), parallelism=f"dp{world}",
-                           flops_per_step={"fp4": fp4, "bf16": bf}),
+                           M_tokens_per_gpu=layers[0].spec.M,
+                           flops_per_step_per_gpu={"fp4": fp4, "bf16": bf}),
             "roofline": {"bound": "tensor", "kernel": "gemm_fp4_lowrank_pair_kernel (every forward and dX GEMM)",
                          "achieved": achieved, "peak": fp4_peak, "unit": "TFLOP/s",
                          "frac": achieved / fp4_peak, "traffic": gemm_traffic(args.workload),
@@ -899,6 +919,8 @@ def main():
                          "GELU, fused")
     ap.add_argument("--tokens", type=int, default=0, help="replace the token count M (multiple of 256)")
     ap.add_argument("--profile", action="store_true", help="plain eager steps only (for profilers)")
+    ap.add_argument("--scaling", default="weak", choices=["weak", "strong"],
+                    help="N > 1: every rank its own batch (weak, default) or token shards of one batch (strong)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     if args.tokens and args.tokens % 256:

@@ -65,3 +65,15 @@ def test_token_shards_cover_the_batch(m, world):
         assert b == c and (b - a) % 128 == 0
     sizes = [b - a for a, b in spans]
     assert max(sizes) - min(sizes) <= 128
+
+
+@pytest.mark.parametrize("world", [1, 2, 3, 4, 8])
+def test_strong_scaling_shards_of_the_single_stream_batch(world):
+    # bench.py --scaling strong: each rank takes a token shard of the 9216-token batch in
+    # multiples of the pair GEMM's 256 rows, and the shards cover the batch once
+    m = 9216
+    spans = [dp.token_shard(m, world, r, multiple=256) for r in range(world)]
+    assert spans[0][0] == 0 and spans[-1][1] == m
+    for (a, b), (c, d) in zip(spans, spans[1:]):
+        assert b == c
+    assert all((b - a) % 256 == 0 and b > a for a, b in spans)
