@@ -57,7 +57,7 @@ DEFAULT_WORKLOAD = "single"
 # ncu DRAM read + write per launch of the 4-bit GEMM (mean over the step's GEMM launches)
 # on a workload, with the hash of the GEMM's sources the counters were taken from: the
 # figure is reported only while the sources still hash to that value.
-GEMM_DRAM_BYTES = {}
+GEMM_DRAM_BYTES = {"single": (271287232, "6b406da2ee05d402")}
 GEMM_SOURCES = ("ft_gemm2.cu", "ft_ptx.cuh")
 
 
