@@ -83,6 +83,10 @@ __global__ void lowrank_finalize_kernel(const LowRankFinalizeArgs a) {
     }
 }
 
+// Shared tile of the transposed factor pieces: 64 rows of up to 256 + 8 bf16, or up to
+// 256 rows of 64 + 8 (r_s + r <= 256).
+constexpr int kTransposeSmemElems = 256 * 72 > 64 * 264 ? 256 * 72 : 64 * 264;
+
 // Concatenated factors, per call (A and B change every optimizer step):
 //   dn     [Rp, K] = [Ls_down; A; 0]
 //   upcat  [N, KL] = [Up, Up, 0]     with Up = [Ls_up, B]   (forward GEMM B operand)
@@ -147,8 +151,6 @@ __global__ void build_factors_kernel(const __nv_bfloat16* __restrict__ ls_down,
     const int R = r_s + r;
     const int stride = fctas * blockDim.x;
     const int t0 = blockIdx.x * blockDim.x + threadIdx.x;
-    auto dn_at = [&](int j, int k) { return j < r_s ? ls_down[j * K + k] : lora_a[(j - r_s) * K + k]; };
-    auto up_at = [&](int n, int j) { return j < r_s ? ls_up[n * r_s + j] : lora_b[n * r + (j - r_s)]; };
     auto pack8 = [](const __nv_bfloat16 (&e)[8]) {
         uint4 v;
         v.x = static_cast<uint32_t>(__bfloat16_as_ushort(e[0])) | (static_cast<uint32_t>(__bfloat16_as_ushort(e[1])) << 16);
@@ -210,29 +212,56 @@ __global__ void build_factors_kernel(const __nv_bfloat16* __restrict__ ls_down,
             }
         }
     }
-    // Transposed pieces: 8 consecutive destination elements per thread (eight gathered
-    // source elements, one 16-byte store); the sources are small and stay in L2.
-    if (upt) {  // [Rp, N] = [Up^T; 0]
-        const int nc = N / 8;
-        for (int i = t0; i < Rp * nc; i += stride) {
-            const int j = i / nc, n = (i % nc) * 8;
-            __nv_bfloat16 e[8];
-#pragma unroll
-            for (int q = 0; q < 8; ++q) e[q] = j < R ? up_at(n + q, j) : zero;
-            *reinterpret_cast<uint4*>(upt + j * N + n) = pack8(e);
-        }
-    }
-    if (dntcat) {  // [K, KL] = [Dn^T, Dn^T, 0]
-        const int cc = KL / 8;
-        for (int i = t0; i < K * cc; i += stride) {
-            const int k = i / cc, c = (i % cc) * 8;
-            __nv_bfloat16 e[8];
-#pragma unroll
-            for (int q = 0; q < 8; ++q) {
-                const int cq = c + q;
-                e[q] = cq < R ? dn_at(cq, k) : (cq < 2 * R ? dn_at(cq - R, k) : zero);
+    // Transposed pieces, through shared memory in tiles of 64 rows: each tile is read with
+    // 16-byte loads along its source rows and written with 16-byte stores along the
+    // destination rows (a thread gathers its 8 elements from the shared tile), so both
+    // sides stay coalesced.  One tile per CTA and trip; upt's tiles come first.
+    //   upt    [Rp, N] = [Up^T; 0]           from Up [N, R] = [Ls_up | B]
+    //   dntcat [K, KL] = [Dn^T, Dn^T, 0]     from Dn [R, K] = [Ls_down; A]
+    __shared__ __align__(16) __nv_bfloat16 tsm[kTransposeSmemElems];
+    const int upt_tiles = upt ? N / 64 : 0;
+    const int dnt_tiles = dntcat ? K / 64 : 0;
+    for (int tile = blockIdx.x; tile < upt_tiles + dnt_tiles; tile += fctas) {
+        __syncthreads();  // the previous tile's reads of tsm are done
+        if (tile < upt_tiles) {
+            const int n0 = tile * 64;
+            const int ld = R + 8;  // tsm[n][j], padded rows
+            const int rc = R / 8;
+            for (int i = threadIdx.x; i < 64 * rc; i += blockDim.x) {
+                const int n = i / rc, c = (i % rc) * 8;
+                const uint4 v = c < r_s ? *reinterpret_cast<const uint4*>(ls_up + (n0 + n) * r_s + c)
+                                        : *reinterpret_cast<const uint4*>(lora_b + (n0 + n) * r + (c - r_s));
+                *reinterpret_cast<uint4*>(tsm + n * ld + c) = v;
             }
-            *reinterpret_cast<uint4*>(dntcat + k * KL + c) = pack8(e);
+            __syncthreads();
+            for (int i = threadIdx.x; i < Rp * 8; i += blockDim.x) {
+                const int j = i / 8, n = (i % 8) * 8;
+                __nv_bfloat16 e[8];
+#pragma unroll
+                for (int q = 0; q < 8; ++q) e[q] = j < R ? tsm[(n + q) * ld + j] : zero;
+                *reinterpret_cast<uint4*>(upt + j * N + n0 + n) = pack8(e);
+            }
+        } else {
+            const int k0 = (tile - upt_tiles) * 64;
+            const int ld = 64 + 8;  // tsm[j][k], padded rows
+            for (int i = threadIdx.x; i < R * 8; i += blockDim.x) {
+                const int j = i / 8, k = (i % 8) * 8;
+                const uint4 v = j < r_s ? *reinterpret_cast<const uint4*>(ls_down + j * K + k0 + k)
+                                        : *reinterpret_cast<const uint4*>(lora_a + (j - r_s) * K + k0 + k);
+                *reinterpret_cast<uint4*>(tsm + j * ld + k) = v;
+            }
+            __syncthreads();
+            const int cc = KL / 8;
+            for (int i = threadIdx.x; i < 64 * cc; i += blockDim.x) {
+                const int k = i / cc, c = (i % cc) * 8;
+                __nv_bfloat16 e[8];
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                    const int cq = c + q;
+                    e[q] = cq < R ? tsm[cq * ld + k] : (cq < 2 * R ? tsm[(cq - R) * ld + k] : zero);
+                }
+                *reinterpret_cast<uint4*>(dntcat + (k0 + k) * KL + c) = pack8(e);
+            }
         }
     }
     // side jobs: V' = [hi(V), lo(V), 0] for dB (8 columns per thread: one group of hi, of
