@@ -794,13 +794,34 @@ def run_layers(args, desc, specs):
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
+    # The copies in go on a second stream in the order the step needs them (each layer's X
+    # for the forward, then each dY in the backward's layer order) and the step waits for
+    # each just before its first use, so later copies overlap earlier layers' kernels.  A
+    # step's copies start only after the previous step is done with the buffers.
+    copy_stream = torch.cuda.Stream(device=dev)
+    main = torch.cuda.current_stream()
+    need = [(L, "x") for L in layers] + [(L, "dy") for L in reversed(layers)]
+    host = {id(L.x): a for L, a in zip(layers, hx)}
+    host.update({id(L.dy): b for L, b in zip(layers, hdy)})
     for i in range(Kst):
         flush.zero_()
         ev_s[i].record()
-        for L, a, b in zip(layers, hx, hdy):
-            L.x.copy_(a, non_blocking=True)
-            L.dy.copy_(b, non_blocking=True)
-        step()
+        copy_stream.wait_stream(main)
+        ready = {}
+        with torch.cuda.stream(copy_stream):
+            for L, name in need:
+                t = getattr(L, name)
+                t.copy_(host[id(t)], non_blocking=True)
+                ready[(id(L), name)] = torch.cuda.Event()
+                ready[(id(L), name)].record(copy_stream)
+        for L in layers:
+            main.wait_event(ready[(id(L), "x")])
+            L.fwd()
+        for L in reversed(layers):
+            main.wait_event(ready[(id(L), "dy")])
+            L.bwd()
+        if world > 1:
+            allreduce()
         for L, a, b in zip(layers, hda, hdb):
             a.copy_(L.da, non_blocking=True)
             b.copy_(L.db, non_blocking=True)
@@ -885,9 +906,10 @@ def run_layers(args, desc, specs):
                 "dx_gemm_ms_stored_copy": [statistics.mean(r[nL + j] for r in gemm_ms) for j in range(nL)],
                 "bytes_saved": sum(L.spec.N * L.spec.K // 2 + L.spec.N * L.spec.K // 256 for L in layers)},
             "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                    "what": "each step copies every layer's X and dY in from pinned host memory and its dA "
-                            "and dB out; Y and dX stay on the device (in a training step they are the next "
-                            "layer's input and the previous layer's gradient)"},
+                    "what": "each step copies every layer's X and dY in from pinned host memory (on a second "
+                            "stream, each waited for just before its first use, so later copies overlap earlier "
+                            "layers' kernels) and its dA and dB out; Y and dX stay on the device (in a training "
+                            "step they are the next layer's input and the previous layer's gradient)"},
             "gpu_launches": launches,
             "launch_mode": "cuda_graph_replay" if graphs else "stream",
             "clocks": clocks.summary(),
