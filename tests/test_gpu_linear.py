@@ -189,6 +189,23 @@ def test_backward_pair_gemm_with_side_split_sums_matches_oracle():
     test_backward_matches_oracle(SIDE_PAIR, 0)
 
 
+# r = 64 (V' 128 columns wide, as in the FLUX single-stream layers) at sizes the oracle
+# checks in full: the adapter-gradient schedule with token ranges only (8 and 6 tiles,
+# split over up to 8 token ranges), and with whole tiles then split ones (N = 19200:
+# 150 tiles on 148 SMs).
+WIDE_LORA_SPLIT = wl.LayerSpec(name="wide_lora_split_512x1024x768", M=512, K=1024, N=768, r_s=16, r=64,
+                               alpha=64.0, n_outlier_cols=5, outlier_gain=20.0, w_std=0.02, plant_rank=4,
+                               plant_sigma=6.0, b_std=0.01, dy_std=1e-2)
+WIDE_LORA_FULL = wl.LayerSpec(name="wide_lora_full_256x512x19200", M=256, K=512, N=19200, r_s=16, r=64,
+                              alpha=64.0, n_outlier_cols=3, outlier_gain=20.0, w_std=0.02, plant_rank=4,
+                              plant_sigma=6.0, b_std=0.01, dy_std=1e-2)
+
+
+@pytest.mark.parametrize("spec", [WIDE_LORA_SPLIT, WIDE_LORA_FULL], ids=lambda s: s.name)
+def test_backward_rank_64_adapter_gradients(spec):
+    test_backward_matches_oracle(spec, 0)
+
+
 def test_given_max_equal_to_the_true_max_gives_the_same_forward():
     # the prologue's per-CTA maxima (reduced by the quantizer) and a caller's max of the
     # same value are two routes to one g: Y and T must agree bit for bit
