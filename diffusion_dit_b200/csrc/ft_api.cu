@@ -611,6 +611,40 @@ ft_status fourtune_linear_fwd_gelu(const ft_linear* L, const void* x_dev, int64_
 
 namespace {
 
+// An upper bound on the slot loads one thread of `workers` makes in lora_split_sums over
+// the two jobs: thread w takes blocks w, w + workers, ... (job 0's blocks first, then job
+// 1's); a block of tile t adds rem_splits slots when t is a split tile, else one.  Each
+// round of `workers` blocks counts the most slots any of its blocks adds.
+double split_sum_rounds(const ft::LoraFinalizeJob& j0, const ft::LoraFinalizeJob& j1, int64_t workers) {
+    const ft::LoraFinalizeJob* jobs[2] = {&j0, &j1};
+    int64_t n[2];
+    for (int k = 0; k < 2; ++k)
+        n[k] = jobs[k]->out ? static_cast<int64_t>(jobs[k]->F / 4) * (jobs[k]->r / 4) : 0;
+    const int64_t total = n[0] + n[1];
+    double rounds = 0.0;
+    for (int64_t lo = 0; lo < total; lo += workers) {
+        const int64_t hi = std::min(total, lo + workers);  // this round's blocks [lo, hi)
+        int most = 0;
+        for (int k = 0, off = 0; k < 2; off += static_cast<int>(n[k]), ++k) {
+            const int64_t a = std::max<int64_t>(lo, off) - off, b = std::min<int64_t>(hi, off + n[k]) - off;
+            if (a >= b) continue;
+            const ft::LoraFinalizeJob& j = *jobs[k];
+            int slots = 1;
+            if (j.rem_tiles > 0) {
+                if (j.transpose_out) {
+                    slots = j.rem_splits;  // blocks walk f fastest: every round meets a split tile
+                } else {
+                    const int64_t per_tile = 32 * static_cast<int64_t>(j.r / 4);  // blocks of one tile
+                    if ((b - 1) / per_tile >= j.full_tiles) slots = j.rem_splits;
+                }
+            }
+            most = std::max(most, slots);
+        }
+        rounds += most;
+    }
+    return rounds;
+}
+
 // The backward of fourtune_linear_bwd; with gelu_in, dx_dev receives bf16(dX * gelu'(gelu_in)).
 ft_status linear_bwd_impl(const ft_linear* L, const void* x_dev, const float* t_saved_dev, const void* dy_dev,
                           int64_t M, const float* amax_or_null, void* dx_dev, float* da_dev, float* db_dev,
@@ -730,18 +764,23 @@ ft_status linear_bwd_impl(const ft_linear* L, const void* x_dev, const float* t_
         fin[0] = ft::LoraFinalizeJob{g.partial, sc.full_tiles, sc.rem_tiles, sc.rem_splits, static_cast<int>(K), NBW,
                                      L->r, L->lora_scale, true, da_dev};
     }
-    // dA's and dB's split sums: on the dX GEMM's epilogue warps when they fit in about half
-    // the time those warps wait for their first accumulator (a k step of 256 takes ~0.42 us;
-    // a thread's block of 4 x 4 outputs costs ~0.6 us per slot it adds: one round trip for
-    // the slot's eight loads), else in a launch of their own before the GEMM.
+    // dA's and dB's split sums: on the dX GEMM's epilogue warps when they fit in the time
+    // those warps wait for their first accumulator (a k step of 256 takes ~0.42 us; a
+    // thread's block of 4 x 4 outputs costs ~0.6 us per slot it adds: one round trip for
+    // the slot's eight loads), else in a launch of their own before the GEMM.  Measured on
+    // the FLUX single-stream linear2 (15 k steps in the first tile, ~5.4 us of sums): the
+    // side path saves the launch and costs the GEMM ~3 us.
     bool side = false;
     if (L->r > 0) {
-        const double blocks = static_cast<double>(N + K) * L->r / 16.0;
-        const double workers = static_cast<double>(dev.num_sms) * (pair_gemm(M, dev) ? 256.0 : 128.0);
-        const double slots = std::max(fin[0].rem_tiles ? fin[0].rem_splits : 1, fin[1].rem_tiles ? fin[1].rem_splits : 1);
-        const double cost_us = std::ceil(blocks / workers) * slots * 0.6;
+        // the dX GEMM's epilogue threads (32 per epilogue warp: 4 per CTA, 8 with the
+        // GELU-backward epilogue; 148 CTAs, or fewer for a small grid)
+        const bool pair = pair_gemm(M, dev);
+        const int64_t gemm_ctas = pair ? 2 * std::min<int64_t>(dev.num_sms / 2, (M / 256) * (K / 256))
+                                       : std::min<int64_t>(dev.num_sms, (M / 128) * (K / 256));
+        const int64_t workers = gemm_ctas * 32 * (pair && gelu_in ? 8 : 4);
+        const double cost_us = split_sum_rounds(fin[0], fin[1], workers) * 0.6;
         const double first_tile_us = (static_cast<double>(N) / 256.0 + (KL + 63) / 64) * 0.42;
-        side = cost_us <= 0.5 * first_tile_us;
+        side = cost_us <= first_tile_us;
         if (!side) FT_CUDA(ft::launch_lora_grad_finalize(fin[0], fin[1], st));
     }
     // The dX GEMM goes last: the GEMM's operand and output traffic would evict G from L2.

@@ -177,9 +177,10 @@ def test_backward_with_separate_split_sums_matches_oracle():
     test_backward_matches_oracle(WIDE_R, 0)
 
 
-# N = 4096 (16 k steps in the dX GEMM's first tile) with r = 8: the split sums fit on the
-# pair GEMM's epilogue warps before their first accumulator
-SIDE_PAIR = wl.LayerSpec(name="side_pair_256x512x4096", M=256, K=512, N=4096, r_s=16, r=8, alpha=8.0,
+# N = 4096 (17 k steps in the dX GEMM's first tile) with r = 8 and enough GEMM CTAs (M = 1024,
+# K = 2048: 32 pair tiles, 8192 epilogue threads): the split sums fit on the pair GEMM's
+# epilogue warps before their first accumulator
+SIDE_PAIR = wl.LayerSpec(name="side_pair_1024x2048x4096", M=1024, K=2048, N=4096, r_s=16, r=8, alpha=8.0,
                          n_outlier_cols=3, outlier_gain=20.0, w_std=0.02, plant_rank=4, plant_sigma=6.0,
                          b_std=0.01, dy_std=1e-2)
 
