@@ -14,10 +14,12 @@ HBM.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--workload single|qkv|mlp|mlp_up|mlp_down|single_l1|single_l2]
-                    [--tokens M] [--profile]
+                    [--scaling weak|strong] [--tokens M] [--profile]
+                    [--no-cpu-baseline] [--no-quant-sweep]
 
 N > 1 runs data-parallel under torchrun: each rank processes its own batch (weak
-scaling) and the adapter gradients are summed with an NCCL all-reduce.  The reference arm
+scaling), or a token shard of one batch with --scaling strong, and the adapter
+gradients are summed with an NCCL all-reduce.  The reference arm
 times the CPU oracle (the only reference this method has) on a bounded sample of the same
 workload.  --tokens M replaces the token count (a smaller case for profilers);
 --profile runs the plain step only (no graphs, no side measurements), for ncu.  One JSON
