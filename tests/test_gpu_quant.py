@@ -99,6 +99,24 @@ def test_fused_down_projection_of_the_quantizer():
     assert ora.rel_frobenius(t.cpu().double().numpy(), ref) < 1e-5
 
 
+def test_strided_input_matches_oracle():
+    # a column window of a wider matrix (row pitch ld = 576 > cols = 512, base 128 bytes
+    # into each row): the tensor max over the window only, the fused quantizer's TMA box
+    # walk over the pitch, and its down-projection
+    ft = _ft()
+    g = torch.Generator().manual_seed(21)
+    big = (torch.randn(256, 576, generator=g) * 0.5).to(torch.bfloat16)
+    big[:, :64] = 100.0  # outside the window: must not reach the tensor max
+    x = big[:, 64:]
+    down = (torch.randn(32, 512, generator=g) * 0.05).to(torch.bfloat16)
+    q, _, t = ft.quantize_block16(big.cuda()[:, 64:], with_sf=True, down=down.cuda())
+    qo = ora.quantize_block16(x.contiguous())
+    _check_equal(q, qo)
+    assert np.array_equal(q.sf_mma.cpu().numpy(), _sf_mma_expected(qo.scales, 256, 512))
+    ref = x.double().numpy() @ down.double().numpy().T
+    assert ora.rel_frobenius(t.cpu().double().numpy(), ref) < 1e-5
+
+
 @pytest.mark.parametrize("amax_t", [1e-30, 3e-4, 1.0, 250.0, 3e5, 1e30])
 def test_every_bf16_block_max(amax_t):
     # Each 16x16 block is the constant v for one of the 32639 positive finite bf16 values
