@@ -80,7 +80,14 @@ MID = wl.LayerSpec(name="mid_384x1024x768", M=384, K=1024, N=768, r_s=16, r=16, 
                    n_outlier_cols=5, outlier_gain=20.0, w_std=0.02, plant_rank=4, plant_sigma=6.0,
                    b_std=0.01, dy_std=1e-2)
 
-CASES = [(wl.PARITY_SMALL, 0), (wl.PARITY_SMALL, 1), (wl.PARITY_SMALL, 2), (MID, 0)]
+# M = 1408 (11 x 128, not a multiple of 256): the one-CTA GEMM kernel with more tiles than
+# SMs (11 x 16 = 176 forward tiles, 11 x 4 dX tiles of 128 x 256), so CTAs loop over
+# several tiles and the accumulator hand-off runs between them
+ONE_CTA_MANY = wl.LayerSpec(name="one_cta_many_1408x1024x4096", M=1408, K=1024, N=4096, r_s=16, r=16,
+                            alpha=32.0, n_outlier_cols=5, outlier_gain=20.0, w_std=0.02, plant_rank=4,
+                            plant_sigma=6.0, b_std=0.01, dy_std=1e-2)
+
+CASES = [(wl.PARITY_SMALL, 0), (wl.PARITY_SMALL, 1), (wl.PARITY_SMALL, 2), (MID, 0), (ONE_CTA_MANY, 0)]
 IDS = [f"{s.name}-seed{k}" for s, k in CASES]
 
 
